@@ -218,7 +218,8 @@ int oracle_topk(const double* S, const int32_t* nrows, const int32_t* kreq, int 
  *  block == 1 : the set is idx[u, 0:k_b), k_b = min(kreq[b], len_b), entries < 0 skipped;
  *  block  > 1 : idx holds block numbers, k_b = min(kreq[b], ceil(len_b/block)), and
  *               each block contributes its valid rows [beta*block, min(+block, len_b)).
- * O is [B, Hq, d].  Returns 3 if an index is out of range, 4 if a set is empty. */
+ * O is [B, Hq, d]; a head whose set is empty gets O = 0.  Returns 3 if an index is
+ * out of range. */
 int oracle_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V, const int32_t* lens,
                 const int32_t* idx, const int32_t* kreq, int k_max, int block, int B, int Hq,
                 int Hkv, int Ncap, int d, double scale, const int32_t* units, int n_units,
@@ -256,9 +257,9 @@ int oracle_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V, const i
                 for (int j = t0; j < t1; ++j) rows[nr++] = j;
             }
         }
-        if (nr == 0) {
-#pragma omp atomic write
-            err = 4;
+        if (nr == 0) { /* nothing to attend (len_b = 0 or k_b = 0): output 0 by definition */
+            for (int hh = 0; hh < g; ++hh)
+                memset(O + ((size_t)b * Hq + (size_t)kvh * g + hh) * d, 0, sizeof(double) * d);
             free(rows);
             continue;
         }

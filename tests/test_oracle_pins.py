@@ -306,3 +306,12 @@ def test_block_mode_selects_planted_block_and_expands_partial_tail():
     assert idx[0, 0, 0] == 3
     ref = _sdpa_fp64(L.Q, L.K, L.V, L.seq_lens, scale, rows=[list(range(384, 390))])
     np.testing.assert_allclose(O, ref, atol=1e-12, rtol=0)
+
+
+def test_empty_sequence_gives_zero_output_and_no_indices():
+    L = _rand_layer(B=2, Hq=4, Hkv=1, N=16, lens=[16, 0], seed=61)
+    O, idx, _ = oracle.decode_step(L.Q, L.K, L.V, L.seq_lens, [4, 4], 4, 0.2)
+    assert (idx[1] == -1).all() and (O[1] == 0).all()
+    Of, _, _ = oracle.decode_step(L.Q, L.K, L.V, L.seq_lens, None, 0, 0.2, mode=0)
+    assert (Of[1] == 0).all()
+    np.testing.assert_allclose(Of[0], _sdpa_fp64(L.Q[:1], L.K[:1], L.V[:1], [16], 0.2)[0], atol=1e-12)
