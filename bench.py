@@ -1,0 +1,502 @@
+"""Benchmark: top-k context-sparse decode at 128K context and 50x sparsity.
+
+One step = one decode step of the long-context index-reuse workload: layer 0
+scores all 131072 cached keys of each of 8 kv-heads, selects the top 2621 and
+attends over them (32 query heads, GQA 4); layers 1-3 reuse layer 0's indices
+(no scan).  Inputs are synthetic (seeded N(0,1) bf16), resident in HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload reuse128k|llama8b|large_batch|hybrid|tiny]
+
+Prints one JSON line.  `value` = algorithmic HBM bytes of the step (full K scan
+of layer 0 + gathered K/V rows of every layer + Q, O, indices) / device time,
+in TB/s, summed over all ranks (each rank runs its own replica: the units of
+the workload are independent, so ranks share no data).  `--impl reference`
+times the fp64 CPU oracle on the host cores instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = ("decode-step µs & achieved HBM TB/s (score+top-k+sparse attn), 128K ctx, 50×")
+FALLBACK_HBM_GBS = 6650.0
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------- workload model
+
+class Plan:
+    """The layers of one step and their algorithmic bytes."""
+
+    def __init__(self, w, lens):
+        self.w = w
+        self.lens = [int(x) for x in lens]
+        self.kreq = w.k_per_seq(self.lens)
+        self.k_max = max(self.kreq)
+        g = w.Hq // w.Hkv
+        d, blk = w.d, w.block
+        self.kb = []
+        for n, k in zip(self.lens, self.kreq):
+            units = n if blk == 1 else -(-n // blk)
+            self.kb.append(min(k, units))
+        q_o = w.B * w.Hq * d * (2 + 4)
+        idx_b = w.B * w.Hkv * self.k_max * 4
+        gather = 0
+        for n, kb in zip(self.lens, self.kb):
+            rows = kb if blk == 1 else min(kb * blk, n)  # block mode: expanded valid rows (bound)
+            gather += w.Hkv * rows * d * 2 * 2
+        scan = sum(w.Hkv * (n if blk == 1 else -(-n // blk)) * d * (2 if blk == 1 else 4)
+                   for n in self.lens)
+        full = sum(w.Hkv * n * d * 2 * 2 for n in self.lens)
+        self.bytes = {"select": scan + gather + q_o + idx_b, "reuse": gather + q_o + idx_b,
+                      "full": full + q_o, "scan": scan, "gather": gather}
+        self.layer_bytes = [self.bytes[{0: "full", 1: "select", 2: "reuse"}[m]] for m in w.route]
+        self.step_bytes = sum(self.layer_bytes)
+        self.tokens_attended = sum(w.Hq * (kb if blk == 1 else min(kb * blk, n))
+                                   for n, kb in zip(self.lens, self.kb))
+
+
+def make_layers(w, dev, lens):
+    from top_sparse_attention_02_b200 import inputs
+
+    layers, Q = [], None
+    for li in range(w.layers):
+        if w.q_drift > 0 and li > 0:
+            Q = inputs.drift_query(Q, w.q_drift, seed=w.seed + 100 + li)
+        L = inputs.decode_layer(w.B, w.Hq, w.Hkv, w.Ncap, lens, plant_frac=w.plant_frac,
+                                seed=w.seed + li, device=dev, Q=Q if w.q_drift > 0 else None)
+        Q = L.Q
+        layers.append(L)
+    return layers
+
+
+def workload_lens(w):
+    from top_sparse_attention_02_b200 import inputs
+
+    if w.lens is None:
+        return [w.Ncap] * w.B
+    return inputs.draw_lengths(w.B, w.lens[0], w.lens[1], seed=w.seed + 1000).tolist()
+
+
+# ---------------------------------------------------------------- clocks
+
+class Clocks:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        try:  # query the GPU by UUID: CUDA and nvidia-smi may number devices differently
+            u = str(torch.cuda.get_device_properties(gpu_index).uuid)
+            self.idx = u if u.startswith("GPU-") else f"GPU-{u}"
+        except Exception:
+            self.idx = str(gpu_index)
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_dev{gpu_index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, dev):
+    from top_sparse_attention_02_b200 import binding as tsa
+    from top_sparse_attention_02_b200 import workloads
+
+    w = workloads.ALL[args.workload]
+    lens = workload_lens(w)
+    plan = Plan(w, lens)
+    layers = make_layers(w, dev, lens)
+    B, Hq, Hkv, d = w.B, w.Hq, w.Hkv, w.d
+    shape = tsa.shape_of(layers[0].Q, layers[0].K)
+    kreq_t = torch.tensor(plan.kreq, dtype=torch.int32, device=dev)
+    ws_bytes = max(tsa.workspace_size(shape, plan.k_max, w.block, m) for m in set(w.route))
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    tsa.workspace_init(ws)
+    O = [torch.empty(B, Hq, d, dtype=torch.float32, device=dev) for _ in range(w.layers)]
+    idx = [torch.full((B, Hkv, plan.k_max), -1, dtype=torch.int32, device=dev)
+           for _ in range(w.layers)]
+    Kmean = []
+    for li, L in enumerate(layers):
+        if w.block > 1 and w.route[li] == tsa.SELECT:
+            NB = -(-w.Ncap // w.block)
+            km = torch.zeros(B, Hkv, NB, d, dtype=torch.float32, device=dev)
+            tsa.block_summarize(L.K, L.seq_lens, w.block, km, ws, shape=shape)
+            Kmean.append(km)
+        else:
+            Kmean.append(None)
+    step_args = []
+    for li, L in enumerate(layers):
+        mode = w.route[li]
+        src = w.reuse_from[li]
+        step_args.append(tsa.step_args(
+            L.Q, L.K, L.V, L.seq_lens, O[li], ws, mode=mode, scale=w.scale, k_max=plan.k_max,
+            block=w.block, k_per_seq=kreq_t, Kmean=Kmean[li],
+            idx_in=idx[src] if mode == tsa.REUSE else None,
+            idx_out=idx[li] if mode == tsa.SELECT else None))
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for a in step_args:
+            tsa.decode_step(a, stream)
+
+    for _ in range(args.warmup):
+        step()
+    tsa.check_device_status(ws)
+    torch.cuda.synchronize()
+
+    # timed region: K whole steps; inputs (K, V of every layer) exceed L2
+    l0 = tsa.launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with Clocks(torch.cuda.current_device()) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    launches = tsa.launch_count() - l0
+    ms = e0.elapsed_time(e1) / args.steps
+    ms = max_over_ranks(ms, world, dev)
+    tsa.check_device_status(ws)
+
+    # per-stage timing pass: the same layers through the stage entry points, events between
+    stages = stage_times(tsa, w, plan, layers, step_args, Kmean, ws, kreq_t, idx, O, args.steps, stream)
+    copy_gbs = copy_probe(tsa, dev, stream)
+
+    peak, peak_kind = measured_peaks()
+    score_us = stages["score_us"]
+    score_bytes = plan.bytes["scan"]
+    achieved = score_bytes / (score_us * 1e-6) / 1e9
+    res = {
+        "metric": METRIC, "value": world * plan.step_bytes / (ms * 1e-3) / 1e12, "unit": "TB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "us_per_step": ms * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16 Q/K/V, resident in HBM)",
+        "config": {"workload": w.name, "B": B, "Hq": Hq, "Hkv": Hkv, "N": w.Ncap,
+                   "k": plan.k_max, "layers": w.layers,
+                   "route": "".join("FSR"[m] for m in w.route), "block": w.block,
+                   "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (%.2f GB of K/V per step)" %
+                         (sum(L.K.numel() + L.V.numel() for L in layers) * 2 / 1e9)},
+        "algorithmic_bytes_per_step": plan.step_bytes,
+        "tokens_attended_per_s": world * plan.tokens_attended * w.layers / (ms * 1e-3),
+        "stages_us": stages,
+        "roofline": {"kernel": "score_kernel (layer-0 K scan)", "bound": "hbm",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, torch copy)",
+                     "copy_probe_gbs_this_run": copy_gbs, "traffic": None,
+                     "algorithmic_bytes_per_launch": score_bytes},
+        "clocks": clk.summary(),
+        "gpu_launches": launches,
+    }
+    res["e2e"] = e2e_measure(tsa, w, plan, layers, step_args, O, idx, stream, args)
+    return res
+
+
+def stage_times(tsa, w, plan, layers, step_args, Kmean, ws, kreq_t, idx, O, steps, stream):
+    """Average device time of each stage of the step's layers (CUDA events on the stream)."""
+    shape = step_args[0].shape
+    NB = -(-w.Ncap // w.block)
+    rows = w.Ncap if w.block == 1 else NB
+    scores = torch.empty(w.B, w.Hkv, rows, dtype=torch.float32, device=layers[0].Q.device)
+    names = []
+    for li, m in enumerate(w.route):
+        if m == tsa.SELECT:
+            names += [f"L{li}_score", f"L{li}_topk", f"L{li}_attn"]
+        else:
+            names += [f"L{li}_attn"]
+    acc = {n: 0.0 for n in names}
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+    for it in range(steps + 1):
+        j = 0
+        ev[0].record(stream)
+        for li, L in enumerate(layers):
+            m = w.route[li]
+            if m == tsa.SELECT:
+                keys = L.K if w.block == 1 else Kmean[li]
+                tsa.sparse_decode_score(L.Q, keys, L.seq_lens, shape, w.block, w.scale, scores, ws, stream)
+                j += 1
+                ev[j].record(stream)
+                tsa.topk_select(scores, L.seq_lens, kreq_t, plan.k_max, shape, w.block, idx[li], ws, stream)
+                j += 1
+                ev[j].record(stream)
+                tsa.sparse_decode_attn(L.Q, L.K, L.V, L.seq_lens, idx[li], kreq_t, plan.k_max,
+                                       w.block, w.scale, O[li], ws, stream)
+            elif m == tsa.REUSE:
+                tsa.sparse_decode_attn(L.Q, L.K, L.V, L.seq_lens, idx[w.reuse_from[li]], kreq_t,
+                                       plan.k_max, w.block, w.scale, O[li], ws, stream)
+            else:
+                tsa.sparse_decode_attn(L.Q, L.K, L.V, L.seq_lens, None, None, 0, 1, w.scale, O[li],
+                                       ws, stream)
+            j += 1
+            ev[j].record(stream)
+        torch.cuda.synchronize()
+        if it == 0:
+            continue  # warm-up pass
+        for k, n in enumerate(names):
+            acc[n] += ev[k].elapsed_time(ev[k + 1]) * 1e3
+    out = {n: v / steps for n, v in acc.items()}
+    sel = [li for li, m in enumerate(w.route) if m == tsa.SELECT]
+    out["score_us"] = statistics.mean(out[f"L{li}_score"] for li in sel) if sel else float("nan")
+    return out
+
+
+def copy_probe(tsa, dev, stream, nbytes=2 << 30):
+    a = torch.empty(nbytes // 2, dtype=torch.uint8, device=dev)
+    b = torch.empty_like(a)
+    a.fill_(1)
+    best = 0.0
+    for _ in range(6):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        tsa.hbm_copy(a, b, a.numel(), stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        best = max(best, 2 * a.numel() / (e0.elapsed_time(e1) * 1e-3) / 1e9)
+    del a, b
+    return best
+
+
+def e2e_measure(tsa, w, plan, layers, step_args, O, idx, stream, args):
+    """The same step through the C ABI, with every input copied from pinned host memory
+    and the outputs (O of every layer, the selected indices) copied back, all inside the
+    timed region."""
+    host_in = [[t.cpu().pin_memory() for t in (L.Q, L.K, L.V, L.seq_lens)] for L in layers]
+    dev_in = [(L.Q, L.K, L.V, L.seq_lens) for L in layers]
+    O_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in O]
+    sel = [li for li, m in enumerate(w.route) if m == tsa.SELECT]
+    idx_host = [torch.empty(idx[li].shape, dtype=torch.int32).pin_memory() for li in sel]
+    h2d = sum(t.numel() * t.element_size() for hs in host_in for t in hs)
+    d2h = sum(t.numel() * t.element_size() for t in O_host + idx_host)
+    reps = max(1, min(args.steps, 5))
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        for hs, ds in zip(host_in, dev_in):
+            for h, d in zip(hs, ds):
+                d.copy_(h, non_blocking=True)
+        for a in step_args:
+            tsa.decode_step(a, stream)
+        for oh, od in zip(O_host, O):
+            oh.copy_(od, non_blocking=True)
+        for ih, li in zip(idx_host, sel):
+            ih.copy_(idx[li], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    return {"value": plan.step_bytes / (ms * 1e-3) / 1e12, "unit": "TB/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": reps,
+            "note": "Q, K, V and lengths of every layer copied host->device from pinned memory, "
+                    "O and indices copied back, inside the timed region"}
+
+
+# ---------------------------------------------------------------- reference arm (oracle on CPU)
+
+def run_reference(args, w_name, rank, world):
+    import numpy as np
+
+    import oracle
+    from top_sparse_attention_02_b200 import workloads
+
+    w = workloads.ALL[w_name]
+    lens = workload_lens(w)
+    plan = Plan(w, lens)
+    layers = make_layers(w, "cpu", lens)
+    cores = oracle.num_threads()
+    kreq = plan.kreq
+
+    def one_step():
+        idx = {}
+        for li, L in enumerate(layers):
+            m = w.route[li]
+            if m == 2:
+                oracle.decode_step(L.Q, L.K, L.V, L.seq_lens, kreq, plan.k_max, w.scale, mode=2,
+                                   block=w.block, idx_in=idx[w.reuse_from[li]])
+            else:
+                _, ix, _ = oracle.decode_step(L.Q, L.K, L.V, L.seq_lens, kreq, plan.k_max, w.scale,
+                                              mode=m, block=w.block)
+                idx[li] = ix
+
+    for _ in range(min(args.warmup, 1)):
+        one_step()
+    t0 = time.perf_counter()
+    n = 0
+    while n < args.steps:
+        one_step()
+        n += 1
+        if time.perf_counter() - t0 > 60:
+            break
+    s = (time.perf_counter() - t0) / n
+    val = plan.step_bytes / s / 1e12
+    return {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "TB/s", "n_gpus": world,
+        "steps": n, "warmup": args.warmup, "ms_per_step": s * 1e3, "us_per_step": s * 1e6,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) bf16 Q/K/V)",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.Ncap,
+                   "k": plan.k_max, "layers": w.layers, "parallelism": "host cores (OpenMP)"},
+        "cpu_baseline": {"value": val, "unit": "TB/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{n} whole step(s) of the workload (all layers, all units)"},
+        "e2e": {"value": val, "unit": "TB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def cpu_baseline(w_name, budget_s=20.0):
+    """The oracle, as it stands, on a bounded sample of the workload: whole layers of
+    the step until about budget_s of host time; scaled to the metric's unit."""
+    import oracle
+    from top_sparse_attention_02_b200 import workloads
+
+    w = workloads.ALL[w_name]
+    lens = workload_lens(w)
+    plan = Plan(w, lens)
+    layers = make_layers(w, "cpu", lens)
+    t0 = time.perf_counter()
+    done_bytes, nlayers, idx = 0, 0, {}
+    while True:
+        for li, L in enumerate(layers):
+            m = w.route[li]
+            if m == 2:
+                oracle.decode_step(L.Q, L.K, L.V, L.seq_lens, plan.kreq, plan.k_max, w.scale, mode=2,
+                                   block=w.block, idx_in=idx[w.reuse_from[li]])
+            else:
+                _, ix, _ = oracle.decode_step(L.Q, L.K, L.V, L.seq_lens, plan.kreq, plan.k_max,
+                                              w.scale, mode=m, block=w.block)
+                idx[li] = ix
+            done_bytes += plan.layer_bytes[li]
+            nlayers += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    s = time.perf_counter() - t0
+    return {"value": done_bytes / s / 1e12, "unit": "TB/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "seconds": s,
+            "sample": f"{nlayers} layers = {nlayers // w.layers} whole step(s) of the workload "
+                      "(every unit), fp64 C oracle, OpenMP over (seq, kv-head) units"}
+
+
+# ---------------------------------------------------------------- distributed plumbing
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(x, world, dev):
+    if world <= 1:
+        return x
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="reuse128k")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        res = run_reference(args, args.workload, rank, world)
+        print(json.dumps(res), flush=True)
+        return
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    try:
+        res = run_ours(args, rank, world, dev)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline(args.workload)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,177 @@
+/*
+ * tsa.h -- C ABI of libtsa: top-k context-sparse attention at decode, B200 (sm_100a).
+ *
+ * The operation (one decode step of one attention layer, GQA):
+ *   1. score  every cached key against the current query group
+ *             ("inference-time context sparsity: illusion or opportunity?",
+ *             sec. 2, oracle Top-K: the k most important tokens are chosen
+ *             exactly, with no approximate indexer; "Flash Attention vs Sparse
+ *             Attention", DeepSeek Sparse Attention stage 1, the indexer pass);
+ *   2. select the top-k token (or 128-token block) indices per sequence and
+ *             kv-head (same sections);
+ *   3. attend exactly, with softmax, over only the selected K/V rows
+ *             (HyLRA sec. 2.3 hybrid inference: attention limited to the
+ *             subset; DSA stage 2 selective attention), computed as split-K
+ *             flash decoding with an online softmax ("Flash Attention vs Sparse
+ *             Attention", tiling + online softmax).
+ * A layer may instead reuse the previous layer's indices (HyLRA sec. 2.1/2.3
+ * tolerant layers; IndexCache in "Flash Attention vs Sparse Attention") or run
+ * full attention (Flux Attention sec. 1/3 hard per-layer routing; HyLRA
+ * sensitive layers).  Block mode scores 128-token blocks by q . (block-mean key)
+ * (HyLRA sec. 2.4, block-level sparsity).
+ *
+ * Conventions (every entry point):
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    never allocates, never frees and never synchronises (except
+ *    tsa_check_device_status).  Work is enqueued on `stream` (a cudaStream_t;
+ *    NULL = the legacy default stream) and runs asynchronously.
+ *  - Shapes: Q [B, Hq, d] bf16; K, V [B, Hkv, Ncap, d] bf16 (row-major,
+ *    contiguous); seq_lens [B] int32 with 0 <= len_b <= Ncap; d must be 128;
+ *    Hq must be g * Hkv with g in {1, 2, 4, 8}.  Kv-head kvh serves query heads
+ *    kvh*g .. kvh*g+g-1.  Q, K, V, Kmean, O must be 16-byte aligned.
+ *  - "Unit" = (b, kvh).  In token mode a unit has n_b = len_b rows; in block
+ *    mode (block > 1) it has n_b = ceil(len_b / block) blocks.
+ *  - k_per_seq [B] int32 (device) or NULL (= k_max for every sequence);
+ *    k_b = min(k_per_seq[b], n_b) and must not exceed k_max.
+ *  - idx [B, Hkv, k_max] int32: the k_b selected rows (or blocks) in ascending
+ *    order, then -1.
+ *  - scale must be finite and > 0 (scores are stored scaled).
+ *  - Errors: an argument error returns a status before anything is enqueued
+ *    (tsa_last_error_string() says which).  A failed launch returns
+ *    TSA_ERR_CUDA.  Errors only the device can see (a len_b above Ncap, a k_b
+ *    above k_max, an index out of range) skip the offending work, never fault,
+ *    and set a flag in the first 256 bytes of `ws`, read by
+ *    tsa_check_device_status.  No C++ exception crosses this boundary.
+ *  - Workspace: `ws` is caller-owned device memory of at least
+ *    tsa_workspace_size(...) bytes, 256-byte aligned, set to zero once with
+ *    tsa_workspace_init before first use.  Calls that share a workspace must be
+ *    ordered on one stream; calls that overlap on the GPU with the same `ws` race.
+ */
+#ifndef TSA_H
+#define TSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    TSA_OK = 0,
+    TSA_ERR_INVALID_ARG = 1,   /* bad pointer, size, alignment or value */
+    TSA_ERR_UNSUPPORTED = 2,   /* valid but not implemented (d != 128, g not in {1,2,4,8}) */
+    TSA_ERR_WORKSPACE = 3,     /* ws NULL or smaller than tsa_workspace_size() */
+    TSA_ERR_CUDA = 4,          /* a CUDA launch or query failed */
+    TSA_ERR_DEVICE_BOUNDS = 5, /* device saw a length / k / index out of range */
+    TSA_ERR_DEVICE_TIMEOUT = 6 /* a bounded device-side wait gave up */
+} tsa_status;
+
+typedef enum { TSA_FULL = 0, TSA_SELECT = 1, TSA_REUSE = 2 } tsa_mode;
+
+typedef struct {
+    int32_t B;    /* sequences in the batch */
+    int32_t Hq;   /* query heads */
+    int32_t Hkv;  /* kv heads (Hq = g * Hkv) */
+    int32_t Ncap; /* cache capacity in tokens (rows of K and V per unit) */
+    int32_t d;    /* head dimension (must be 128) */
+} tsa_shape;
+
+/* ------------------------------------------------------------------ sizing */
+
+/* Bytes of workspace that tsa_decode_step needs for (shape, k_max, block, mode);
+ * enough for every other entry point called with the same arguments.  Returns 0
+ * on invalid arguments (see tsa_last_error_string). */
+size_t tsa_workspace_size(tsa_shape shape, int32_t k_max, int32_t block, int32_t mode);
+
+/* Zero a workspace (enqueued memset).  Call once after allocating it. */
+tsa_status tsa_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------ stages */
+
+/* Block summaries for block mode (HyLRA sec. 2.4): Kmean[b,kvh,beta,:] = fp32
+ * mean of the valid K rows [beta*block, min(beta*block+block, len_b)).  Kmean is
+ * [B, Hkv, ceil(Ncap/block), d] fp32; blocks past ceil(len_b/block) are not
+ * written.  Run when the cache is appended to, outside the decode step. */
+tsa_status tsa_block_summarize(const void* K, const int32_t* seq_lens, tsa_shape shape,
+                               int32_t block, float* Kmean, void* ws, size_t ws_bytes,
+                               void* stream);
+
+/* Step 1, score (oracle Top-K criterion; DSA indexer pass):
+ *   scores[b,kvh,j] = max over the group's heads h of scale * <q_h, key_j>,
+ * bf16 products accumulated in fp32.  block == 1: keys = K (bf16, rows Ncap);
+ * block > 1: keys = Kmean (fp32, rows ceil(Ncap/block)).  scores is
+ * [B, Hkv, rows] fp32; only rows j < n_b are written. */
+tsa_status sparse_decode_score(const void* Q, const void* keys, const int32_t* seq_lens,
+                               tsa_shape shape, int32_t block, float scale, float* scores,
+                               void* ws, size_t ws_bytes, void* stream);
+
+/* Step 2, exact top-k per unit over scores [B, Hkv, rows] (rows as in
+ * sparse_decode_score): the k_b largest, ties to the lower index, written to
+ * idx in ascending order and padded with -1 (oracle Top-K, exact selection). */
+tsa_status topk_select(const float* scores, const int32_t* seq_lens, const int32_t* k_per_seq,
+                       int32_t k_max, tsa_shape shape, int32_t block, int32_t* idx, void* ws,
+                       size_t ws_bytes, void* stream);
+
+/* Step 3, exact softmax attention over the selected rows (selective attention;
+ * split-K flash decoding with an online softmax, then a combine of the splits).
+ *   idx == NULL : every valid row [0, len_b) (a full-attention layer);
+ *   block == 1  : rows idx[b,kvh,0:k_b] (entries < 0 skipped);
+ *   block  > 1  : idx holds block numbers; each expands to its valid rows.
+ * O is [B, Hq, d] fp32; a head with no attended row gets O = 0.
+ * Index reuse (HyLRA tolerant layers, IndexCache) is this call with a previous
+ * layer's idx and no score/select. */
+tsa_status sparse_decode_attn(const void* Q, const void* K, const void* V,
+                              const int32_t* seq_lens, const int32_t* idx,
+                              const int32_t* k_per_seq, int32_t k_max, int32_t block,
+                              tsa_shape shape, float scale, float* O, void* ws, size_t ws_bytes,
+                              void* stream);
+
+/* ------------------------------------------------------------------ one step */
+
+typedef struct {
+    tsa_shape shape;          /* as for the stage calls */
+    const void* Q;            /* [B, Hq, d] bf16 */
+    const void* K;            /* [B, Hkv, Ncap, d] bf16 */
+    const void* V;            /* [B, Hkv, Ncap, d] bf16 */
+    const float* Kmean;       /* block mode SELECT only: output of tsa_block_summarize */
+    const int32_t* seq_lens;  /* [B] */
+    const int32_t* k_per_seq; /* [B] or NULL (= k_max) */
+    int32_t k_max;            /* columns of idx; ignored for TSA_FULL */
+    int32_t block;            /* 1 = token mode, > 1 = block mode (128 in the pages) */
+    int32_t mode;             /* TSA_FULL, TSA_SELECT or TSA_REUSE */
+    float scale;              /* softmax scale, > 0 (1/sqrt(d) usually) */
+    const int32_t* idx_in;    /* TSA_REUSE: the earlier layer's idx [B, Hkv, k_max] */
+    int32_t* idx_out;         /* TSA_SELECT: this layer's idx [B, Hkv, k_max] */
+    float* O;                 /* [B, Hq, d] fp32 */
+    void* ws;                 /* workspace */
+    size_t ws_bytes;
+} tsa_step_args;
+
+/* One decode step of one layer: TSA_SELECT = score -> top-k -> attention;
+ * TSA_REUSE = attention over idx_in; TSA_FULL = attention over every valid row. */
+tsa_status tsa_decode_step(const tsa_step_args* args, void* stream);
+
+/* ------------------------------------------------------------------ status */
+
+/* Wait for `stream`, then read and clear the device error flag in `ws`:
+ * TSA_OK, TSA_ERR_DEVICE_BOUNDS or TSA_ERR_DEVICE_TIMEOUT (or TSA_ERR_CUDA). */
+tsa_status tsa_check_device_status(void* ws, void* stream);
+
+/* Text of the last error on this thread ("" if none). */
+const char* tsa_last_error_string(void);
+
+/* Kernels this library has launched in this process (all entry points). */
+uint64_t tsa_launch_count(void);
+
+/* ------------------------------------------------------------------ measurement */
+
+/* HBM roofline probe: dst[0:bytes] = src[0:bytes] with 16-byte vector loads
+ * and stores over a grid sized to the SM count.  bytes must be a multiple of 16. */
+tsa_status tsa_hbm_copy(const void* src, void* dst, size_t bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TSA_H */

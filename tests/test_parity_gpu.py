@@ -1,0 +1,265 @@
+"""GPU vs oracle parity, stage by stage and for whole decode steps (needs a B200)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity import check_output, compare_idx, sub_problem
+from top_sparse_attention_02_b200 import binding as tsa
+from top_sparse_attention_02_b200 import inputs
+
+import gpu_run as G
+
+pytestmark = pytest.mark.gpu
+SCALE = 1 / math.sqrt(128)
+
+
+def layer(B, Hq, Hkv, N, lens=None, seed=0, plant=0.01, tail_fill=None):
+    lens = lens if lens is not None else [N] * B
+    return inputs.decode_layer(B, Hq, Hkv, N, lens, plant_frac=plant, seed=seed, tail_fill=tail_fill)
+
+
+# ------------------------------------------------------------------ score stage
+
+@pytest.mark.parametrize("Hq,Hkv,N,lens", [(8, 2, 4096, None), (32, 8, 1000, [1000, 999, 1, 0]),
+                                           (8, 8, 333, None), (16, 8, 2048, [2048, 77]),
+                                           (64, 8, 777, None)])
+def test_score_stage(cuda_dev, Hq, Hkv, N, lens):
+    B = len(lens) if lens else 1
+    L = layer(B, Hq, Hkv, N, lens, seed=3, tail_fill=float("nan"))
+    Q, K, V, ln = G.to_dev(L, cuda_dev)
+    S = G.run_score(Q, K, ln, SCALE).cpu().numpy()
+    ref = oracle.scores(L.Q, L.K, L.seq_lens, SCALE)
+    for b in range(B):
+        n = int(L.seq_lens[b])
+        # fp32 sum of 128 exact bf16 products vs fp64: |err| <= 128 * 2^-24 * sum|terms|
+        np.testing.assert_allclose(S[b, :, :n], ref[b, :, :n], rtol=2e-5, atol=2e-5)
+        assert np.isnan(S[b, :, n:]).all(), "rows past len_b were written"
+
+
+# ------------------------------------------------------------------ top-k stage (bit-exact)
+
+def _topk_case(dev, S_np, lens, kreq, k_max, Hq=8, block=1, Ncap=None):
+    S = torch.from_numpy(S_np.astype(np.float32)).to(dev)
+    B, Hkv, rows = S.shape
+    lens_t = torch.tensor(lens, dtype=torch.int32, device=dev)
+    Ncap = Ncap or rows
+    got = G.run_topk(S, lens_t, kreq, k_max, Hq if Hq % Hkv == 0 else Hkv, Ncap, block).cpu().numpy()
+    nrows = lens if block == 1 else [-(-x // block) for x in lens]
+    want = oracle.topk(S_np.astype(np.float32).astype(np.float64), nrows,
+                       kreq if kreq is not None else [k_max] * B, k_max)
+    np.testing.assert_array_equal(got, want)
+
+
+@pytest.mark.parametrize("rows", [1, 31, 100, 4096, 16385, 40000, 131072])
+def test_topk_exact_random(cuda_dev, rows):
+    rng = np.random.default_rng(rows)
+    B, Hkv = 2, 2
+    S = rng.standard_normal((B, Hkv, rows))
+    lens = [rows, max(rows // 3, 1)]
+    for k in sorted({1, 2, min(rows, 17), max(rows // 50, 1), max(rows - 1, 1), rows, rows + 5}):
+        _topk_case(cuda_dev, S, lens, [k, k], k, Hq=Hkv * 4)
+
+
+def test_topk_ties_signed_zeros_and_duplicates(cuda_dev):
+    rng = np.random.default_rng(7)
+    rows = 20000
+    S = rng.integers(-4, 5, size=(1, 2, rows)).astype(np.float64) * 0.5  # heavy exact ties
+    S[0, 0, ::7] = -0.0
+    S[0, 1] = 0.0  # every score tied: lowest indices win
+    S[0, 1, 5::11] = -0.0
+    for k in (1, 10, 1234, 19999):
+        _topk_case(cuda_dev, S, [rows], [k], k, Hq=8)
+    S2 = -np.abs(rng.standard_normal((1, 2, 5000))) - 1.0  # all negative
+    _topk_case(cuda_dev, S2, [5000], [100], 100)
+
+
+def test_topk_ragged_per_sequence_k(cuda_dev):
+    rng = np.random.default_rng(11)
+    B, Hkv, rows = 6, 3, 9000
+    S = rng.standard_normal((B, Hkv, rows))
+    lens = [9000, 8192, 1, 0, 4097, 333]
+    kreq = [180, 17, 5, 3, 4097, 0]
+    _topk_case(cuda_dev, S, lens, kreq, 4097, Hq=Hkv * 2)
+
+
+# ------------------------------------------------------------------ attention stage
+
+def _rand_idx(rng, B, Hkv, lens, k_max, kb):
+    idx = np.full((B, Hkv, k_max), -1, dtype=np.int32)
+    for b in range(B):
+        for h in range(Hkv):
+            n = min(kb[b], lens[b])
+            idx[b, h, :n] = np.sort(rng.choice(lens[b], size=n, replace=False))
+    return idx
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(8, 2), (32, 8), (8, 8), (64, 8), (4, 2)])
+def test_attn_stage_random_sets(cuda_dev, Hq, Hkv):
+    rng = np.random.default_rng(Hq * 10 + Hkv)
+    lens = [3000, 1, 700]
+    L = layer(3, Hq, Hkv, 3000, lens, seed=5, tail_fill=float("nan"))
+    Q, K, V, ln = G.to_dev(L, cuda_dev)
+    kb = [611, 1, 700]
+    idx = _rand_idx(rng, 3, Hkv, lens, 700, kb)
+    O, _ = G.run_attn(Q, K, V, ln, torch.from_numpy(idx).to(cuda_dev), kb, 700, 1, SCALE)
+    ref = oracle.attn(L.Q, L.K, L.V, L.seq_lens, idx, kb, 700, 1, SCALE)
+    check_output(O.cpu().numpy(), ref, "random sets")
+
+
+def test_attn_stage_sliding_window_and_padding(cuda_dev):
+    lens = [500, 64]
+    L = layer(2, 8, 2, 512, lens, seed=9, tail_fill=float("nan"))
+    Q, K, V, ln = G.to_dev(L, cuda_dev)
+    idx = np.full((2, 2, 64), -1, dtype=np.int32)
+    idx[0, :, :64] = np.arange(436, 500)  # the last 64 tokens (a sliding window)
+    idx[1, :, :10] = np.arange(54, 64)
+    idx[1, 1, 3] = -1  # a skipped entry inside the list
+    kb = [64, 64]
+    O, _ = G.run_attn(Q, K, V, ln, torch.from_numpy(idx).to(cuda_dev), kb, 64, 1, SCALE)
+    ref = oracle.attn(L.Q, L.K, L.V, L.seq_lens, idx, kb, 64, 1, SCALE)
+    check_output(O.cpu().numpy(), ref, "window")
+
+
+@pytest.mark.parametrize("lens", [[5000, 1], [128, 129], [0, 77]])
+def test_attn_dense_mode(cuda_dev, lens):
+    L = layer(len(lens), 32, 8, 5000, lens, seed=13, tail_fill=float("nan"))
+    Q, K, V, ln = G.to_dev(L, cuda_dev)
+    O, _ = G.run_attn(Q, K, V, ln, None, None, 0, 1, SCALE)
+    ref = oracle.attn(L.Q, L.K, L.V, L.seq_lens, None, None, 0, 1, SCALE)
+    check_output(O.cpu().numpy(), ref, "dense")
+
+
+def test_attn_block_mode_expansion(cuda_dev):
+    lens = [1000, 130]
+    L = layer(2, 8, 2, 1024, lens, seed=17, tail_fill=float("nan"))
+    Q, K, V, ln = G.to_dev(L, cuda_dev)
+    idx = np.full((2, 2, 4), -1, dtype=np.int32)
+    idx[0, 0, :3] = [0, 5, 7]  # block 7 is the partial last block (rows 896..999)
+    idx[0, 1, :4] = [1, 2, 3, 4]
+    idx[1, 0, :2] = [0, 1]  # block 1 holds 2 valid rows
+    idx[1, 1, :1] = [1]
+    kb = [4, 2]
+    O, _ = G.run_attn(Q, K, V, ln, torch.from_numpy(idx).to(cuda_dev), kb, 4, 128, SCALE)
+    ref = oracle.attn(L.Q, L.K, L.V, L.seq_lens, idx, kb, 4, 128, SCALE)
+    check_output(O.cpu().numpy(), ref, "block expansion")
+
+
+# ------------------------------------------------------------------ block summaries
+
+def test_block_summarize(cuda_dev):
+    lens = [1000, 128, 5]
+    L = layer(3, 8, 2, 1024, lens, seed=19, tail_fill=float("nan"))
+    Q, K, V, ln = G.to_dev(L, cuda_dev)
+    M = G.block_means(K, ln, 128).cpu().numpy()
+    ref = oracle.block_means(L.K, L.seq_lens, 128)
+    for b, n in enumerate(lens):
+        nb = -(-n // 128)
+        np.testing.assert_allclose(M[b, :, :nb], ref[b, :, :nb], rtol=0, atol=2e-6)
+
+
+# ------------------------------------------------------------------ whole steps
+
+def _select_and_check(dev, L, kreq, k_max, block=1, units=None):
+    Q, K, V, ln = G.to_dev(L, dev)
+    Kmean = G.block_means(K, ln, block) if block > 1 else None
+    O, idx = G.step(Q, K, V, ln, mode=tsa.SELECT, scale=SCALE, k_max=k_max, block=block, kreq=kreq,
+                    Kmean=Kmean)
+    idx_np = idx.cpu().numpy()
+    if block == 1:
+        S = oracle.scores(L.Q, L.K, L.seq_lens, SCALE)
+        nrows = L.seq_lens.numpy()
+    else:
+        nrows = oracle.nblocks_of(L.seq_lens, block)
+        S = oracle.block_scores(L.Q, oracle.block_means(L.K, L.seq_lens, block), nrows, SCALE)
+    counts = compare_idx(idx_np, S, nrows, kreq)
+    ref = oracle.attn(L.Q, L.K, L.V, L.seq_lens, idx_np, kreq, k_max, block, SCALE)
+    check_output(O.cpu().numpy(), ref, "select step")
+    return counts, idx, O, (Q, K, V, ln)
+
+
+def test_tiny_workload_end_to_end(cuda_dev):
+    """B=1, 8/2 heads, N=4096, k=128, 1% planted keys, seed 0: the small workload."""
+    L = layer(1, 8, 2, 4096, seed=0, plant=0.01)
+    counts, idx, O, _ = _select_and_check(cuda_dev, L, [128], 128)
+    assert counts["exact"] + counts["near_tie"] == 2
+    # the planted heavy keys are found (a property of the data, not of the kernel)
+    for kvh in range(2):
+        planted = set(L.planted[kvh].tolist())
+        got = set(idx[0, kvh].cpu().numpy().tolist())
+        assert len(planted & got) >= 0.9 * len(planted)
+
+
+@pytest.mark.parametrize("case", ["ragged", "k_gt_len", "k_eq_len", "k1", "equal_keys", "len_lt_128"])
+def test_select_step_edge_cases(cuda_dev, case):
+    if case == "ragged":
+        L, kreq, k_max = layer(4, 32, 8, 3000, [3000, 1, 129, 0], seed=21, tail_fill=float("nan")), \
+            [60, 60, 60, 60], 60
+    elif case == "k_gt_len":
+        L, kreq, k_max = layer(2, 8, 2, 256, [100, 256], seed=22), [150, 150], 150
+    elif case == "k_eq_len":
+        L, kreq, k_max = layer(1, 8, 2, 300, [300], seed=23), [300], 300
+    elif case == "k1":
+        L, kreq, k_max = layer(2, 16, 2, 2000, [2000, 1500], seed=24), [1, 1], 1
+    elif case == "equal_keys":
+        L = layer(1, 8, 2, 1000, seed=25)
+        L.K[0, :, :] = L.K[0, :, :1]
+        kreq, k_max = [40], 40
+    else:
+        L, kreq, k_max = layer(3, 8, 2, 127, [127, 100, 5], seed=26, tail_fill=float("nan")), \
+            [12, 12, 12], 12
+    counts, idx, O, _ = _select_and_check(cuda_dev, L, kreq, k_max)
+    if case == "equal_keys":
+        assert (idx[0, :, :40].cpu().numpy() == np.arange(40)).all()
+
+
+def test_block_mode_step(cuda_dev):
+    L = layer(2, 32, 8, 9000, [9000, 4100], seed=27, plant=0.01)
+    counts, idx, O, _ = _select_and_check(cuda_dev, L, [32, 32], 32, block=128)
+    assert counts["exact"] + counts["near_tie"] == 16
+
+
+def test_reuse_and_full_steps(cuda_dev):
+    L0 = layer(2, 32, 8, 6000, [6000, 3001], seed=29)
+    counts, idx, O, _ = _select_and_check(cuda_dev, L0, [120, 120], 120)
+    L1 = inputs.decode_layer(2, 32, 8, 6000, [6000, 3001], seed=30, Q=inputs.drift_query(L0.Q, 0.3, 31))
+    Q, K, V, ln = G.to_dev(L1, cuda_dev)
+    before = idx.clone()
+    O1, _ = G.step(Q, K, V, ln, mode=tsa.REUSE, scale=SCALE, k_max=120, kreq=[120, 120], idx_in=idx)
+    assert torch.equal(before, idx), "reuse must not touch the indices"
+    ref = oracle.attn(L1.Q, L1.K, L1.V, L1.seq_lens, idx.cpu().numpy(), [120, 120], 120, 1, SCALE)
+    check_output(O1.cpu().numpy(), ref, "reuse")
+    O2, _ = G.step(Q, K, V, ln, mode=tsa.FULL, scale=SCALE)
+    ref2 = oracle.attn(L1.Q, L1.K, L1.V, L1.seq_lens, None, None, 0, 1, SCALE)
+    check_output(O2.cpu().numpy(), ref2, "full")
+
+
+def test_select_is_deterministic(cuda_dev):
+    L = layer(4, 32, 8, 20000, seed=33)
+    Q, K, V, ln = G.to_dev(L, cuda_dev)
+    a = G.step(Q, K, V, ln, mode=tsa.SELECT, scale=SCALE, k_max=400)
+    b = G.step(Q, K, V, ln, mode=tsa.SELECT, scale=SCALE, k_max=400)
+    assert torch.equal(a[1], b[1])
+    assert torch.equal(a[0].view(torch.int32), b[0].view(torch.int32))
+
+
+# ------------------------------------------------------------------ device-side errors
+
+def test_device_bounds_flag_and_recovery(cuda_dev):
+    L = layer(2, 8, 2, 512, seed=35)
+    Q, K, V, ln = G.to_dev(L, cuda_dev)
+    bad = torch.tensor([512, 600], dtype=torch.int32, device=cuda_dev)  # 600 > Ncap
+    with pytest.raises(tsa.TsaError) as e:
+        G.step(Q, K, V, bad, mode=tsa.SELECT, scale=SCALE, k_max=8)
+    assert e.value.status == tsa.TSA_ERR_DEVICE_BOUNDS
+    idx = torch.full((2, 2, 4), -1, dtype=torch.int32, device=cuda_dev)
+    idx[0, 0, 0] = 700  # row past len_b
+    O, ws = G.run_attn(Q, K, V, ln, idx, [4, 4], 4, 1, SCALE, check=False)
+    with pytest.raises(tsa.TsaError) as e:
+        tsa.check_device_status(ws)
+    assert e.value.status == tsa.TSA_ERR_DEVICE_BOUNDS
+    tsa.check_device_status(ws)  # the flag was cleared by the read
+    O, _ = G.step(Q, K, V, ln, mode=tsa.SELECT, scale=SCALE, k_max=8)  # the context still works
+    assert torch.isfinite(O).all()

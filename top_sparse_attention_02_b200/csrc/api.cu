@@ -1,0 +1,281 @@
+// api.cu -- the C ABI of libtsa (declared in include/tsa.h): argument checks,
+// workspace layout and stream-ordered launches.  No allocation, no
+// synchronisation (except tsa_check_device_status), no exceptions.
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+
+#include "launch.h"
+#include "tsa.h"
+
+namespace tsa {
+static std::atomic<uint64_t> g_launches{0};
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+}  // namespace tsa
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+tsa_status fail(tsa_status st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+tsa_status cuda_fail(cudaError_t e, const char* where) {
+    return fail(TSA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+tsa_status check_shape(const tsa_shape& s, tsa::Dims* d) {
+    if (s.B < 0 || s.Hq <= 0 || s.Hkv <= 0 || s.Ncap < 0)
+        return fail(TSA_ERR_INVALID_ARG, "shape: need B >= 0, Hq > 0, Hkv > 0, Ncap >= 0 (got B=%d Hq=%d Hkv=%d Ncap=%d)",
+                    s.B, s.Hq, s.Hkv, s.Ncap);
+    if (s.d != tsa::kDHead) return fail(TSA_ERR_UNSUPPORTED, "shape: head dimension must be 128 (got %d)", s.d);
+    if (s.Hq % s.Hkv != 0) return fail(TSA_ERR_INVALID_ARG, "shape: Hq=%d is not a multiple of Hkv=%d", s.Hq, s.Hkv);
+    const int G = s.Hq / s.Hkv;
+    if (G != 1 && G != 2 && G != 4 && G != 8)
+        return fail(TSA_ERR_UNSUPPORTED, "shape: GQA group Hq/Hkv=%d not in {1,2,4,8}", G);
+    if ((long long)s.B * s.Hkv > 65535)
+        return fail(TSA_ERR_UNSUPPORTED, "shape: B*Hkv=%lld above 65535", (long long)s.B * s.Hkv);
+    d->B = s.B;
+    d->Hq = s.Hq;
+    d->Hkv = s.Hkv;
+    d->Ncap = s.Ncap;
+    d->G = G;
+    return TSA_OK;
+}
+
+tsa_status check_block(int block) {
+    if (block < 1 || block > 4096) return fail(TSA_ERR_INVALID_ARG, "block must be in [1, 4096] (got %d)", block);
+    return TSA_OK;
+}
+
+tsa_status check_scale(float scale) {
+    if (!std::isfinite(scale) || !(scale > 0.f))
+        return fail(TSA_ERR_INVALID_ARG, "scale must be finite and > 0 (got %g)", (double)scale);
+    return TSA_OK;
+}
+
+size_t a256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+constexpr size_t kFlagBytes = 256;
+
+// Workspace: [flag 256 B][split counters][split partials][scores (SELECT only)]
+struct Layout {
+    size_t counters = 0, partials = 0, scores = 0, total = kFlagBytes;
+    int splits = 0;
+};
+
+Layout layout(const tsa::Dims& d, int k_max, int block, bool attn, bool dense, bool scores) {
+    Layout L;
+    size_t off = kFlagBytes;
+    if (attn) {
+        L.splits = tsa::attn_splits(d, k_max, block, dense);
+        L.counters = off;
+        off += a256((size_t)d.units() * sizeof(unsigned));
+        L.partials = off;
+        off += a256(tsa::attn_partials_floats(d, L.splits) * sizeof(float));
+    }
+    if (scores) {
+        L.scores = off;
+        off += a256((size_t)d.units() * tsa::rows_cap_of(d, block) * sizeof(float));
+    }
+    L.total = off;
+    return L;
+}
+
+tsa_status check_ws(const void* ws, size_t ws_bytes, size_t need) {
+    if (ws == nullptr) return fail(TSA_ERR_WORKSPACE, "workspace pointer is NULL");
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(TSA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+    if (ws_bytes < need) return fail(TSA_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, need);
+    return TSA_OK;
+}
+
+unsigned* flag_of(void* ws) { return static_cast<unsigned*>(ws); }
+
+tsa_status check_kmax(int k_max) {
+    if (k_max < 0) return fail(TSA_ERR_INVALID_ARG, "k_max must be >= 0 (got %d)", k_max);
+    return TSA_OK;
+}
+
+}  // namespace
+
+#define TSA_TRY(x)                       \
+    do {                                 \
+        tsa_status _st = (x);            \
+        if (_st != TSA_OK) return _st;   \
+    } while (0)
+
+extern "C" {
+
+size_t tsa_workspace_size(tsa_shape shape, int32_t k_max, int32_t block, int32_t mode) {
+    tsa::Dims d;
+    if (check_shape(shape, &d) != TSA_OK || check_block(block) != TSA_OK || check_kmax(k_max) != TSA_OK) return 0;
+    switch (mode) {
+        case TSA_FULL: return layout(d, 0, 1, true, true, false).total;
+        case TSA_SELECT: return layout(d, k_max, block, true, false, true).total;
+        case TSA_REUSE: return layout(d, k_max, block, true, false, false).total;
+        default:
+            fail(TSA_ERR_INVALID_ARG, "unknown mode %d", mode);
+            return 0;
+    }
+}
+
+tsa_status tsa_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+    TSA_TRY(check_ws(ws, ws_bytes, kFlagBytes));
+    cudaError_t e = cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "tsa_workspace_init");
+    return TSA_OK;
+}
+
+tsa_status tsa_block_summarize(const void* K, const int32_t* seq_lens, tsa_shape shape,
+                               int32_t block, float* Kmean, void* ws, size_t ws_bytes,
+                               void* stream) {
+    tsa::Dims d;
+    TSA_TRY(check_shape(shape, &d));
+    TSA_TRY(check_block(block));
+    if (!K || !seq_lens || !Kmean) return fail(TSA_ERR_INVALID_ARG, "tsa_block_summarize: NULL pointer");
+    if (!aligned16(K) || !aligned16(Kmean)) return fail(TSA_ERR_INVALID_ARG, "tsa_block_summarize: K and Kmean must be 16-byte aligned");
+    TSA_TRY(check_ws(ws, ws_bytes, kFlagBytes));
+    cudaError_t e = tsa::launch_block_summarize(K, seq_lens, d, block, Kmean, flag_of(ws),
+                                                static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "tsa_block_summarize");
+    return TSA_OK;
+}
+
+tsa_status sparse_decode_score(const void* Q, const void* keys, const int32_t* seq_lens,
+                               tsa_shape shape, int32_t block, float scale, float* scores,
+                               void* ws, size_t ws_bytes, void* stream) {
+    tsa::Dims d;
+    TSA_TRY(check_shape(shape, &d));
+    TSA_TRY(check_block(block));
+    TSA_TRY(check_scale(scale));
+    if (!Q || !keys || !seq_lens || !scores) return fail(TSA_ERR_INVALID_ARG, "sparse_decode_score: NULL pointer");
+    if (!aligned16(Q) || !aligned16(keys)) return fail(TSA_ERR_INVALID_ARG, "sparse_decode_score: Q and keys must be 16-byte aligned");
+    TSA_TRY(check_ws(ws, ws_bytes, kFlagBytes));
+    cudaError_t e = tsa::launch_score(Q, keys, seq_lens, d, block, scale, scores, flag_of(ws),
+                                      static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "sparse_decode_score");
+    return TSA_OK;
+}
+
+tsa_status topk_select(const float* scores, const int32_t* seq_lens, const int32_t* k_per_seq,
+                       int32_t k_max, tsa_shape shape, int32_t block, int32_t* idx, void* ws,
+                       size_t ws_bytes, void* stream) {
+    tsa::Dims d;
+    TSA_TRY(check_shape(shape, &d));
+    TSA_TRY(check_block(block));
+    TSA_TRY(check_kmax(k_max));
+    if (!scores || !seq_lens || !idx) return fail(TSA_ERR_INVALID_ARG, "topk_select: NULL pointer");
+    int C, chunk;
+    if (!tsa::topk_plan(tsa::rows_cap_of(d, block), &C, &chunk))
+        return fail(TSA_ERR_UNSUPPORTED, "topk_select: %d rows per unit exceed the cluster capacity", tsa::rows_cap_of(d, block));
+    TSA_TRY(check_ws(ws, ws_bytes, kFlagBytes));
+    cudaError_t e = tsa::launch_topk(scores, seq_lens, k_per_seq, k_max, d, block, idx,
+                                     flag_of(ws), static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "topk_select");
+    return TSA_OK;
+}
+
+tsa_status sparse_decode_attn(const void* Q, const void* K, const void* V,
+                              const int32_t* seq_lens, const int32_t* idx,
+                              const int32_t* k_per_seq, int32_t k_max, int32_t block,
+                              tsa_shape shape, float scale, float* O, void* ws, size_t ws_bytes,
+                              void* stream) {
+    tsa::Dims d;
+    TSA_TRY(check_shape(shape, &d));
+    TSA_TRY(check_block(block));
+    TSA_TRY(check_scale(scale));
+    TSA_TRY(check_kmax(k_max));
+    if (!Q || !K || !V || !seq_lens || !O) return fail(TSA_ERR_INVALID_ARG, "sparse_decode_attn: NULL pointer");
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
+        return fail(TSA_ERR_INVALID_ARG, "sparse_decode_attn: Q, K, V and O must be 16-byte aligned");
+    const bool dense = idx == nullptr;
+    if (!dense && k_max == 0) return fail(TSA_ERR_INVALID_ARG, "sparse_decode_attn: k_max must be > 0 with an index list");
+    const Layout L = layout(d, dense ? 0 : k_max, dense ? 1 : block, true, dense, false);
+    TSA_TRY(check_ws(ws, ws_bytes, L.total));
+    char* w = static_cast<char*>(ws);
+    cudaError_t e = tsa::launch_attn(Q, K, V, seq_lens, idx, k_per_seq, k_max, dense ? 1 : block, d,
+                                     scale, L.splits, reinterpret_cast<float*>(w + L.partials),
+                                     reinterpret_cast<unsigned*>(w + L.counters), O, flag_of(ws),
+                                     static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "sparse_decode_attn");
+    return TSA_OK;
+}
+
+tsa_status tsa_decode_step(const tsa_step_args* a, void* stream) {
+    if (!a) return fail(TSA_ERR_INVALID_ARG, "tsa_decode_step: NULL args");
+    tsa::Dims d;
+    TSA_TRY(check_shape(a->shape, &d));
+    switch (a->mode) {
+        case TSA_FULL:
+            return sparse_decode_attn(a->Q, a->K, a->V, a->seq_lens, nullptr, nullptr, 0, 1, a->shape,
+                                      a->scale, a->O, a->ws, a->ws_bytes, stream);
+        case TSA_REUSE:
+            if (!a->idx_in) return fail(TSA_ERR_INVALID_ARG, "tsa_decode_step: TSA_REUSE needs idx_in");
+            return sparse_decode_attn(a->Q, a->K, a->V, a->seq_lens, a->idx_in, a->k_per_seq, a->k_max,
+                                      a->block, a->shape, a->scale, a->O, a->ws, a->ws_bytes, stream);
+        case TSA_SELECT: {
+            TSA_TRY(check_block(a->block));
+            TSA_TRY(check_scale(a->scale));
+            TSA_TRY(check_kmax(a->k_max));
+            if (a->k_max == 0) return fail(TSA_ERR_INVALID_ARG, "tsa_decode_step: TSA_SELECT needs k_max > 0");
+            if (!a->idx_out) return fail(TSA_ERR_INVALID_ARG, "tsa_decode_step: TSA_SELECT needs idx_out");
+            if (a->block > 1 && !a->Kmean) return fail(TSA_ERR_INVALID_ARG, "tsa_decode_step: block mode needs Kmean");
+            if (!a->Q || !a->K || !a->V || !a->seq_lens || !a->O) return fail(TSA_ERR_INVALID_ARG, "tsa_decode_step: NULL pointer");
+            if (!aligned16(a->Q) || !aligned16(a->K) || !aligned16(a->V) || !aligned16(a->O) ||
+                (a->block > 1 && !aligned16(a->Kmean)))
+                return fail(TSA_ERR_INVALID_ARG, "tsa_decode_step: Q, K, V, Kmean and O must be 16-byte aligned");
+            int C, chunk;
+            if (!tsa::topk_plan(tsa::rows_cap_of(d, a->block), &C, &chunk))
+                return fail(TSA_ERR_UNSUPPORTED, "tsa_decode_step: %d rows per unit exceed the top-k cluster capacity",
+                            tsa::rows_cap_of(d, a->block));
+            const Layout L = layout(d, a->k_max, a->block, true, false, true);
+            TSA_TRY(check_ws(a->ws, a->ws_bytes, L.total));
+            float* scores = reinterpret_cast<float*>(static_cast<char*>(a->ws) + L.scores);
+            const void* keys = a->block == 1 ? a->K : static_cast<const void*>(a->Kmean);
+            TSA_TRY(sparse_decode_score(a->Q, keys, a->seq_lens, a->shape, a->block, a->scale, scores,
+                                        a->ws, a->ws_bytes, stream));
+            TSA_TRY(topk_select(scores, a->seq_lens, a->k_per_seq, a->k_max, a->shape, a->block,
+                                a->idx_out, a->ws, a->ws_bytes, stream));
+            return sparse_decode_attn(a->Q, a->K, a->V, a->seq_lens, a->idx_out, a->k_per_seq, a->k_max,
+                                      a->block, a->shape, a->scale, a->O, a->ws, a->ws_bytes, stream);
+        }
+        default:
+            return fail(TSA_ERR_INVALID_ARG, "tsa_decode_step: unknown mode %d", a->mode);
+    }
+}
+
+tsa_status tsa_check_device_status(void* ws, void* stream) {
+    if (!ws) return fail(TSA_ERR_INVALID_ARG, "tsa_check_device_status: NULL workspace");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    unsigned h = 0;
+    cudaError_t e = cudaMemcpyAsync(&h, ws, sizeof h, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ws, 0, sizeof h, st);
+    if (e != cudaSuccess) return cuda_fail(e, "tsa_check_device_status");
+    if (h & tsa::kFlagTimeoutBit) return fail(TSA_ERR_DEVICE_TIMEOUT, "a bounded device-side wait gave up");
+    if (h & tsa::kFlagBoundsBit) return fail(TSA_ERR_DEVICE_BOUNDS, "device saw a length, k or index out of range");
+    return TSA_OK;
+}
+
+const char* tsa_last_error_string(void) { return g_err; }
+
+uint64_t tsa_launch_count(void) { return tsa::g_launches.load(std::memory_order_relaxed); }
+
+tsa_status tsa_hbm_copy(const void* src, void* dst, size_t bytes, void* stream) {
+    if (!src || !dst) return fail(TSA_ERR_INVALID_ARG, "tsa_hbm_copy: NULL pointer");
+    if (!aligned16(src) || !aligned16(dst) || bytes % 16 != 0)
+        return fail(TSA_ERR_INVALID_ARG, "tsa_hbm_copy: pointers and size must be multiples of 16 bytes");
+    cudaError_t e = tsa::launch_copy(src, dst, bytes, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "tsa_hbm_copy");
+    return TSA_OK;
+}
+
+}  // extern "C"

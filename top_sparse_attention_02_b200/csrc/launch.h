@@ -1,0 +1,46 @@
+// launch.h -- host-side launchers of the libtsa kernels (internal to the library).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace tsa {
+
+constexpr int kDHead = 128;              // the only head dimension supported
+constexpr unsigned kFlagBoundsBit = 1u;  // device flag: length / k / index out of range
+constexpr unsigned kFlagTimeoutBit = 2u; // device flag: a bounded wait gave up
+
+struct Dims {
+    int B, Hq, Hkv, Ncap, G;  // G = Hq / Hkv
+    int units() const { return B * Hkv; }
+};
+
+// rows a unit's key table has: Ncap tokens, or ceil(Ncap/block) block means
+inline int rows_cap_of(const Dims& d, int block) { return block == 1 ? d.Ncap : (d.Ncap + block - 1) / block; }
+
+void note_launch();
+
+cudaError_t launch_block_summarize(const void* K, const int32_t* lens, const Dims& d, int block,
+                                   float* Kmean, unsigned* flag, cudaStream_t st);
+
+cudaError_t launch_score(const void* Q, const void* keys, const int32_t* lens, const Dims& d,
+                         int block, float scale, float* scores, unsigned* flag, cudaStream_t st);
+
+// top-k plan: cluster size and keys per CTA for a row count; false if too large
+bool topk_plan(int rows_cap, int* cluster, int* chunk);
+cudaError_t launch_topk(const float* scores, const int32_t* lens, const int32_t* kreq, int k_max,
+                        const Dims& d, int block, int32_t* idx, unsigned* flag, cudaStream_t st);
+
+// split-K plan for the attention stage (a pure function of the arguments, so
+// that workspace sizing and launch agree)
+int attn_splits(const Dims& d, int k_max, int block, bool dense);
+size_t attn_partials_floats(const Dims& d, int splits);
+cudaError_t launch_attn(const void* Q, const void* K, const void* V, const int32_t* lens,
+                        const int32_t* idx, const int32_t* kreq, int k_max, int block,
+                        const Dims& d, float scale, int splits, float* partials,
+                        unsigned* counters, float* O, unsigned* flag, cudaStream_t st);
+
+cudaError_t launch_copy(const void* src, void* dst, size_t bytes, cudaStream_t st);
+
+}  // namespace tsa
