@@ -185,11 +185,6 @@ def test_tiny_workload_end_to_end(cuda_dev):
     L = layer(1, 8, 2, 4096, seed=0, plant=0.01)
     counts, idx, O, _ = _select_and_check(cuda_dev, L, [128], 128)
     assert counts["exact"] + counts["near_tie"] == 2
-    # the planted heavy keys are found (a property of the data, not of the kernel)
-    for kvh in range(2):
-        planted = set(L.planted[kvh].tolist())
-        got = set(idx[0, kvh].cpu().numpy().tolist())
-        assert len(planted & got) >= 0.9 * len(planted)
 
 
 @pytest.mark.parametrize("case", ["ragged", "k_gt_len", "k_eq_len", "k1", "equal_keys", "len_lt_128"])

@@ -45,7 +45,8 @@ def _check_attn_units(L, idx, O, kreq, k_max, units, scale, block=1):
     g = L.Q.shape[1] // L.K.shape[1]
     sp = sub_problem(L.Q, L.K, L.V, L.seq_lens, units, kreq=kreq)
     gi = None if idx is None else gather_units(idx.cpu().numpy(), units, L.K.shape[1])
-    ref = oracle.attn(sp["Q"], sp["K"], sp["V"], sp["seq_lens"], gi, sp["kreq"], k_max, block, scale)
+    ref = oracle.attn(sp["Q"], sp["K"], sp["V"], sp["seq_lens"], gi, sp.get("kreq"), k_max, block,
+                      scale)
     check_output(gather_units(O.cpu().numpy(), units, L.K.shape[1], g), ref, "attn")
 
 
