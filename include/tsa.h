@@ -127,6 +127,34 @@ tsa_status sparse_decode_attn(const void* Q, const void* K, const void* V,
                               tsa_shape shape, float scale, float* O, void* ws, size_t ws_bytes,
                               void* stream);
 
+/* Step 3 without a workspace.  The pages have no counterpart to this entry
+ * point: it exists for callers that cannot allocate device memory for a
+ * workspace (a plugin host that passes an operator only its inputs and outputs,
+ * a runtime whose device memory all belongs to another allocator, a serving loop
+ * that must not call cudaMalloc or cudaFree, which can block or synchronise the
+ * device).  Same arguments, meaning and result as sparse_decode_attn, minus
+ * ws/ws_bytes.  Its scratch (split counters and split partials) is a fixed
+ * 8 MiB device array inside the library, which every GPU that loads the library
+ * holds until the process exits.  It allocates nothing (no cudaMalloc, cudaFree
+ * or allocating library routine).
+ *  - The first call on a device looks up that array's device address (with that
+ *    device current) and caches it; later calls reuse it.
+ *  - Every call clears the counters it needs, then launches: all calls share the
+ *    one array, so calls that overlap on the GPU (different streams, or other
+ *    host threads, on the same device) race and must be ordered by the caller.
+ *  - A shape whose scratch exceeds 8 MiB returns TSA_ERR_WORKSPACE with the
+ *    bytes it needs (use sparse_decode_attn with a workspace instead).  The
+ *    array holds about 16000 split partials of 520 bytes (one per unit, split
+ *    and query head); the 128K-token shape (8 units, 74 splits, 4 heads) uses
+ *    1.2 MB of it.
+ *  - Device-detected range errors skip the offending rows as in
+ *    sparse_decode_attn, but are not reported: the flag lives in the shared
+ *    array and is cleared by the next call. */
+tsa_status sparse_decode_attn_noalloc(const void* Q, const void* K, const void* V,
+                                      const int32_t* seq_lens, const int32_t* idx,
+                                      const int32_t* k_per_seq, int32_t k_max, int32_t block,
+                                      tsa_shape shape, float scale, float* O, void* stream);
+
 /* ------------------------------------------------------------------ one step */
 
 typedef struct {

@@ -48,6 +48,8 @@ _SIGS = {
     "topk_select": (ctypes.c_int, [_vp, _vp, _vp, _i32, tsa_shape, _i32, _vp, _vp, _sz, _vp]),
     "sparse_decode_attn": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, tsa_shape, _f32,
                                           _vp, _vp, _sz, _vp]),
+    "sparse_decode_attn_noalloc": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, tsa_shape,
+                                                  _f32, _vp, _vp]),
     "tsa_decode_step": (ctypes.c_int, [ctypes.POINTER(tsa_step_args), _vp]),
     "tsa_check_device_status": (ctypes.c_int, [_vp, _vp]),
     "tsa_last_error_string": (ctypes.c_char_p, []),
@@ -148,6 +150,16 @@ def sparse_decode_attn(Q, K, V, seq_lens, idx, k_per_seq, k_max: int, block: int
     _ok(_lib.sparse_decode_attn(_ptr(Q), _ptr(K), _ptr(V), _ptr(seq_lens), _ptr(idx),
                                 _ptr(k_per_seq), k_max, block, s, scale, _ptr(O), *_wsargs(ws),
                                 _stream(stream)))
+
+
+def sparse_decode_attn_noalloc(Q, K, V, seq_lens, idx, k_per_seq, k_max: int, block: int,
+                               scale: float, O, stream=None, shape=None):
+    """sparse_decode_attn with the library's fixed internal scratch instead of a workspace
+    (for callers that cannot allocate one); calls on one device must not overlap."""
+    s = shape or shape_of(Q, K)
+    _ok(_lib.sparse_decode_attn_noalloc(_ptr(Q), _ptr(K), _ptr(V), _ptr(seq_lens), _ptr(idx),
+                                        _ptr(k_per_seq), k_max, block, s, scale, _ptr(O),
+                                        _stream(stream)))
 
 
 def step_args(Q, K, V, seq_lens, O, ws, *, mode: int, scale: float, k_max: int = 0, block: int = 1,

@@ -26,6 +26,14 @@ tsa_status fail(tsa_status st, const char* fmt, ...) {
     return st;
 }
 
+}  // namespace
+
+namespace tsa {
+void set_error_message(const char* msg) { snprintf(g_err, sizeof g_err, "%s", msg); }
+}  // namespace tsa
+
+namespace {
+
 tsa_status cuda_fail(cudaError_t e, const char* where) {
     return fail(TSA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
 }

@@ -21,6 +21,9 @@ inline int rows_cap_of(const Dims& d, int block) { return block == 1 ? d.Ncap : 
 
 void note_launch();
 
+// set the text tsa_last_error_string() returns on this thread
+void set_error_message(const char* msg);
+
 cudaError_t launch_block_summarize(const void* K, const int32_t* lens, const Dims& d, int block,
                                    float* Kmean, unsigned* flag, cudaStream_t st);
 
