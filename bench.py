@@ -193,36 +193,51 @@ def run_ours(args, rank, world, dev):
             block=w.block, k_per_seq=kreq_t, Kmean=Kmean[li],
             idx_in=idx[src] if mode == tsa.REUSE else None,
             idx_out=idx[li] if mode == tsa.SELECT else None))
-    stream = torch.cuda.current_stream()
+    # The step is captured once into a CUDA graph (the library never allocates or
+    # synchronises, so its calls capture cleanly) and replayed: the timing is
+    # device time, not Python/ctypes launch overhead.
+    stream = torch.cuda.Stream(device=dev)
 
     def step():
         for a in step_args:
             tsa.decode_step(a, stream)
 
-    for _ in range(args.warmup):
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    stream.synchronize()
+    tsa.check_device_status(ws, stream)
+    l0 = tsa.launch_count()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
         step()
-    tsa.check_device_status(ws)
-    torch.cuda.synchronize()
+    launches_per_step = tsa.launch_count() - l0
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            graph.replay()
+    stream.synchronize()
+    tsa.check_device_status(ws, stream)
 
     # timed region: K whole steps; inputs (K, V of every layer) exceed L2
-    l0 = tsa.launch_count()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
     with Clocks(torch.cuda.current_device()) as clk:
-        e0.record(stream)
-        for _ in range(args.steps):
-            step()
-        e1.record(stream)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(args.steps):
+                graph.replay()
+            e1.record(stream)
         torch.cuda.synchronize()
     barrier(world)
-    launches = tsa.launch_count() - l0
+    launches = launches_per_step * args.steps
     ms = e0.elapsed_time(e1) / args.steps
     ms = max_over_ranks(ms, world, dev)
-    tsa.check_device_status(ws)
+    tsa.check_device_status(ws, stream)
+    del graph
 
-    # per-stage timing pass: the same layers through the stage entry points, events between
-    stages = stage_times(tsa, w, plan, layers, step_args, Kmean, ws, kreq_t, idx, O, args.steps, stream)
+    # per-stage device times: each stage alone, repeated in its own graph
+    stages = stage_times(tsa, w, plan, layers, Kmean, ws, kreq_t, idx, O, stream)
     copy_gbs = copy_probe(tsa, dev, stream)
 
     peak, peak_kind = measured_peaks()
@@ -250,56 +265,61 @@ def run_ours(args, rank, world, dev):
                      "algorithmic_bytes_per_launch": score_bytes},
         "clocks": clk.summary(),
         "gpu_launches": launches,
+        "timing": "CUDA graph of one whole step, replayed K times between CUDA events",
     }
     res["e2e"] = e2e_measure(tsa, w, plan, layers, step_args, O, idx, stream, args)
     return res
 
 
-def stage_times(tsa, w, plan, layers, step_args, Kmean, ws, kreq_t, idx, O, steps, stream):
-    """Average device time of each stage of the step's layers (CUDA events on the stream)."""
-    shape = step_args[0].shape
+def stage_times(tsa, w, plan, layers, Kmean, ws, kreq_t, idx, O, stream, reps=10):
+    """Average device time of each stage, each launched `reps` times back to back in a
+    CUDA graph.  The score stage streams more than L2 per launch; the top-k and the
+    attention stages read L2-sized data, so their repeated launches run L2-warm."""
+    from top_sparse_attention_02_b200 import binding as _b
+
+    shape = _b.shape_of(layers[0].Q, layers[0].K)
     NB = -(-w.Ncap // w.block)
     rows = w.Ncap if w.block == 1 else NB
     scores = torch.empty(w.B, w.Hkv, rows, dtype=torch.float32, device=layers[0].Q.device)
-    names = []
-    for li, m in enumerate(w.route):
+    calls = {}
+    for li, L in enumerate(layers):
+        m = w.route[li]
         if m == tsa.SELECT:
-            names += [f"L{li}_score", f"L{li}_topk", f"L{li}_attn"]
+            keys = L.K if w.block == 1 else Kmean[li]
+            calls[f"L{li}_score"] = lambda L=L, keys=keys: tsa.sparse_decode_score(
+                L.Q, keys, L.seq_lens, shape, w.block, w.scale, scores, ws, stream)
+            calls[f"L{li}_topk"] = lambda L=L, li=li: tsa.topk_select(
+                scores, L.seq_lens, kreq_t, plan.k_max, shape, w.block, idx[li], ws, stream)
+            calls[f"L{li}_attn"] = lambda L=L, li=li: tsa.sparse_decode_attn(
+                L.Q, L.K, L.V, L.seq_lens, idx[li], kreq_t, plan.k_max, w.block, w.scale, O[li], ws, stream)
+        elif m == tsa.REUSE:
+            calls[f"L{li}_attn"] = lambda L=L, li=li: tsa.sparse_decode_attn(
+                L.Q, L.K, L.V, L.seq_lens, idx[w.reuse_from[li]], kreq_t, plan.k_max, w.block, w.scale,
+                O[li], ws, stream)
         else:
-            names += [f"L{li}_attn"]
-    acc = {n: 0.0 for n in names}
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
-    for it in range(steps + 1):
-        j = 0
-        ev[0].record(stream)
-        for li, L in enumerate(layers):
-            m = w.route[li]
-            if m == tsa.SELECT:
-                keys = L.K if w.block == 1 else Kmean[li]
-                tsa.sparse_decode_score(L.Q, keys, L.seq_lens, shape, w.block, w.scale, scores, ws, stream)
-                j += 1
-                ev[j].record(stream)
-                tsa.topk_select(scores, L.seq_lens, kreq_t, plan.k_max, shape, w.block, idx[li], ws, stream)
-                j += 1
-                ev[j].record(stream)
-                tsa.sparse_decode_attn(L.Q, L.K, L.V, L.seq_lens, idx[li], kreq_t, plan.k_max,
-                                       w.block, w.scale, O[li], ws, stream)
-            elif m == tsa.REUSE:
-                tsa.sparse_decode_attn(L.Q, L.K, L.V, L.seq_lens, idx[w.reuse_from[li]], kreq_t,
-                                       plan.k_max, w.block, w.scale, O[li], ws, stream)
-            else:
-                tsa.sparse_decode_attn(L.Q, L.K, L.V, L.seq_lens, None, None, 0, 1, w.scale, O[li],
-                                       ws, stream)
-            j += 1
-            ev[j].record(stream)
-        torch.cuda.synchronize()
-        if it == 0:
-            continue  # warm-up pass
-        for k, n in enumerate(names):
-            acc[n] += ev[k].elapsed_time(ev[k + 1]) * 1e3
-    out = {n: v / steps for n, v in acc.items()}
+            calls[f"L{li}_attn"] = lambda L=L, li=li: tsa.sparse_decode_attn(
+                L.Q, L.K, L.V, L.seq_lens, None, None, 0, 1, w.scale, O[li], ws, stream)
+    out = {}
+    for name, fn in calls.items():
+        with torch.cuda.stream(stream):
+            fn()
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for _ in range(reps):
+                fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            g.replay()
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+        stream.synchronize()
+        out[name] = e0.elapsed_time(e1) * 1e3 / reps
+        del g
     sel = [li for li, m in enumerate(w.route) if m == tsa.SELECT]
     out["score_us"] = statistics.mean(out[f"L{li}_score"] for li in sel) if sel else float("nan")
+    out["note"] = "each stage alone, %d launches back to back in a CUDA graph" % reps
     return out
 
 
@@ -333,18 +353,19 @@ def e2e_measure(tsa, w, plan, layers, step_args, O, idx, stream, args):
     reps = max(1, min(args.steps, 5))
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(reps):
-        for hs, ds in zip(host_in, dev_in):
-            for h, d in zip(hs, ds):
-                d.copy_(h, non_blocking=True)
-        for a in step_args:
-            tsa.decode_step(a, stream)
-        for oh, od in zip(O_host, O):
-            oh.copy_(od, non_blocking=True)
-        for ih, li in zip(idx_host, sel):
-            ih.copy_(idx[li], non_blocking=True)
-    e1.record(stream)
+    with torch.cuda.stream(stream):  # copies and kernels in one stream order
+        e0.record(stream)
+        for _ in range(reps):
+            for hs, ds in zip(host_in, dev_in):
+                for h, d in zip(hs, ds):
+                    d.copy_(h, non_blocking=True)
+            for a in step_args:
+                tsa.decode_step(a, stream)
+            for oh, od in zip(O_host, O):
+                oh.copy_(od, non_blocking=True)
+            for ih, li in zip(idx_host, sel):
+                ih.copy_(idx[li], non_blocking=True)
+        e1.record(stream)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / reps
     return {"value": plan.step_bytes / (ms * 1e-3) / 1e12, "unit": "TB/s", "ms_per_step": ms,

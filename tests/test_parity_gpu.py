@@ -258,3 +258,21 @@ def test_device_bounds_flag_and_recovery(cuda_dev):
     tsa.check_device_status(ws)  # the flag was cleared by the read
     O, _ = G.step(Q, K, V, ln, mode=tsa.SELECT, scale=SCALE, k_max=8)  # the context still works
     assert torch.isfinite(O).all()
+
+
+@pytest.mark.parametrize("dense", [True, False])
+def test_attn_many_splits_workspace_combine(cuda_dev, dense):
+    """Few units with a long range: more than 16 splits per unit, so the splits
+    combine through the workspace (last CTA to arrive) instead of a cluster."""
+    N = 20000
+    L = layer(1, 8, 2, N, [N - 3], seed=41, tail_fill=float("nan"))
+    Q, K, V, ln = G.to_dev(L, cuda_dev)
+    if dense:
+        O, _ = G.run_attn(Q, K, V, ln, None, None, 0, 1, SCALE)
+        ref = oracle.attn(L.Q, L.K, L.V, L.seq_lens, None, None, 0, 1, SCALE)
+    else:
+        rng = np.random.default_rng(3)
+        idx = _rand_idx(rng, 1, 2, [N - 3], 3000, [3000])
+        O, _ = G.run_attn(Q, K, V, ln, torch.from_numpy(idx).to(cuda_dev), [3000], 3000, 1, SCALE)
+        ref = oracle.attn(L.Q, L.K, L.V, L.seq_lens, idx, [3000], 3000, 1, SCALE)
+    check_output(O.cpu().numpy(), ref, "many splits")

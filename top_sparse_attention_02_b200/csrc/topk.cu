@@ -107,7 +107,19 @@ topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ lens,
     }
 
     const float* su = scores + (size_t)unit * rows_cap + lo;
-    for (int i = tid; i < nloc; i += kTkThreads) keys[i] = order_key(su[i]);
+    for (int i0 = tid; i0 < nloc; i0 += 8 * kTkThreads) {  // 8 independent loads in flight
+        float f[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int i = i0 + j * kTkThreads;
+            f[j] = i < nloc ? __ldcg(su + i) : 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int i = i0 + j * kTkThreads;
+            if (i < nloc) keys[i] = order_key(f[j]);
+        }
+    }
 
     // ---- radix select of the k-th largest key: digits [31:21], [20:10], [9:0]
     uint32_t prefix = 0, pmask = 0, krem = (uint32_t)kb;
@@ -128,6 +140,7 @@ topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ lens,
         const int hb0 = nbins - 1 - 2 * tid, hb1 = hb0 - 1;
         uint32_t c0 = 0, c1 = 0;
         if (hb1 >= 0) {
+#pragma unroll 4
             for (int r = 0; r < C; ++r) {
                 const uint32_t* rh = cluster.map_shared_rank(h, r);
                 c0 += rh[hb0];
