@@ -9,26 +9,35 @@
 // A null index list means every valid row (a full-attention layer, as the
 // Flux Attention router or a HyLRA sensitive layer chooses).
 //
-// Design: grid = (split, unit).  A CTA owns a contiguous range of the unit's
-// index list and walks it in tiles of 64 rows.  The rows' K and V (256 B each)
-// are gathered into shared memory with 16-byte cp.async copies (a 3-stage ring
-// when the range spans several tiles, one stage when it fits in one tile, so
-// that short sparse ranges leave room for more CTAs per SM).  Per tile, with
-// tile-level online softmax:
-//   A. logits: each half-warp owns 4 rows of the tile, each lane 8 dims; the g
-//      query heads stay in registers; partial dots are reduce-scattered across
-//      the half-warp and written to shared memory as z[row][head] (log2 units);
-//   B. one warp per head takes the tile max, the running max M, the rescale
-//      factor of the accumulators and p = 2^(z - M), and updates the running
-//      sum L;
-//   C. each lane accumulates p * V for its 8 dims and every head (no per-row
-//      rescaling, no cross-lane traffic).
-// Halves and warps are merged at the end into the CTA's partial (M, L,
-// acc[128]) per head.  With at most 16 splits per unit the splits of a unit
-// form one thread-block cluster and combine through distributed shared memory
-// (no scratch).  With more (few units, long ranges) each CTA writes its partial
-// to the workspace and the last CTA of the unit to arrive (an atomic counter in
-// the workspace, reset by that CTA) combines the partials into O.
+// Design: grid = (split, unit); a CTA is 8 warps and owns a contiguous range of
+// the unit's index list, walked in tiles of 128 rows (16 per warp).  The rows' K
+// and V (256 B each) are gathered into shared memory by the TMA engine, one
+// 256-byte bulk copy (cp.async.bulk) per K or V row completing on the stage's
+// mbarrier; rows are padded to 272 B so the tensor-core fragment loads below are
+// free of bank conflicts.  (16-byte cp.async copies issue from the load/store
+// unit, whose in-flight capacity held a gather to ~33 GB/s per SM.)  The index reads of the first three
+// tiles go out in one round, then all their copies, so a split of up to 384
+// rows has every gather in flight at once; a longer range refills each stage
+// as soon as its tile is consumed (one stage when the range fits in a tile).  Each warp then runs, on its
+// 16 rows, the two contractions of flash decoding on the tensor cores
+// (mma.sync m16n8k16, bf16 in, fp32 accumulate), with the g <= 8 query heads as
+// the M dimension padded to 16:
+//   S = Q K^T   (8 k-steps, K fragments by ldmatrix),
+//   online softmax per head on the S fragments (fp32, log2 units),
+//   O += P V    (P split as bf16 hi + bf16 lo so that the weights keep ~16
+//               bits; V fragments by ldmatrix.trans).
+// tcgen05's smallest M is 64, so there 87-94% of every MMA would be padding;
+// the m16 warp MMA fits a GQA group.  The 8 warps are merged at the end into
+// the CTA's partial (M, L, acc[128]) per head.  With at most 8 splits per unit
+// the splits of a unit form one thread-block cluster: each CTA pushes the slices
+// of its partial to the CTAs that own those output slices (posted
+// distributed-shared-memory stores), one cluster barrier, and each CTA combines
+// its slice locally (no scratch).  Clusters stay at <= 8 CTAs: on B200 only 7
+// clusters of 16 are co-resident, so 8 units of 16 would run in two waves.
+// With more splits (few units, or a long dense range)
+// each CTA writes its partial to the workspace and the last CTA of the unit to
+// arrive (an atomic counter in the workspace, reset by that CTA) combines the
+// partials into O.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -38,54 +47,105 @@ namespace cg = cooperative_groups;
 
 namespace tsa {
 
-constexpr int kAttnThreads = 256;
-constexpr int kAttnWarps = kAttnThreads / 32;
-constexpr int kTileRows = 64;                         // rows per staged tile
-constexpr int kRowGroups = kAttnThreads / 16;         // half-warps: 16
-constexpr int kRowsPerGroup = kTileRows / kRowGroups; // 4 rows of a tile per half-warp
-constexpr int kStageBytes = kTileRows * kD * 2 * 2;   // K and V of one tile (32 KB)
 constexpr int kMaxSplits = 256;
-constexpr int kClusterMax = 16;  // splits per unit that combine inside one cluster
+constexpr int kClusterMax = 8;  // splits per unit that combine inside one (portable) cluster
 constexpr int kSms = 148;
 constexpr int kPartStride = kD + 4;  // M, L, 2 pad, acc[128]: 528 B, 16-byte aligned
+constexpr int kAttnThreads = 256;
+constexpr int kAttnWarps = 8;
+constexpr int kTileRows = 128;                         // 16 rows per warp
+constexpr int kRowStride = kD * 2 + 16;                // 272 B: padded so 8 rows hit 8 bank groups
+constexpr int kStageBytes = kTileRows * kRowStride * 2;  // K and V of one tile: 68 KB
+constexpr int kRing = 3;                               // tiles in flight (the multi-tile kernel)
+constexpr long kWaitSpins = 1L << 22;                  // bounded mbarrier wait (then flag + go on)
 
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
-    const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
-}
+template <int G>
+struct AttnCfg {
+    static constexpr int kPer = G * 16;  // output float4 slots per CTA when S >= 2
+    static constexpr int kRecvBytes = kClusterMax * kPer * 16;
+    static constexpr int kAccBytes = kAttnWarps * G * kD * 4;
+    static constexpr int work_bytes(int stages) {
+        return stages * kStageBytes > kAccBytes ? stages * kStageBytes : kAccBytes;
+    }
+    static constexpr int smem_bytes(int stages, bool cluster) {
+        return work_bytes(stages) + (cluster ? kRecvBytes : 0);
+    }
+};
 
-__host__ __device__ constexpr int attn_smem_bytes(int G, int stages) {
-    return stages * kStageBytes > kAttnWarps * G * kD * 4 ? stages * kStageBytes : kAttnWarps * G * kD * 4;
+__device__ __forceinline__ unsigned smem_u32(const void* p) { return (unsigned)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count) : "memory");
 }
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("{\n .reg .b64 st;\n mbarrier.arrive.shared::cta.b64 st, [%0];\n}\n" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, unsigned bytes) {
+    asm volatile("{\n .reg .b64 st;\n mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n}\n"
+                 ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+// Wait for the phase with the given parity; gives up after kWaitSpins polls,
+// raising the timeout flag (the copies are still bounded: they read valid rows).
+__device__ __forceinline__ void mbar_wait(uint64_t* bar, unsigned parity, unsigned* flag) {
+    const unsigned a = smem_u32(bar);
+    for (long i = 0; i < kWaitSpins; ++i) {
+        unsigned done;
+        asm volatile("{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+                     : "=r"(done) : "r"(a), "r"(parity) : "memory");
+        if (done) return;
+    }
+    atomicOr(flag, kFlagTimeout);
+}
+// 1-D bulk copy (TMA engine) global -> this CTA's shared memory, completing on `bar`
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
+                 ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
+__device__ __forceinline__ void ldsm_x4(unsigned addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];\n"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(unsigned addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];\n"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+// D += A * B, m16n8k16, bf16 inputs, fp32 accumulate.  Only the rows of A that
+// carry query heads (a0/a1 and a4/a5: row lane/4) are non-zero here, so the
+// rows lane/4 + 8 of A are passed as zero.
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&v);
+}
+// byte offset of 16-byte chunk `chunk` of row `row` in a tile of padded rows
+__device__ __forceinline__ int roff(int row, int chunk) { return row * kRowStride + (chunk << 4); }
 
 template <int G, int STAGES, bool CLUSTER>
-__global__ void __launch_bounds__(kAttnThreads, G >= 8 ? 1 : 2)
+__global__ void __launch_bounds__(kAttnThreads)
 attn_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
             const __nv_bfloat16* __restrict__ V, const int32_t* __restrict__ lens,
             const int32_t* __restrict__ idx, const int32_t* __restrict__ kreq, int k_max,
             int block, int Hkv, int Ncap, float scale_log2, int S, float* __restrict__ part,
             unsigned* __restrict__ counters, float* __restrict__ O, unsigned* __restrict__ flag) {
-    constexpr int R = 16 / G;  // rows per half-warp per logit pass (R*G = 16 partial dots)
-    constexpr int kPassesA = (kRowsPerGroup + R - 1) / R;
-    extern __shared__ __align__(16) unsigned char smem[];
+    using Cfg = AttnCfg<G>;
+    extern __shared__ __align__(128) unsigned char smem[];
     __shared__ int s_row[STAGES][kTileRows];
-    __shared__ __align__(16) float s_z[kTileRows][G];  // logits, then weights p
-    __shared__ float s_M[G], s_L[G], s_alpha[G];
-    __shared__ float s_m[kAttnWarps][G], s_l[kAttnWarps][G];
-    __shared__ float s_cm[kMaxSplits * G], s_cl[kMaxSplits * G];
-    __shared__ __align__(16) float s_part[G][kD];  // the cluster path's partial
+    __shared__ float s_wm[kAttnWarps][G], s_wl[kAttnWarps][G];
+    __shared__ float s_M[G], s_L[G];
+    __shared__ float s_Mr[kClusterMax][G], s_Lr[kClusterMax][G];  // cluster path: received (M, L)
     __shared__ int s_last;
+    __shared__ __align__(8) uint64_t s_bar[STAGES];
 
     const int s = blockIdx.x, unit = blockIdx.y;
     const int b = unit / Hkv;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int half = lane >> 4, c = lane & 15;
-    const int rg = tid >> 4;  // this half-warp's row group
+    const int g = lane >> 2, t4 = lane & 3;  // mma fragment coordinates
 
     int len = lens[b];
     if (len < 0 || len > Ncap) {
@@ -133,257 +193,283 @@ attn_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict
         const int r = e * block + (pos - slot * block);
         return r < len ? r : -1;
     };
-    // stage tile t: thread (slot = tid/4, quarter = tid%4) copies 64 B of K and 64 B of V
-    auto issue = [&](int t) {
-        if (t < ntiles) {
-            const int st = t % STAGES;
-            const int slot = tid >> 2, q4 = tid & 3;
-            const int pos = p0 + t * kTileRows + slot;
-            const int row = pos < p1 ? row_of(pos) : -1;
-            if (q4 == 0) s_row[st][slot] = row;
-            if (row >= 0) {
-                unsigned char* kd = smem + st * kStageBytes + slot * (kD * 2) + q4 * 64;
-                unsigned char* vd = kd + kTileRows * kD * 2;
-                const unsigned char* ks = reinterpret_cast<const unsigned char*>(Ku + (size_t)row * kD) + q4 * 64;
-                const unsigned char* vs = reinterpret_cast<const unsigned char*>(Vu + (size_t)row * kD) + q4 * 64;
+    // thread slot (< 128) owns row `slot` of every tile: two 256-byte bulk copies
+    // (K and V) per valid row, each thread arriving once per tile on that
+    // stage's mbarrier (with the bytes it expects); unused rows are zero-filled.
+    const int my_slot = tid;
+    auto row_for_tile = [&](int t) -> int {
+        const int pos = p0 + t * kTileRows + my_slot;
+        return (my_slot < kTileRows && t < ntiles && pos < p1) ? row_of(pos) : -1;
+    };
+    auto stage_tile = [&](int t, int row) {
+        if (t >= ntiles || my_slot >= kTileRows) return;
+        const int st = t % STAGES;
+        s_row[st][my_slot] = row;
+        unsigned char* kd = smem + st * kStageBytes + my_slot * kRowStride;
+        unsigned char* vd = kd + kTileRows * kRowStride;
+        if (row >= 0) {
+            fence_proxy_async();  // earlier generic accesses of this stage come first
+            mbar_arrive_expect_tx(&s_bar[st], 2 * kD * 2);
+            bulk_g2s(kd, Ku + (size_t)row * kD, kD * 2, &s_bar[st]);
+            bulk_g2s(vd, Vu + (size_t)row * kD, kD * 2, &s_bar[st]);
+        } else {  // an unused row must hold zeros: its weight is 0 and 0 * garbage may be NaN
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    cp_async16(kd + 16 * j, ks + 16 * j);
-                    cp_async16(vd + 16 * j, vs + 16 * j);
-                }
+            for (int ch = 0; ch < 16; ++ch) {
+                *reinterpret_cast<uint4*>(kd + 16 * ch) = make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4*>(vd + 16 * ch) = make_uint4(0, 0, 0, 0);
             }
+            mbar_arrive(&s_bar[st]);
         }
-        cp_async_commit();  // one group per tile slot, empty past the end: uniform accounting
     };
 
-    float q[G][8];
+    if (tid == 0) {
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-        unpack8(*reinterpret_cast<const uint4*>(Q + ((size_t)unit * G + h) * kD + 8 * c), q[h]);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) q[h][e] *= scale_log2;
+        for (int i = 0; i < STAGES; ++i) mbar_init(&s_bar[i], kTileRows);
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
-    float acc[G][8];
+    __syncthreads();
+    // the first STAGES tiles: index reads in one round, then every copy
+    {
+        int pre[STAGES];
 #pragma unroll
-    for (int h = 0; h < G; ++h)
+        for (int t = 0; t < STAGES; ++t) pre[t] = row_for_tile(t);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[h][e] = 0.f;
-    if (tid < G) {
-        s_M[tid] = -INFINITY;
-        s_L[tid] = 0.f;
+        for (int t = 0; t < STAGES; ++t) stage_tile(t, pre[t]);
     }
 
+    // A fragments of Q (bf16, unscaled: the scale is applied to S in fp32).
+    // Row g of A = query head g of the group (zero for g >= G); rows g+8 are zero.
+    uint32_t qa[8][2];
+    {
+        const uint32_t* qrow = reinterpret_cast<const uint32_t*>(Q + ((size_t)unit * G + (g < G ? g : 0)) * kD);
 #pragma unroll
-    for (int t = 0; t < STAGES - 1; ++t) issue(t);
+        for (int ks = 0; ks < 8; ++ks) {
+            qa[ks][0] = g < G ? qrow[ks * 8 + t4] : 0u;       // dims 16ks + 2t4, +1
+            qa[ks][1] = g < G ? qrow[ks * 8 + 4 + t4] : 0u;   // dims 16ks + 8 + 2t4, +1
+        }
+    }
+    float o[16][4];  // O fragments: head g, dims 8n + 2t4 (+1); [2],[3] are padding rows
+#pragma unroll
+    for (int n = 0; n < 16; ++n)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[n][e] = 0.f;
+    float m_run = -INFINITY, l_run = 0.f;  // this warp's running max / sum for head g
+
+    const unsigned sbase = smem_u32(smem);
     for (int t = 0; t < ntiles; ++t) {
-        issue(t + STAGES - 1);
-        cp_async_wait<STAGES - 1>();
-        __syncthreads();
+        mbar_wait(&s_bar[t % STAGES], (unsigned)(t / STAGES) & 1u, flag);  // tile t has landed
         const int st = t % STAGES;
         const int tile_rows = min(kTileRows, p1 - p0 - t * kTileRows);
-        const unsigned char* ks = smem + st * kStageBytes;
-        const unsigned char* vs = ks + kTileRows * kD * 2;
-
-        // A. logits z[slot][h] for this half-warp's rows
+        const int r0 = warp * 16;  // this warp's rows in the tile
+        if (r0 < tile_rows) {      // warp-uniform
+            const unsigned kt = sbase + st * kStageBytes, vt = kt + kTileRows * kRowStride;
+            // ---- S = Q K^T over this warp's 16 rows (two n-tiles of 8 rows)
+            float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            {
+                const int m = lane >> 3, i = lane & 7;  // ldmatrix: matrix m, row i
+                const int row = r0 + (m >> 1) * 8 + i;   // n-tile (m>>1), k-half (m&1)
 #pragma unroll
-        for (int pa = 0; pa < kPassesA; ++pa) {
-            bool ok[R];
-            uint4 kr[R];
-#pragma unroll
-            for (int r = 0; r < R; ++r) {
-                const int slot = rg + kRowGroups * (pa * R + r);
-                ok[r] = slot < tile_rows && s_row[st][slot] >= 0;
-                kr[r] = ok[r] ? *reinterpret_cast<const uint4*>(ks + slot * (kD * 2) + 16 * c) : make_uint4(0, 0, 0, 0);
-            }
-            float v[16];
-#pragma unroll
-            for (int r = 0; r < R; ++r) {
-                float kf[8];
-                unpack8(kr[r], kf);
-#pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    float d = 0.f;
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) d = fmaf(kf[e], q[h][e], d);
-                    v[r * G + h] = d;
+                for (int ks = 0; ks < 8; ++ks) {
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4(kt + roff(row, 2 * ks + (m & 1)), b0, b1, b2, b3);
+                    mma_bf16(sc[0], qa[ks][0], qa[ks][1], b0, b1);
+                    mma_bf16(sc[1], qa[ks][0], qa[ks][1], b2, b3);
                 }
             }
-            halfwarp_reduce_scatter16(v, c);  // lane c: row pa*R + c/G of the group, head c%G
-            const int r = c / G, h = c - (c / G) * G;
-            const int slot = rg + kRowGroups * (pa * R + r);
-            if (slot < kTileRows) {
-                const bool valid = slot < tile_rows && s_row[st][slot] >= 0;
-                s_z[slot][h] = valid ? v[0] : -INFINITY;
+            // ---- online softmax for head g (columns = rows of the tile)
+            float z[4];
+            {
+                const int ra = r0 + 2 * t4;  // rows of sc[0][0..1]; sc[1] adds 8
+                const bool v0 = ra < tile_rows && s_row[st][ra] >= 0;
+                const bool v1 = ra + 1 < tile_rows && s_row[st][ra + 1] >= 0;
+                const bool v2 = ra + 8 < tile_rows && s_row[st][ra + 8] >= 0;
+                const bool v3 = ra + 9 < tile_rows && s_row[st][ra + 9] >= 0;
+                z[0] = v0 ? sc[0][0] * scale_log2 : -INFINITY;
+                z[1] = v1 ? sc[0][1] * scale_log2 : -INFINITY;
+                z[2] = v2 ? sc[1][0] * scale_log2 : -INFINITY;
+                z[3] = v3 ? sc[1][1] * scale_log2 : -INFINITY;
+            }
+            float mt = fmaxf(fmaxf(z[0], z[1]), fmaxf(z[2], z[3]));
+            mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
+            mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
+            const float mnew = fmaxf(m_run, mt);
+            if (mnew != -INFINITY) {  // uniform across the 4 lanes of head g
+                const float alpha = m_run == -INFINITY ? 0.f : exp2f(m_run - mnew);
+                float p[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) p[e] = z[e] == -INFINITY ? 0.f : exp2f(z[e] - mnew);
+                float ps = (p[0] + p[1]) + (p[2] + p[3]);
+                ps += __shfl_xor_sync(0xffffffffu, ps, 1);
+                ps += __shfl_xor_sync(0xffffffffu, ps, 2);
+                l_run = l_run * alpha + ps;
+                m_run = mnew;
+#pragma unroll
+                for (int n = 0; n < 16; ++n) {
+                    o[n][0] *= alpha;
+                    o[n][1] *= alpha;
+                }
+                // P as the A operand (row g, k = tile rows), split hi + lo
+                const uint32_t ph0 = pack_bf16(p[0], p[1]), ph1 = pack_bf16(p[2], p[3]);
+                const __nv_bfloat162 h0 = *reinterpret_cast<const __nv_bfloat162*>(&ph0);
+                const __nv_bfloat162 h1 = *reinterpret_cast<const __nv_bfloat162*>(&ph1);
+                const uint32_t pl0 = pack_bf16(p[0] - __low2float(h0), p[1] - __high2float(h0));
+                const uint32_t pl1 = pack_bf16(p[2] - __low2float(h1), p[3] - __high2float(h1));
+                // ---- O += P V over 16 dim n-tiles
+                const int m = lane >> 3, i = lane & 7;  // ldmatrix.trans: matrix m, row i
+                const int row = r0 + (m & 1) * 8 + i;    // k-half (m&1), dim n-tile (m>>1)
+#pragma unroll
+                for (int np = 0; np < 8; ++np) {
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4_t(vt + roff(row, 2 * np + (m >> 1)), b0, b1, b2, b3);
+                    mma_bf16(o[2 * np], ph0, ph1, b0, b1);
+                    mma_bf16(o[2 * np], pl0, pl1, b0, b1);
+                    mma_bf16(o[2 * np + 1], ph0, ph1, b2, b3);
+                    mma_bf16(o[2 * np + 1], pl0, pl1, b2, b3);
+                }
             }
         }
-        __syncthreads();
-        // B. warp h: tile max, running max and sum, weights p = 2^(z - M)
-        if (warp < G) {
-            const int h = warp;
-            const float z0 = s_z[lane][h], z1 = s_z[lane + 32][h];
-            float mt = fmaxf(z0, z1);
-#pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, o));
-            const float Mold = s_M[h];
-            const float Mnew = fmaxf(Mold, mt);
-            const float alpha = Mold == -INFINITY ? 0.f : exp2f(Mold - Mnew);
-            const float p0v = z0 == -INFINITY ? 0.f : exp2f(z0 - Mnew);
-            const float p1v = z1 == -INFINITY ? 0.f : exp2f(z1 - Mnew);
-            s_z[lane][h] = p0v;
-            s_z[lane + 32][h] = p1v;
-            float ps = p0v + p1v;
-#pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
-            if (lane == 0) {
-                s_M[h] = Mnew;
-                s_L[h] = s_L[h] * alpha + ps;
-                s_alpha[h] = alpha;
-            }
-        }
-        __syncthreads();
-        // C. acc[h][8 dims] = alpha_h * acc + sum over this group's rows of p[row][h] * V[row]
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-            const float a = s_alpha[h];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) acc[h][e] *= a;
-        }
-#pragma unroll
-        for (int i = 0; i < kRowsPerGroup; ++i) {
-            const int slot = rg + kRowGroups * i;
-            if (slot >= tile_rows || s_row[st][slot] < 0) continue;
-            float vf[8];
-            unpack8(*reinterpret_cast<const uint4*>(vs + slot * (kD * 2) + 16 * c), vf);
-#pragma unroll
-            for (int h = 0; h < G; ++h) {
-                const float p = s_z[slot][h];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) acc[h][e] = fmaf(p, vf[e], acc[h][e]);
-            }
-        }
-        __syncthreads();  // this stage and s_z are refilled next iteration
+        __syncthreads();               // every warp is done with this stage
+        stage_tile(t + STAGES, row_for_tile(t + STAGES));  // refill it (nothing past the end)
     }
-    cp_async_wait<0>();
+    __syncthreads();
 
-    // merge the two halves of each warp, then the warps (all share the CTA's M)
+    // ---- merge the 4 warps: each warp's (m, l, o) for heads g < G
+    float* s_acc = reinterpret_cast<float*>(smem);  // [kAttnWarps][G][128], over the staging ring
+    if (g < G) {
 #pragma unroll
-    for (int h = 0; h < G; ++h)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[h][e] += __shfl_xor_sync(0xffffffffu, acc[h][e], 16);
-    __syncthreads();
-    float* s_acc = reinterpret_cast<float*>(smem);  // [kAttnWarps][G][128]
-    if (half == 0) {
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-            float* dst = s_acc + (warp * G + h) * kD + 8 * c;
-            *reinterpret_cast<float4*>(dst) = make_float4(acc[h][0], acc[h][1], acc[h][2], acc[h][3]);
-            *reinterpret_cast<float4*>(dst + 4) = make_float4(acc[h][4], acc[h][5], acc[h][6], acc[h][7]);
+        for (int n = 0; n < 16; ++n)
+            *reinterpret_cast<float2*>(s_acc + (warp * G + g) * kD + 8 * n + 2 * t4) = make_float2(o[n][0], o[n][1]);
+        if (t4 == 0) {
+            s_wm[warp][g] = m_run;
+            s_wl[warp][g] = l_run;
         }
     }
     __syncthreads();
-    if (tid < G * 32) {  // thread (h, quad): dims 4*quad..4*quad+3 of head h
-        const int h = tid >> 5, qd = tid & 31;
-        float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (tid < G) {
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, s_wm[w][tid]);
+        float L = 0.f;
+#pragma unroll
+        for (int w = 0; w < kAttnWarps; ++w)
+            L += s_wm[w][tid] == -INFINITY ? 0.f : s_wl[w][tid] * exp2f(s_wm[w][tid] - M);
+        s_M[tid] = M;
+        s_L[tid] = L;
+    }
+    __syncthreads();
+    const int nslots = G * 32;  // (head, quad of dims) output slots: thread tid owns slot tid
+    const bool has_slot = tid < nslots;
+    const int h_me = tid >> 5, qd_me = tid & 31;
+    float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (has_slot) {
+        const float M = s_M[h_me];
 #pragma unroll
         for (int w = 0; w < kAttnWarps; ++w) {
-            const float4 a = *reinterpret_cast<const float4*>(s_acc + (w * G + h) * kD + 4 * qd);
-            A.x += a.x;
-            A.y += a.y;
-            A.z += a.z;
-            A.w += a.w;
-        }
-        if constexpr (CLUSTER) {
-            *reinterpret_cast<float4*>(&s_part[h][4 * qd]) = A;
-        } else {
-            float* pu = part + (((size_t)unit * S + s) * G + h) * kPartStride;
-            *reinterpret_cast<float4*>(pu + 4 + 4 * qd) = A;
-            if (qd == 0) *reinterpret_cast<float2*>(pu) = make_float2(s_M[h], s_L[h]);
+            const float wm = s_wm[w][h_me];
+            const float sc = (wm == -INFINITY || M == -INFINITY) ? 0.f : exp2f(wm - M);
+            const float4 a = *reinterpret_cast<const float4*>(s_acc + (w * G + h_me) * kD + 4 * qd_me);
+            A.x += a.x * sc;
+            A.y += a.y * sc;
+            A.z += a.z * sc;
+            A.w += a.w * sc;
         }
     }
 
     if constexpr (CLUSTER) {
+        if (S == 1) {  // nothing to combine
+            if (has_slot) {
+                const float L = s_L[h_me];
+                float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (L > 0.f) r = make_float4(A.x / L, A.y / L, A.z / L, A.w / L);
+                *reinterpret_cast<float4*>(O + ((size_t)unit * G + h_me) * kD + 4 * qd_me) = r;
+            }
+            return;
+        }
         // the S splits of this unit are the S CTAs of this cluster (rank = split)
         cg::cluster_group cluster = cg::this_cluster();
-        cluster.sync();  // every partial (s_M, s_L, s_part) is complete
-        const int per = (G * 32 + S - 1) / S;  // float4 output slots per CTA
-        if (tid < per) {
-            const int slot = s * per + tid;
-            if (slot < G * 32) {
-                const int h = slot >> 5, qd = slot & 31;
-                float mj[kClusterMax], lj[kClusterMax];
-                float M = -INFINITY;
-#pragma unroll
-                for (int j = 0; j < kClusterMax; ++j) {
-                    mj[j] = -INFINITY;
-                    lj[j] = 0.f;
-                    if (j < S) {
-                        mj[j] = *cluster.map_shared_rank(&s_M[h], j);
-                        lj[j] = *cluster.map_shared_rank(&s_L[h], j);
-                    }
-                    M = fmaxf(M, mj[j]);
-                }
-                float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-                float den = 0.f;
-                if (M != -INFINITY) {
-#pragma unroll
-                    for (int j = 0; j < kClusterMax; ++j) {
-                        if (j >= S) break;
-                        const float w = mj[j] == -INFINITY ? 0.f : exp2f(mj[j] - M);
-                        const float4 o = *reinterpret_cast<const float4*>(cluster.map_shared_rank(&s_part[h][4 * qd], j));
-                        den += w * lj[j];
-                        num.x += w * o.x;
-                        num.y += w * o.y;
-                        num.z += w * o.z;
-                        num.w += w * o.w;
-                    }
-                }
-                float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (den > 0.f) r = make_float4(num.x / den, num.y / den, num.z / den, num.w / den);
-                *reinterpret_cast<float4*>(O + ((size_t)unit * G + h) * kD + 4 * qd) = r;
-            }
+        const int per = ceil_div(nslots, S);  // output slots owned by each CTA
+        float4* recv = reinterpret_cast<float4*>(smem + Cfg::work_bytes(STAGES));  // [src][Cfg::kPer]
+        if (has_slot) {
+            const int owner = tid / per, lslot = tid - owner * per;
+            *cluster.map_shared_rank(recv + s * Cfg::kPer + lslot, owner) = A;
         }
-        cluster.sync();  // no CTA leaves while another may still read its shared memory
-        return;
-    }
-
-    // the last CTA of this unit to arrive combines all splits
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) s_last = atomicAdd(&counters[unit], 1u) == (unsigned)(S - 1);
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    const float* pall = part + (size_t)unit * S * G * kPartStride;
-    for (int i = tid; i < S * G; i += kAttnThreads) {
-        const float2 ml = __ldcg(reinterpret_cast<const float2*>(pall + (size_t)i * kPartStride));
-        s_cm[i] = ml.x;
-        s_cl[i] = ml.y;
-    }
-    __syncthreads();
-    if (tid < G * 32) {
-        const int h = tid >> 5, qd = tid & 31;
-        float M = -INFINITY;
-        for (int j = 0; j < S; ++j) M = fmaxf(M, s_cm[j * G + h]);
-        float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-        float den = 0.f;
-        if (M != -INFINITY) {
+        if (tid < G * S) {
+            const int r = tid / G, h = tid - (tid / G) * G;
+            *cluster.map_shared_rank(&s_Mr[s][h], r) = s_M[h];
+            *cluster.map_shared_rank(&s_Lr[s][h], r) = s_L[h];
+        }
+        cluster.sync();  // every slice has arrived at its owner
+        for (int ls = tid; ls < per; ls += kAttnThreads) {
+            const int slot = s * per + ls;
+            if (slot >= nslots) break;
+            const int h = slot >> 5, qd = slot & 31;
+            float M = -INFINITY;
+            for (int j = 0; j < S; ++j) M = fmaxf(M, s_Mr[j][h]);
+            float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+            float den = 0.f;
+            if (M != -INFINITY) {
+                for (int j = 0; j < S; ++j) {
+                    const float w = s_Mr[j][h] == -INFINITY ? 0.f : exp2f(s_Mr[j][h] - M);
+                    const float4 oj = recv[j * Cfg::kPer + ls];
+                    den += w * s_Lr[j][h];
+                    num.x += w * oj.x;
+                    num.y += w * oj.y;
+                    num.z += w * oj.z;
+                    num.w += w * oj.w;
+                }
+            }
+            float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (den > 0.f) r = make_float4(num.x / den, num.y / den, num.z / den, num.w / den);
+            *reinterpret_cast<float4*>(O + ((size_t)unit * G + h) * kD + 4 * qd) = r;
+        }
+        return;  // no remote access after the barrier: CTAs may leave in any order
+    } else {
+        if (has_slot) {
+            float* pu = part + (((size_t)unit * S + s) * G + h_me) * kPartStride;
+            *reinterpret_cast<float4*>(pu + 4 + 4 * qd_me) = A;
+            if (qd_me == 0) *reinterpret_cast<float2*>(pu) = make_float2(s_M[h_me], s_L[h_me]);
+        }
+        // the last CTA of this unit to arrive combines all splits
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) s_last = atomicAdd(&counters[unit], 1u) == (unsigned)(S - 1);
+        __syncthreads();
+        if (!s_last) return;
+        __threadfence();
+        float* s_cm = reinterpret_cast<float*>(smem);  // [S*G], over the staging ring
+        float* s_cl = s_cm + kMaxSplits * G;
+        const float* pall = part + (size_t)unit * S * G * kPartStride;
+        for (int i = tid; i < S * G; i += kAttnThreads) {
+            const float2 ml = __ldcg(reinterpret_cast<const float2*>(pall + (size_t)i * kPartStride));
+            s_cm[i] = ml.x;
+            s_cl[i] = ml.y;
+        }
+        __syncthreads();
+        for (int slot = tid; slot < nslots; slot += kAttnThreads) {
+            const int h = slot >> 5, qd = slot & 31;
+            float M = -INFINITY;
+            for (int j = 0; j < S; ++j) M = fmaxf(M, s_cm[j * G + h]);
+            float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+            float den = 0.f;
+            if (M != -INFINITY) {
 #pragma unroll 8
-            for (int j = 0; j < S; ++j) {
-                const float mj = s_cm[j * G + h];
-                const float w = mj == -INFINITY ? 0.f : exp2f(mj - M);
-                const float4 o = __ldcg(reinterpret_cast<const float4*>(pall + ((size_t)j * G + h) * kPartStride + 4 + 4 * qd));
-                den += w * s_cl[j * G + h];
-                num.x += w * o.x;
-                num.y += w * o.y;
-                num.z += w * o.z;
-                num.w += w * o.w;
+                for (int j = 0; j < S; ++j) {
+                    const float mj = s_cm[j * G + h];
+                    const float w = mj == -INFINITY ? 0.f : exp2f(mj - M);
+                    const float4 oj = __ldcg(reinterpret_cast<const float4*>(pall + ((size_t)j * G + h) * kPartStride + 4 + 4 * qd));
+                    den += w * s_cl[j * G + h];
+                    num.x += w * oj.x;
+                    num.y += w * oj.y;
+                    num.z += w * oj.z;
+                    num.w += w * oj.w;
+                }
             }
+            float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (den > 0.f) r = make_float4(num.x / den, num.y / den, num.z / den, num.w / den);
+            *reinterpret_cast<float4*>(O + ((size_t)unit * G + h) * kD + 4 * qd) = r;
         }
-        float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (den > 0.f) r = make_float4(num.x / den, num.y / den, num.z / den, num.w / den);
-        *reinterpret_cast<float4*>(O + ((size_t)unit * G + h) * kD + 4 * qd) = r;
+        if (tid == 0) counters[unit] = 0u;  // ready for the next launch on this workspace
     }
-    if (tid == 0) counters[unit] = 0u;  // ready for the next launch on this workspace
 }
 
 int attn_splits(const Dims& d, int k_max, int block, bool dense) {
@@ -391,16 +477,21 @@ int attn_splits(const Dims& d, int k_max, int block, bool dense) {
     long long rows;
     int s;
     if (dense) {
+        // bandwidth-bound streaming: one wave at one CTA per SM; past 8 splits
+        // the workspace combine (its cost is small next to the stream)
         rows = d.Ncap;
-        s = ceil_div(2 * kSms, units);  // one wave at two CTAs per SM
+        s = ceil_div(kSms, units);
     } else {
+        // latency-bound gather: splits of at most kRing tiles (all in flight at
+        // once), one tile each where the GPU has room, at most 8 splits (one
+        // cluster) unless fewer than 4 units would leave most SMs idle
         const long long nbmax = block == 1 ? d.Ncap : ceil_div(d.Ncap, block);
         rows = (long long)(k_max < nbmax ? k_max : nbmax) * block;
-        s = (int)((rows + kTileRows - 1) / kTileRows);  // one tile per split where possible
+        s = (int)((rows + kTileRows - 1) / kTileRows);
+        const int room = kSms / units > 1 ? kSms / units : 1;
+        if (s > room) s = room;
+        if (s > kClusterMax && units >= 4) s = kClusterMax;
     }
-    // Up to 16 splits combine inside a cluster (no scratch round trip).  Past 16,
-    // stay at 16 unless that leaves most of the GPU idle (fewer than 4 units).
-    if (s > kClusterMax && units * kClusterMax >= 4 * kClusterMax) s = kClusterMax;
     const long long smax = (rows + 31) / 32;  // at least 32 positions per split
     if (s > smax) s = (int)smax;
     if (s > kMaxSplits) s = kMaxSplits;
@@ -424,7 +515,7 @@ static cudaError_t attn_launch_g(dim3 grid, cudaStream_t st, const __nv_bfloat16
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = dim3(kAttnThreads);
-    cfg.dynamicSmemBytes = attn_smem_bytes(G, STAGES);
+    cfg.dynamicSmemBytes = AttnCfg<G>::smem_bytes(STAGES, CLUSTER);
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -439,8 +530,8 @@ static cudaError_t attn_launch_g(dim3 grid, cudaStream_t st, const __nv_bfloat16
 
 template <int G, int STAGES, bool CLUSTER>
 static cudaError_t attn_configure_one() {
-    cudaError_t e = cudaFuncSetAttribute(attn_kernel<G, STAGES, CLUSTER>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem_bytes(G, STAGES));
+    cudaError_t e = cudaFuncSetAttribute(attn_kernel<G, STAGES, CLUSTER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         AttnCfg<G>::smem_bytes(STAGES, CLUSTER));
     if (e == cudaSuccess && CLUSTER)
         e = cudaFuncSetAttribute(attn_kernel<G, STAGES, CLUSTER>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     return e;
@@ -449,9 +540,9 @@ static cudaError_t attn_configure_one() {
 template <int G>
 static cudaError_t attn_configure() {
     cudaError_t e = attn_configure_one<G, 1, true>();
-    if (e == cudaSuccess) e = attn_configure_one<G, 3, true>();
+    if (e == cudaSuccess) e = attn_configure_one<G, kRing, true>();
     if (e == cudaSuccess) e = attn_configure_one<G, 1, false>();
-    if (e == cudaSuccess) e = attn_configure_one<G, 3, false>();
+    if (e == cudaSuccess) e = attn_configure_one<G, kRing, false>();
     return e;
 }
 
@@ -465,13 +556,13 @@ static cudaError_t attn_dispatch(bool one_tile, bool cluster, dim3 grid, cudaStr
         if (one_tile)
             return attn_launch_g<G, 1, true>(grid, st, q, k, v, lens, idx, kreq, k_max, block, d, sl2, splits,
                                              partials, counters, O, flag);
-        return attn_launch_g<G, 3, true>(grid, st, q, k, v, lens, idx, kreq, k_max, block, d, sl2, splits,
+        return attn_launch_g<G, kRing, true>(grid, st, q, k, v, lens, idx, kreq, k_max, block, d, sl2, splits,
                                          partials, counters, O, flag);
     }
     if (one_tile)
         return attn_launch_g<G, 1, false>(grid, st, q, k, v, lens, idx, kreq, k_max, block, d, sl2, splits,
                                           partials, counters, O, flag);
-    return attn_launch_g<G, 3, false>(grid, st, q, k, v, lens, idx, kreq, k_max, block, d, sl2, splits, partials,
+    return attn_launch_g<G, kRing, false>(grid, st, q, k, v, lens, idx, kreq, k_max, block, d, sl2, splits, partials,
                                       counters, O, flag);
 }
 
