@@ -29,6 +29,9 @@ cudaError_t launch_block_summarize(const void* K, const int32_t* lens, const Dim
 
 cudaError_t launch_score(const void* Q, const void* keys, const int32_t* lens, const Dims& d,
                          int block, float scale, float* scores, unsigned* flag, cudaStream_t st);
+// token mode on the tensor cores (TMA + tcgen05); used by launch_score for bf16 keys
+cudaError_t launch_score_tc(const void* Q, const void* K, const int32_t* lens, const Dims& d, float scale,
+                            float* scores, unsigned* flag, cudaStream_t st);
 
 // top-k plan: cluster size and keys per CTA for a row count; false if too large
 bool topk_plan(int rows_cap, int* cluster, int* chunk);

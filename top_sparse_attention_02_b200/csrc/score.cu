@@ -163,7 +163,7 @@ static cudaError_t score_dispatch(const void* Q, const void* keys, const int32_t
 cudaError_t launch_score(const void* Q, const void* keys, const int32_t* lens, const Dims& d,
                          int block, float scale, float* scores, unsigned* flag, cudaStream_t st) {
     if (d.units() == 0 || d.Ncap == 0) return cudaSuccess;
-    if (block == 1) return score_dispatch<false>(Q, keys, lens, d, block, scale, scores, flag, st);
+    if (block == 1) return launch_score_tc(Q, keys, lens, d, scale, scores, flag, st);
     return score_dispatch<true>(Q, keys, lens, d, block, scale, scores, flag, st);
 }
 
