@@ -239,6 +239,7 @@ def run_ours(args, rank, world, dev):
     # per-stage device times: each stage alone, repeated in its own graph
     stages = stage_times(tsa, w, plan, layers, Kmean, ws, kreq_t, idx, O, stream)
     copy_gbs = copy_probe(tsa, dev, stream)
+    gather = gather_probe(tsa, w, plan, layers, idx, ws, stream)
 
     peak, peak_kind = measured_peaks()
     score_us = stages["score_us"]
@@ -263,6 +264,7 @@ def run_ours(args, rank, world, dev):
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, torch copy)",
                      "copy_probe_gbs_this_run": copy_gbs, "traffic": None,
                      "algorithmic_bytes_per_launch": score_bytes},
+        "attn_roofline": attn_roofline(w, plan, stages, gather),
         "clocks": clk.summary(),
         "gpu_launches": launches,
         "timing": "CUDA graph of one whole step, replayed K times between CUDA events",
@@ -337,6 +339,56 @@ def copy_probe(tsa, dev, stream, nbytes=2 << 30):
         best = max(best, 2 * a.numel() / (e0.elapsed_time(e1) * 1e-3) / 1e9)
     del a, b
     return best
+
+
+def gather_probe(tsa, w, plan, layers, idx, ws, stream, reps=10):
+    """Random-row gather ceiling on the attention stage's own rows: the rows layer 0
+    selected, fetched from a reuse layer's K and V by tsa_hbm_gather (bulk copies
+    into shared memory, nothing kept).  Returns GB/s over the bytes fetched."""
+    sel = [li for li, m in enumerate(w.route) if m == 1]
+    if not sel or w.block != 1:
+        return None
+    src_layer = layers[1] if len(layers) > 1 else layers[0]
+    ix = idx[sel[0]].reshape(w.B * w.Hkv, -1).long()
+    base = torch.arange(w.B * w.Hkv, device=ix.device).unsqueeze(1) * w.Ncap
+    rows = (ix + base)[ix >= 0].to(torch.int32).contiguous()
+    K2 = src_layer.K.view(torch.uint8).reshape(-1)
+    V2 = src_layer.V.view(torch.uint8).reshape(-1)
+    with torch.cuda.stream(stream):
+        tsa.hbm_gather(K2, rows, ws, stream)
+        tsa.hbm_gather(V2, rows, ws, stream)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for _ in range(reps):
+            tsa.hbm_gather(K2, rows, ws, stream)
+            tsa.hbm_gather(V2, rows, ws, stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        g.replay()
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+    stream.synchronize()
+    tsa.check_device_status(ws, stream)
+    us = e0.elapsed_time(e1) * 1e3 / reps
+    nbytes = 2 * rows.numel() * 256
+    del g
+    return {"gbs": nbytes / (us * 1e-6) / 1e9, "us": us, "bytes": nbytes,
+            "rows": "the K and V rows layer 0 selected, in another layer's cache"}
+
+
+def attn_roofline(w, plan, stages, gather):
+    """The attention stage against the random-row gather ceiling measured in this run."""
+    if gather is None:
+        return None
+    reuse = [k for k in stages if k.endswith("_attn") and not k.startswith("L0")]
+    us = statistics.mean(stages[k] for k in reuse) if reuse else stages.get("L0_attn")
+    achieved = plan.bytes["gather"] / (us * 1e-6) / 1e9
+    return {"kernel": "attn_kernel (one reuse layer)", "bound": "hbm random-row gather",
+            "achieved": achieved, "peak": gather["gbs"], "unit": "GB/s", "frac": achieved / gather["gbs"],
+            "peak_source": "tsa_hbm_gather on the same rows in this run", "algorithmic_bytes_per_launch":
+            plan.bytes["gather"]}
 
 
 def e2e_measure(tsa, w, plan, layers, step_args, O, idx, stream, args):

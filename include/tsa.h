@@ -198,6 +198,15 @@ uint64_t tsa_launch_count(void);
  * and stores over a grid sized to the SM count.  bytes must be a multiple of 16. */
 tsa_status tsa_hbm_copy(const void* src, void* dst, size_t bytes, void* stream);
 
+/* Random-row gather probe: fetch the 256-byte rows base[rows[i]*256 .. +256)
+ * (rows[] on the device, nrows of them) into shared memory with bulk copies and
+ * drop them.  Its bandwidth is the ceiling of a gather-bound stage (the
+ * attention stage reads the selected K/V rows at random).  base_bytes must be a
+ * multiple of 256; a row number outside [0, base_bytes/256) is skipped and sets
+ * the device flag in ws (>= 256 bytes). */
+tsa_status tsa_hbm_gather(const void* base, size_t base_bytes, const int32_t* rows, int32_t nrows, void* ws,
+                          size_t ws_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -276,3 +276,16 @@ def test_attn_many_splits_workspace_combine(cuda_dev, dense):
         O, _ = G.run_attn(Q, K, V, ln, torch.from_numpy(idx).to(cuda_dev), [3000], 3000, 1, SCALE)
         ref = oracle.attn(L.Q, L.K, L.V, L.seq_lens, idx, [3000], 3000, 1, SCALE)
     check_output(O.cpu().numpy(), ref, "many splits")
+
+
+def test_gather_probe_runs_and_flags_bad_rows(cuda_dev):
+    base = torch.zeros(1 << 20, dtype=torch.uint8, device=cuda_dev)  # 4096 rows of 256 B
+    ws = torch.zeros(256, dtype=torch.uint8, device=cuda_dev)
+    rows = torch.randint(0, 4096, (1000,), dtype=torch.int32, device=cuda_dev)
+    tsa.hbm_gather(base, rows, ws)
+    tsa.check_device_status(ws)
+    rows[7] = 4096  # one past the end: skipped and flagged, never read
+    tsa.hbm_gather(base, rows, ws)
+    with pytest.raises(tsa.TsaError) as e:
+        tsa.check_device_status(ws)
+    assert e.value.status == tsa.TSA_ERR_DEVICE_BOUNDS

@@ -55,6 +55,7 @@ _SIGS = {
     "tsa_last_error_string": (ctypes.c_char_p, []),
     "tsa_launch_count": (ctypes.c_uint64, []),
     "tsa_hbm_copy": (ctypes.c_int, [_vp, _vp, _sz, _vp]),
+    "tsa_hbm_gather": (ctypes.c_int, [_vp, _sz, _vp, _i32, _vp, _sz, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -188,3 +189,9 @@ def launch_count() -> int:
 
 def hbm_copy(src, dst, nbytes: int, stream=None):
     _ok(_lib.tsa_hbm_copy(_ptr(src), _ptr(dst), nbytes, _stream(stream)))
+
+
+def hbm_gather(base, rows, ws, stream=None):
+    """Gather the 256-byte rows `rows` (int32, device) of `base` (the probe; nothing is kept)."""
+    nbytes = base.numel() * base.element_size()
+    _ok(_lib.tsa_hbm_gather(_ptr(base), nbytes, _ptr(rows), rows.numel(), *_wsargs(ws), _stream(stream)))

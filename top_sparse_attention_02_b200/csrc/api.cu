@@ -286,4 +286,16 @@ tsa_status tsa_hbm_copy(const void* src, void* dst, size_t bytes, void* stream) 
     return TSA_OK;
 }
 
+tsa_status tsa_hbm_gather(const void* base, size_t base_bytes, const int32_t* rows, int32_t nrows, void* ws,
+                          size_t ws_bytes, void* stream) {
+    if (!base || (!rows && nrows > 0)) return fail(TSA_ERR_INVALID_ARG, "tsa_hbm_gather: NULL pointer");
+    if (!aligned16(base) || base_bytes % 256 != 0)
+        return fail(TSA_ERR_INVALID_ARG, "tsa_hbm_gather: base must be 16-byte aligned and a whole number of 256-byte rows");
+    if (nrows < 0) return fail(TSA_ERR_INVALID_ARG, "tsa_hbm_gather: nrows must be >= 0");
+    TSA_TRY(check_ws(ws, ws_bytes, kFlagBytes));
+    cudaError_t e = tsa::launch_gather(base, base_bytes, rows, nrows, flag_of(ws), static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "tsa_hbm_gather");
+    return TSA_OK;
+}
+
 }  // extern "C"

@@ -1,6 +1,10 @@
-// copy.cu -- HBM roofline probe: a plain 16-byte-vector device-to-device copy
-// over a grid sized to the SM count.  Its bandwidth (read + write bytes / time)
-// is the denominator the decode kernels are compared against in the same run.
+// copy.cu -- HBM roofline probes.
+//  - copy: a plain 16-byte-vector device-to-device copy over a grid sized to the
+//    SM count; its bandwidth (read + write bytes / time) is the streaming peak
+//    the scan kernels are compared against in the same run.
+//  - gather: 256-byte rows at given row numbers, fetched by TMA bulk copies into
+//    shared memory and dropped; its bandwidth is the random-row ceiling the
+//    attention stage (which gathers the selected K/V rows) is compared against.
 #include "common.cuh"
 #include "launch.h"
 
@@ -19,6 +23,72 @@ __global__ void __launch_bounds__(256) copy_kernel(const uint4* __restrict__ src
         dst[i + 3 * stride] = d;
     }
     for (; i < n16; i += stride) dst[i] = ld_stream(src + i);
+}
+
+constexpr int kGatherRowsPerCta = 256;  // a 64 KB shared-memory window per CTA
+constexpr long kGatherSpins = 1L << 22;
+
+__global__ void __launch_bounds__(128) gather_kernel(const unsigned char* __restrict__ base, size_t nrows_base,
+                                                     const int32_t* __restrict__ rows, int nrows,
+                                                     unsigned* __restrict__ flag) {
+    extern __shared__ __align__(128) unsigned char gsm[];
+    __shared__ __align__(8) uint64_t bar;
+    const unsigned bar_a = (unsigned)__cvta_generic_to_shared(&bar);
+    if (threadIdx.x == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar_a), "r"(128) : "memory");
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    __syncthreads();
+    const int r0 = blockIdx.x * kGatherRowsPerCta;
+    const int r1 = min(r0 + kGatherRowsPerCta, nrows);
+    unsigned bytes = 0;
+    for (int j = r0 + threadIdx.x; j < r1; j += 128) {
+        const int32_t r = rows[j];
+        if (r >= 0 && (size_t)r < nrows_base) bytes += 256;
+    }
+    asm volatile("{\n .reg .b64 st;\n mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n}\n" ::"r"(bar_a),
+                 "r"(bytes)
+                 : "memory");
+    for (int j = r0 + threadIdx.x; j < r1; j += 128) {
+        const int32_t r = rows[j];
+        if (r < 0 || (size_t)r >= nrows_base) {
+            atomicOr(flag, kFlagBounds);
+            continue;
+        }
+        const unsigned dst = (unsigned)__cvta_generic_to_shared(gsm + (j - r0) * 256);
+        asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], 256, [%2];\n" ::"r"(
+                         dst),
+                     "l"(base + (size_t)r * 256), "r"(bar_a)
+                     : "memory");
+    }
+    for (long i = 0; i < kGatherSpins; ++i) {
+        unsigned done;
+        asm volatile(
+            "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], 0;\n selp.u32 %0, 1, 0, p;\n}\n"
+            : "=r"(done)
+            : "r"(bar_a)
+            : "memory");
+        if (done) return;
+    }
+    atomicOr(flag, kFlagTimeout);
+}
+
+cudaError_t launch_gather(const void* base, size_t base_bytes, const int32_t* rows, int nrows, unsigned* flag,
+                          cudaStream_t st) {
+    if (nrows <= 0) return cudaSuccess;
+    static int configured[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64 && !configured[dev]) {
+        e = cudaFuncSetAttribute(gather_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGatherRowsPerCta * 256);
+        if (e != cudaSuccess) return e;
+        configured[dev] = 1;
+    }
+    gather_kernel<<<ceil_div(nrows, kGatherRowsPerCta), 128, kGatherRowsPerCta * 256, st>>>(
+        static_cast<const unsigned char*>(base), base_bytes / 256, rows, nrows, flag);
+    note_launch();
+    return cudaGetLastError();
 }
 
 cudaError_t launch_copy(const void* src, void* dst, size_t bytes, cudaStream_t st) {

@@ -48,5 +48,7 @@ cudaError_t launch_attn(const void* Q, const void* K, const void* V, const int32
                         unsigned* counters, float* O, unsigned* flag, cudaStream_t st);
 
 cudaError_t launch_copy(const void* src, void* dst, size_t bytes, cudaStream_t st);
+cudaError_t launch_gather(const void* base, size_t base_bytes, const int32_t* rows, int nrows, unsigned* flag,
+                          cudaStream_t st);
 
 }  // namespace tsa
