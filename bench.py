@@ -34,6 +34,22 @@ METRIC = ("decode-step µs & achieved HBM TB/s (score+top-k+sparse attn), 128K c
 FALLBACK_HBM_GBS = 6650.0
 
 
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu record, or None when
+    the kernel's source has changed since the counters were taken."""
+    import hashlib
+
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            rec = json.load(f)[kernel]
+        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+    except (OSError, KeyError, ValueError):
+        return None
+    return rec["bytes_per_launch"] if sha == rec["source_sha256"] else None
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -259,10 +275,11 @@ def run_ours(args, rank, world, dev):
         "algorithmic_bytes_per_step": plan.step_bytes,
         "tokens_attended_per_s": world * plan.tokens_attended * w.layers / (ms * 1e-3),
         "stages_us": stages,
-        "roofline": {"kernel": "score_kernel (layer-0 K scan)", "bound": "hbm",
+        "roofline": {"kernel": "score_tc_kernel (layer-0 K scan)", "bound": "hbm",
                      "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, torch copy)",
-                     "copy_probe_gbs_this_run": copy_gbs, "traffic": None,
+                     "copy_probe_gbs_this_run": copy_gbs,
+                     "traffic": recorded_traffic("score_tc_kernel") if w is workloads.REUSE128K else None,
                      "algorithmic_bytes_per_launch": score_bytes},
         "attn_roofline": attn_roofline(w, plan, stages, gather),
         "clocks": clk.summary(),
