@@ -146,6 +146,8 @@ attn_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict
     const int b = unit / Hkv;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t4 = lane & 3;  // mma fragment coordinates
+    griddep_wait();
+    griddep_launch();
 
     int len = lens[b];
     if (len < 0 || len > Ncap) {
@@ -517,13 +519,14 @@ static cudaError_t attn_launch_g(dim3 grid, cudaStream_t st, const __nv_bfloat16
     cfg.blockDim = dim3(kAttnThreads);
     cfg.dynamicSmemBytes = AttnCfg<G>::smem_bytes(STAGES, CLUSTER);
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = CLUSTER ? (unsigned)splits : 1u;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1] = pdl_attr();
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, attn_kernel<G, STAGES, CLUSTER>, q, k, v, lens, idx, kreq, k_max, block,
                               d.Hkv, d.Ncap, sl2, splits, partials, counters, O, flag);
 }

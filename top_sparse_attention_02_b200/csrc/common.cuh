@@ -75,6 +75,14 @@ __device__ __forceinline__ void halfwarp_reduce_scatter16(float (&v)[16], int c)
     }
 }
 
+// Programmatic dependent launch: the kernels of a decode step are launched so
+// that the next one may start (launch, set-up) while this one finishes.  Every
+// kernel waits for its predecessor before touching global memory, which keeps
+// the stream's order for data; and lets its successor launch once all of its
+// CTAs are running.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
 __device__ __forceinline__ int clamp_len(int len, int Ncap, unsigned* flag) {
     if (len < 0 || len > Ncap) {
         atomicOr(flag, kFlagBounds);

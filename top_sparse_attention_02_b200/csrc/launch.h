@@ -21,6 +21,14 @@ inline int rows_cap_of(const Dims& d, int block) { return block == 1 ? d.Ncap : 
 
 void note_launch();
 
+// launch attribute for programmatic dependent launch (see griddep_wait)
+inline cudaLaunchAttribute pdl_attr() {
+    cudaLaunchAttribute a;
+    a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    a.val.programmaticStreamSerializationAllowed = 1;
+    return a;
+}
+
 // set the text tsa_last_error_string() returns on this thread
 void set_error_message(const char* msg);
 

@@ -31,6 +31,8 @@ score_kernel(const __nv_bfloat16* __restrict__ Q, const void* __restrict__ keys,
     constexpr int kRowsCta = kRowsStep * kScoreWarps * kScoreSteps;
     const int unit = blockIdx.y;
     const int b = unit / Hkv, kvh = unit - b * Hkv;
+    griddep_wait();
+    griddep_launch();
     int len = lens[b];
     if (len < 0 || len > Ncap) {
         if (threadIdx.x == 0) atomicOr(flag, kFlagBounds);
@@ -141,22 +143,23 @@ static cudaError_t score_dispatch(const void* Q, const void* keys, const int32_t
     const int rows_cta = 2 * (16 / d.G) * kScoreWarps * kScoreSteps;
     dim3 grid(ceil_div(rows_cap, rows_cta), d.units());
     const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(Q);
-#define TSA_SCORE_CASE(g)                                                                      \
-    case g:                                                                                    \
-        score_kernel<g, kMeans><<<grid, kScoreThreads, 0, st>>>(q, keys, lens, d.Hkv, d.Ncap,   \
-                                                                rows_cap, block, scale, scores, \
-                                                                flag);                          \
-        break;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kScoreThreads);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1] = {pdl_attr()};
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e;
     switch (d.G) {
-        TSA_SCORE_CASE(1)
-        TSA_SCORE_CASE(2)
-        TSA_SCORE_CASE(4)
-        TSA_SCORE_CASE(8)
-        default:
-            return cudaErrorInvalidValue;
+        case 1: e = cudaLaunchKernelEx(&cfg, score_kernel<1, kMeans>, q, keys, lens, d.Hkv, d.Ncap, rows_cap, block, scale, scores, flag); break;
+        case 2: e = cudaLaunchKernelEx(&cfg, score_kernel<2, kMeans>, q, keys, lens, d.Hkv, d.Ncap, rows_cap, block, scale, scores, flag); break;
+        case 4: e = cudaLaunchKernelEx(&cfg, score_kernel<4, kMeans>, q, keys, lens, d.Hkv, d.Ncap, rows_cap, block, scale, scores, flag); break;
+        case 8: e = cudaLaunchKernelEx(&cfg, score_kernel<8, kMeans>, q, keys, lens, d.Hkv, d.Ncap, rows_cap, block, scale, scores, flag); break;
+        default: return cudaErrorInvalidValue;
     }
-#undef TSA_SCORE_CASE
     note_launch();
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -95,6 +95,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16* _
     const int unit = blockIdx.y;
     const int b = unit / Hkv;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    griddep_wait();
     int len = lens[b];
     if (len < 0 || len > Ncap) {
         if (tid == 0 && blockIdx.x == 0) atomicOr(flag, kFlagBounds);
@@ -229,6 +230,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16* _
             tc_arrive(su32(&s_tempty[bsel]));
         }
     }
+    griddep_launch();
     asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
     __syncthreads();
     if (warp == 1) {
@@ -282,14 +284,23 @@ cudaError_t launch_score_tc(const void* Q, const void* K, const int32_t* lens, c
     const int tiles = ceil_div(d.Ncap, kTcTileRows);
     dim3 grid(ceil_div(tiles, kTcTilesPerCta), d.units());
     const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(Q);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kTcThreads);
+    cfg.dynamicSmemBytes = kTcSmem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1] = {pdl_attr()};
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     switch (d.G) {
-        case 1: score_tc_kernel<1><<<grid, kTcThreads, kTcSmem, st>>>(map, q, lens, d.Hkv, d.Ncap, scale, scores, flag); break;
-        case 2: score_tc_kernel<2><<<grid, kTcThreads, kTcSmem, st>>>(map, q, lens, d.Hkv, d.Ncap, scale, scores, flag); break;
-        case 4: score_tc_kernel<4><<<grid, kTcThreads, kTcSmem, st>>>(map, q, lens, d.Hkv, d.Ncap, scale, scores, flag); break;
-        case 8: score_tc_kernel<8><<<grid, kTcThreads, kTcSmem, st>>>(map, q, lens, d.Hkv, d.Ncap, scale, scores, flag); break;
+        case 1: e = cudaLaunchKernelEx(&cfg, score_tc_kernel<1>, map, q, lens, d.Hkv, d.Ncap, scale, scores, flag); break;
+        case 2: e = cudaLaunchKernelEx(&cfg, score_tc_kernel<2>, map, q, lens, d.Hkv, d.Ncap, scale, scores, flag); break;
+        case 4: e = cudaLaunchKernelEx(&cfg, score_tc_kernel<4>, map, q, lens, d.Hkv, d.Ncap, scale, scores, flag); break;
+        case 8: e = cudaLaunchKernelEx(&cfg, score_tc_kernel<8>, map, q, lens, d.Hkv, d.Ncap, scale, scores, flag); break;
         default: return cudaErrorInvalidValue;
     }
     note_launch();
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -79,6 +79,8 @@ topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ lens,
     const int unit = blockIdx.x / C;
     const int b = unit / Hkv;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    griddep_wait();
+    griddep_launch();
 
     extern __shared__ __align__(16) uint32_t tk_smem[];
     uint32_t* keys = tk_smem;                                      // [chunk]
@@ -393,13 +395,14 @@ cudaError_t launch_topk(const float* scores, const int32_t* lens, const int32_t*
     cfg.blockDim = dim3(kTkThreads);
     cfg.dynamicSmemBytes = topk_smem_bytes(chunk);
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)C;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1] = pdl_attr();
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     e = cudaLaunchKernelEx(&cfg, topk_kernel, scores, lens, kreq, k_max, d.Hkv, d.Ncap, rows_cap,
                            block, chunk, idx, flag);
     note_launch();
