@@ -289,3 +289,21 @@ def test_gather_probe_runs_and_flags_bad_rows(cuda_dev):
     with pytest.raises(tsa.TsaError) as e:
         tsa.check_device_status(ws)
     assert e.value.status == tsa.TSA_ERR_DEVICE_BOUNDS
+
+
+def test_select_steps_share_one_workspace(cuda_dev):
+    """The scorer leaves a first-pass histogram in the workspace that the top-k
+    kernel consumes and clears: consecutive steps on one workspace (with units
+    where every row is taken, which skip the select) must each match the oracle."""
+    B, Hq, Hkv, N = 3, 16, 4, 3000
+    lens, kreq, k_max = [3000, 40, 2999], [50, 60, 50], 60
+    ws = G.ws_for(torch.empty(B, Hq, 128, device=cuda_dev, dtype=torch.bfloat16),
+                  torch.empty(B, Hkv, N, 128, device=cuda_dev, dtype=torch.bfloat16), k_max, 1, tsa.SELECT)
+    for seed in (51, 52, 53):
+        L = layer(B, Hq, Hkv, N, lens, seed=seed)
+        Q, K, V, ln = G.to_dev(L, cuda_dev)
+        O, idx = G.step(Q, K, V, ln, mode=tsa.SELECT, scale=SCALE, k_max=k_max, kreq=kreq, ws=ws)
+        S = oracle.scores(L.Q, L.K, L.seq_lens, SCALE)
+        compare_idx(idx.cpu().numpy(), S, lens, kreq)
+        ref = oracle.attn(L.Q, L.K, L.V, L.seq_lens, idx.cpu().numpy(), kreq, k_max, 1, SCALE)
+        check_output(O.cpu().numpy(), ref, f"step with seed {seed}")
