@@ -17,6 +17,7 @@ times the fp64 CPU oracle on the host cores instead (rank 0 only).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -106,6 +107,19 @@ def make_layers(w, dev, lens):
     return layers
 
 
+def workload_of(args):
+    """The named workload; --ncap shrinks its context (a smaller case for profiler
+    captures, never a bench line of the named workload)."""
+    from top_sparse_attention_02_b200 import workloads
+
+    w = workloads.ALL[args.workload]
+    if args.ncap:
+        n = int(args.ncap)
+        lens = None if w.lens is None else (min(w.lens[0], n), min(w.lens[1], n))
+        w = dataclasses.replace(w, Ncap=n, lens=lens, name=f"{w.name} [reduced to N={n} for profiling]")
+    return w
+
+
 def workload_lens(w):
     from top_sparse_attention_02_b200 import inputs
 
@@ -178,7 +192,7 @@ def run_ours(args, rank, world, dev):
     from top_sparse_attention_02_b200 import binding as tsa
     from top_sparse_attention_02_b200 import workloads
 
-    w = workloads.ALL[args.workload]
+    w = workload_of(args)
     lens = workload_lens(w)
     plan = Plan(w, lens)
     layers = make_layers(w, dev, lens)
@@ -286,7 +300,8 @@ def run_ours(args, rank, world, dev):
         "gpu_launches": launches,
         "timing": "CUDA graph of one whole step, replayed K times between CUDA events",
     }
-    res["e2e"] = e2e_measure(tsa, w, plan, layers, step_args, O, idx, stream, args)
+    if not args.no_e2e:
+        res["e2e"] = e2e_measure(tsa, w, plan, layers, step_args, O, idx, stream, args)
     return res
 
 
@@ -560,6 +575,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="reuse128k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--ncap", type=int, default=0,
+                    help="shrink the workload's context to this many tokens (profiler captures only)")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))

@@ -132,9 +132,13 @@ def test_attn_dense_mode(cuda_dev, lens):
     check_output(O.cpu().numpy(), ref, "dense")
 
 
-def test_attn_block_mode_expansion(cuda_dev):
+@pytest.mark.parametrize("Ncap", [1024, 1000])
+def test_attn_block_mode_expansion(cuda_dev, Ncap):
+    """128-token blocks; Ncap = 1000 puts the partial last block against the end of
+    each unit's cache, so its 128-row tile reaches into the next unit's rows (or
+    past the end of the cache for the last unit)."""
     lens = [1000, 130]
-    L = layer(2, 8, 2, 1024, lens, seed=17, tail_fill=float("nan"))
+    L = layer(2, 8, 2, Ncap, lens, seed=17, tail_fill=float("nan"))
     Q, K, V, ln = G.to_dev(L, cuda_dev)
     idx = np.full((2, 2, 4), -1, dtype=np.int32)
     idx[0, 0, :3] = [0, 5, 7]  # block 7 is the partial last block (rows 896..999)

@@ -39,6 +39,9 @@
 // arrive (an atomic counter in the workspace, reset by that CTA) combines the
 // partials into O.
 #include <cooperative_groups.h>
+#include <cstring>
+#include <cuda.h>
+#include <cudaTypedefs.h>
 
 #include "common.cuh"
 #include "launch.h"
@@ -68,7 +71,7 @@ struct AttnCfg {
         return stages * kStageBytes > kAccBytes ? stages * kStageBytes : kAccBytes;
     }
     static constexpr int smem_bytes(int stages, bool cluster) {
-        return work_bytes(stages) + (cluster ? kRecvBytes : 0);
+        return 1024 /* alignment slack */ + work_bytes(stages) + (cluster ? kRecvBytes : 0);
     }
 };
 
@@ -126,21 +129,29 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 // byte offset of 16-byte chunk `chunk` of row `row` in a tile of padded rows
 __device__ __forceinline__ int roff(int row, int chunk) { return row * kRowStride + (chunk << 4); }
 
-template <int G, int STAGES, bool CLUSTER>
+// CONTIG: every tile is 128 consecutive cache rows (a full-attention range, or
+// one 128-token block in block mode) and arrives by 2-D TMA tensor loads in the
+// 128-byte-swizzled layout (4 loads per tile); otherwise each row is its own
+// 256-byte bulk copy into rows padded to 272 bytes.
+template <int G, int STAGES, bool CLUSTER, bool CONTIG>
 __global__ void __launch_bounds__(kAttnThreads)
-attn_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
+attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+            const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
             const __nv_bfloat16* __restrict__ V, const int32_t* __restrict__ lens,
             const int32_t* __restrict__ idx, const int32_t* __restrict__ kreq, int k_max,
             int block, int Hkv, int Ncap, float scale_log2, int S, float* __restrict__ part,
             unsigned* __restrict__ counters, float* __restrict__ O, unsigned* __restrict__ flag) {
     using Cfg = AttnCfg<G>;
-    extern __shared__ __align__(128) unsigned char smem[];
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    // 1024-byte aligned work area (the swizzled layout needs it)
+    unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     __shared__ int s_row[STAGES][kTileRows];
     __shared__ float s_wm[kAttnWarps][G], s_wl[kAttnWarps][G];
     __shared__ float s_M[G], s_L[G];
     __shared__ float s_Mr[kClusterMax][G], s_Lr[kClusterMax][G];  // cluster path: received (M, L)
     __shared__ int s_last;
     __shared__ __align__(8) uint64_t s_bar[STAGES];
+    __shared__ int s_first[STAGES];  // CONTIG: first cache row of the tile in each stage, or -1
 
     const int s = blockIdx.x, unit = blockIdx.y;
     const int b = unit / Hkv;
@@ -167,7 +178,7 @@ attn_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict
         }
         npos = kb * block;
     }
-    const int chunk = ceil_div(npos, S);
+    const int chunk = CONTIG ? ceil_div(ceil_div(npos, S), kTileRows) * kTileRows : ceil_div(npos, S);
     const int p0 = min(s * chunk, npos), p1 = min(p0 + chunk, npos);
     const int ntiles = ceil_div(p1 - p0, kTileRows);
     const int32_t* iu = idx ? idx + (size_t)unit * k_max : nullptr;
@@ -203,6 +214,48 @@ attn_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict
         const int pos = p0 + t * kTileRows + my_slot;
         return (my_slot < kTileRows && t < ntiles && pos < p1) ? row_of(pos) : -1;
     };
+    // CONTIG: the tile's first cache row (dense: its position; block mode: the
+    // chosen block's first row), or -1 when the block entry is absent
+    auto tile_first = [&](int t) -> int {
+        const int pos0 = p0 + t * kTileRows;
+        if (t >= ntiles) return -1;
+        if (iu == nullptr) return pos0;
+        const int e = iu[pos0 / kTileRows];
+        if (e >= nb) {
+            atomicOr(flag, kFlagBounds);
+            return -1;
+        }
+        return e < 0 ? -1 : e * kTileRows;
+    };
+    // thread 0 issues the tile's four tensor loads (K and V, two 64-dim halves
+    // each); `first` was read ahead of time so the index latency stays hidden
+    auto stage_contig = [&](int t, int first) {
+        if (t >= ntiles) return;
+        const int st = t % STAGES;
+        s_first[st] = first;
+        if (first >= 0) {
+            fence_proxy_async();
+            mbar_arrive_expect_tx(&s_bar[st], 4 * 64 * kTileRows * 2);
+            const unsigned dst = smem_u32(smem + st * kStageBytes);
+            const unsigned bar = smem_u32(&s_bar[st]);
+            const int y = unit * Ncap + first;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                asm volatile(
+                    "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::"r"(
+                        dst + h * 64 * kTileRows * 2),
+                    "l"(&kmap), "r"(h * 64), "r"(y), "r"(bar)
+                    : "memory");
+                asm volatile(
+                    "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::"r"(
+                        dst + 2 * 64 * kTileRows * 2 + h * 64 * kTileRows * 2),
+                    "l"(&vmap), "r"(h * 64), "r"(y), "r"(bar)
+                    : "memory");
+            }
+        } else {
+            mbar_arrive(&s_bar[st]);
+        }
+    };
     auto stage_tile = [&](int t, int row) {
         if (t >= ntiles || my_slot >= kTileRows) return;
         const int st = t % STAGES;
@@ -226,12 +279,21 @@ attn_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict
 
     if (tid == 0) {
 #pragma unroll
-        for (int i = 0; i < STAGES; ++i) mbar_init(&s_bar[i], kTileRows);
+        for (int i = 0; i < STAGES; ++i) mbar_init(&s_bar[i], CONTIG ? 1 : kTileRows);
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
     __syncthreads();
     // the first STAGES tiles: index reads in one round, then every copy
-    {
+    int next_first = -1;  // CONTIG, thread 0: first row of the tile that refills the stage next
+    if constexpr (CONTIG) {
+        if (tid == 0) {
+            int f[STAGES];
+#pragma unroll
+            for (int t = 0; t < STAGES; ++t) f[t] = tile_first(t);
+#pragma unroll
+            for (int t = 0; t < STAGES; ++t) stage_contig(t, f[t]);
+        }
+    } else {
         int pre[STAGES];
 #pragma unroll
         for (int t = 0; t < STAGES; ++t) pre[t] = row_for_tile(t);
@@ -259,12 +321,41 @@ attn_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict
 
     const unsigned sbase = smem_u32(smem);
     for (int t = 0; t < ntiles; ++t) {
+        if (CONTIG && tid == 0) next_first = tile_first(t + STAGES);  // in flight during this tile
         mbar_wait(&s_bar[t % STAGES], (unsigned)(t / STAGES) & 1u, flag);  // tile t has landed
         const int st = t % STAGES;
-        const int tile_rows = min(kTileRows, p1 - p0 - t * kTileRows);
+        int tile_rows = min(kTileRows, p1 - p0 - t * kTileRows);
+        if constexpr (CONTIG) {
+            // the valid rows are a prefix: the range's and the sequence's ends cut it;
+            // an absent block (first < 0) has none and nothing landed
+            const int first = s_first[st];
+            tile_rows = first < 0 ? 0 : max(0, min(tile_rows, len - first));
+            // rows past it hold real cache data, which may be anything: give V
+            // there zeros, since their weight 0 times NaN is NaN
+            const bool zero = tile_rows > 0 && tid >= tile_rows && tid < kTileRows;
+            if (zero) {
+                unsigned char* vrow = smem + st * kStageBytes + 2 * 64 * kTileRows * 2 + tid * 128;
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        *reinterpret_cast<uint4*>(vrow + h * 64 * kTileRows * 2 + 16 * c) = make_uint4(0, 0, 0, 0);
+                fence_proxy_async();  // before the stage's next tensor load overwrites them
+            }
+            __syncthreads();  // every thread, every tile (never a divergent barrier)
+        }
         const int r0 = warp * 16;  // this warp's rows in the tile
         if (r0 < tile_rows) {      // warp-uniform
-            const unsigned kt = sbase + st * kStageBytes, vt = kt + kTileRows * kRowStride;
+            const unsigned kt = sbase + st * kStageBytes;
+            const unsigned vt = kt + (CONTIG ? 2 * 64 * kTileRows * 2 : kTileRows * kRowStride);
+            // byte offset of 16-byte chunk c of tile row r (padded rows, or the
+            // 128-byte swizzle of the TMA tensor loads: two 64-dim halves)
+            auto off = [&](int r, int c) -> unsigned {
+                if constexpr (CONTIG)
+                    return (unsigned)((c >> 3) * 64 * kTileRows * 2 + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+                else
+                    return (unsigned)roff(r, c);
+            };
             // ---- S = Q K^T over this warp's 16 rows (two n-tiles of 8 rows)
             float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
             {
@@ -273,7 +364,7 @@ attn_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
                     uint32_t b0, b1, b2, b3;
-                    ldsm_x4(kt + roff(row, 2 * ks + (m & 1)), b0, b1, b2, b3);
+                    ldsm_x4(kt + off(row, 2 * ks + (m & 1)), b0, b1, b2, b3);
                     mma_bf16(sc[0], qa[ks][0], qa[ks][1], b0, b1);
                     mma_bf16(sc[1], qa[ks][0], qa[ks][1], b2, b3);
                 }
@@ -282,10 +373,10 @@ attn_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict
             float z[4];
             {
                 const int ra = r0 + 2 * t4;  // rows of sc[0][0..1]; sc[1] adds 8
-                const bool v0 = ra < tile_rows && s_row[st][ra] >= 0;
-                const bool v1 = ra + 1 < tile_rows && s_row[st][ra + 1] >= 0;
-                const bool v2 = ra + 8 < tile_rows && s_row[st][ra + 8] >= 0;
-                const bool v3 = ra + 9 < tile_rows && s_row[st][ra + 9] >= 0;
+                const bool v0 = ra < tile_rows && (CONTIG || s_row[st][ra] >= 0);
+                const bool v1 = ra + 1 < tile_rows && (CONTIG || s_row[st][ra + 1] >= 0);
+                const bool v2 = ra + 8 < tile_rows && (CONTIG || s_row[st][ra + 8] >= 0);
+                const bool v3 = ra + 9 < tile_rows && (CONTIG || s_row[st][ra + 9] >= 0);
                 z[0] = v0 ? sc[0][0] * scale_log2 : -INFINITY;
                 z[1] = v1 ? sc[0][1] * scale_log2 : -INFINITY;
                 z[2] = v2 ? sc[1][0] * scale_log2 : -INFINITY;
@@ -322,7 +413,7 @@ attn_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict
 #pragma unroll
                 for (int np = 0; np < 8; ++np) {
                     uint32_t b0, b1, b2, b3;
-                    ldsm_x4_t(vt + roff(row, 2 * np + (m >> 1)), b0, b1, b2, b3);
+                    ldsm_x4_t(vt + off(row, 2 * np + (m >> 1)), b0, b1, b2, b3);
                     mma_bf16(o[2 * np], ph0, ph1, b0, b1);
                     mma_bf16(o[2 * np], pl0, pl1, b0, b1);
                     mma_bf16(o[2 * np + 1], ph0, ph1, b2, b3);
@@ -331,7 +422,10 @@ attn_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict
             }
         }
         __syncthreads();               // every warp is done with this stage
-        stage_tile(t + STAGES, row_for_tile(t + STAGES));  // refill it (nothing past the end)
+        if constexpr (CONTIG) {
+            if (tid == 0) stage_contig(t + STAGES, next_first);  // refill it (nothing past the end)
+        }
+        else stage_tile(t + STAGES, row_for_tile(t + STAGES));
     }
     __syncthreads();
 
@@ -479,10 +573,22 @@ int attn_splits(const Dims& d, int k_max, int block, bool dense) {
     long long rows;
     int s;
     if (dense) {
-        // bandwidth-bound streaming: one wave at one CTA per SM; past 8 splits
-        // the workspace combine (its cost is small next to the stream)
+        // bandwidth-bound streaming at one CTA per SM: the split count that
+        // minimises (waves) x (tiles per CTA + ~2 tiles of fixed cost), so no
+        // second wave runs a handful of CTAs alone; past 8 splits the partials
+        // combine through the workspace (small next to the stream)
         rows = d.Ncap;
-        s = ceil_div(kSms, units);
+        const long long tiles = (rows + kTileRows - 1) / kTileRows;
+        long long best = -1;
+        s = 1;
+        for (int c = 1; c <= kMaxSplits && c <= tiles; ++c) {
+            const long long waves = ((long long)units * c + kSms - 1) / kSms;
+            const long long cost = waves * ((tiles + c - 1) / c + 2);
+            if (best < 0 || cost < best) {
+                best = cost;
+                s = c;
+            }
+        }
     } else {
         // latency-bound gather: splits of at most kRing tiles (all in flight at
         // once), one tile each where the GPU has room, at most 8 splits (one
@@ -509,11 +615,21 @@ static int g_attn_configured[64];
 
 bool attn_uses_cluster(int splits) { return splits <= kClusterMax; }
 
-template <int G, int STAGES, bool CLUSTER>
-static cudaError_t attn_launch_g(dim3 grid, cudaStream_t st, const __nv_bfloat16* q, const __nv_bfloat16* k,
-                                 const __nv_bfloat16* v, const int32_t* lens, const int32_t* idx,
-                                 const int32_t* kreq, int k_max, int block, const Dims& d, float sl2,
-                                 int splits, float* partials, unsigned* counters, float* O, unsigned* flag) {
+struct AttnArgs {
+    CUtensorMap kmap, vmap;
+    const __nv_bfloat16 *q, *k, *v;
+    const int32_t *lens, *idx, *kreq;
+    int k_max, block, Hkv, Ncap;
+    float sl2;
+    int splits;
+    float* partials;
+    unsigned* counters;
+    float* O;
+    unsigned* flag;
+};
+
+template <int G, int STAGES, bool CLUSTER, bool CONTIG>
+static cudaError_t attn_launch_g(dim3 grid, cudaStream_t st, const AttnArgs& a) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = dim3(kAttnThreads);
@@ -521,52 +637,73 @@ static cudaError_t attn_launch_g(dim3 grid, cudaStream_t st, const __nv_bfloat16
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = CLUSTER ? (unsigned)splits : 1u;
+    attr[0].val.clusterDim.x = CLUSTER ? (unsigned)a.splits : 1u;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     attr[1] = pdl_attr();
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, attn_kernel<G, STAGES, CLUSTER>, q, k, v, lens, idx, kreq, k_max, block,
-                              d.Hkv, d.Ncap, sl2, splits, partials, counters, O, flag);
+    return cudaLaunchKernelEx(&cfg, attn_kernel<G, STAGES, CLUSTER, CONTIG>, a.kmap, a.vmap, a.q, a.k, a.v, a.lens,
+                              a.idx, a.kreq, a.k_max, a.block, a.Hkv, a.Ncap, a.sl2, a.splits, a.partials, a.counters,
+                              a.O, a.flag);
 }
 
-template <int G, int STAGES, bool CLUSTER>
+template <int G, int STAGES, bool CLUSTER, bool CONTIG>
 static cudaError_t attn_configure_one() {
-    cudaError_t e = cudaFuncSetAttribute(attn_kernel<G, STAGES, CLUSTER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    const void* f = (const void*)attn_kernel<G, STAGES, CLUSTER, CONTIG>;
+    cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          AttnCfg<G>::smem_bytes(STAGES, CLUSTER));
-    if (e == cudaSuccess && CLUSTER)
-        e = cudaFuncSetAttribute(attn_kernel<G, STAGES, CLUSTER>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e == cudaSuccess && CLUSTER) e = cudaFuncSetAttribute(f, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     return e;
 }
 
 template <int G>
 static cudaError_t attn_configure() {
-    cudaError_t e = attn_configure_one<G, 1, true>();
-    if (e == cudaSuccess) e = attn_configure_one<G, kRing, true>();
-    if (e == cudaSuccess) e = attn_configure_one<G, 1, false>();
-    if (e == cudaSuccess) e = attn_configure_one<G, kRing, false>();
+    cudaError_t e = cudaSuccess;
+    if (e == cudaSuccess) e = attn_configure_one<G, 1, true, false>();
+    if (e == cudaSuccess) e = attn_configure_one<G, kRing, true, false>();
+    if (e == cudaSuccess) e = attn_configure_one<G, 1, false, false>();
+    if (e == cudaSuccess) e = attn_configure_one<G, kRing, false, false>();
+    if (e == cudaSuccess) e = attn_configure_one<G, 1, true, true>();
+    if (e == cudaSuccess) e = attn_configure_one<G, kRing, true, true>();
+    if (e == cudaSuccess) e = attn_configure_one<G, 1, false, true>();
+    if (e == cudaSuccess) e = attn_configure_one<G, kRing, false, true>();
     return e;
 }
 
+template <int G, bool CONTIG>
+static cudaError_t attn_dispatch2(bool one_tile, bool cluster, dim3 grid, cudaStream_t st, const AttnArgs& a) {
+    if (cluster)
+        return one_tile ? attn_launch_g<G, 1, true, CONTIG>(grid, st, a) : attn_launch_g<G, kRing, true, CONTIG>(grid, st, a);
+    return one_tile ? attn_launch_g<G, 1, false, CONTIG>(grid, st, a) : attn_launch_g<G, kRing, false, CONTIG>(grid, st, a);
+}
+
 template <int G>
-static cudaError_t attn_dispatch(bool one_tile, bool cluster, dim3 grid, cudaStream_t st, const __nv_bfloat16* q,
-                                 const __nv_bfloat16* k, const __nv_bfloat16* v, const int32_t* lens,
-                                 const int32_t* idx, const int32_t* kreq, int k_max, int block, const Dims& d,
-                                 float sl2, int splits, float* partials, unsigned* counters, float* O,
-                                 unsigned* flag) {
-    if (cluster) {
-        if (one_tile)
-            return attn_launch_g<G, 1, true>(grid, st, q, k, v, lens, idx, kreq, k_max, block, d, sl2, splits,
-                                             partials, counters, O, flag);
-        return attn_launch_g<G, kRing, true>(grid, st, q, k, v, lens, idx, kreq, k_max, block, d, sl2, splits,
-                                         partials, counters, O, flag);
+static cudaError_t attn_dispatch(bool contig, bool one_tile, bool cluster, dim3 grid, cudaStream_t st,
+                                 const AttnArgs& a) {
+    return contig ? attn_dispatch2<G, true>(one_tile, cluster, grid, st, a)
+                  : attn_dispatch2<G, false>(one_tile, cluster, grid, st, a);
+}
+
+// tensor map over a [units * Ncap rows] x [128 dims] bf16 cache, box 64 dims x 128 rows, 128-byte swizzle
+static cudaError_t make_row_map(CUtensorMap* map, const void* base, const Dims& d) {
+    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    if (!encode) {
+        cudaDriverEntryPointQueryResult q;
+        void* fn = nullptr;
+        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+        if (e != cudaSuccess) return e;
+        if (q != cudaDriverEntryPointSuccess || fn == nullptr) return cudaErrorNotSupported;
+        encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     }
-    if (one_tile)
-        return attn_launch_g<G, 1, false>(grid, st, q, k, v, lens, idx, kreq, k_max, block, d, sl2, splits,
-                                          partials, counters, O, flag);
-    return attn_launch_g<G, kRing, false>(grid, st, q, k, v, lens, idx, kreq, k_max, block, d, sl2, splits, partials,
-                                      counters, O, flag);
+    const cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)d.units() * (cuuint64_t)d.Ncap};
+    const cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)kTileRows};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 cudaError_t launch_attn(const void* Q, const void* K, const void* V, const int32_t* lens,
@@ -592,18 +729,41 @@ cudaError_t launch_attn(const void* Q, const void* K, const void* V, const int32
         const long long nbmax = block == 1 ? d.Ncap : ceil_div(d.Ncap, block);
         rows = (long long)(k_max < nbmax ? k_max : nbmax) * block;
     }
-    const bool one_tile = (rows + splits - 1) / splits <= kTileRows;
+    // whole 128-row tiles of consecutive cache rows: full attention, or 128-token blocks
+    const bool contig = idx == nullptr || block == kTileRows;
+    const long long per_split = contig ? ((rows + splits - 1) / splits + kTileRows - 1) / kTileRows * kTileRows
+                                       : (rows + splits - 1) / splits;
+    const bool one_tile = per_split <= kTileRows;
     const bool cluster = attn_uses_cluster(splits);
+    AttnArgs a;
+    memset(&a.kmap, 0, sizeof a.kmap);
+    memset(&a.vmap, 0, sizeof a.vmap);
+    if (contig) {
+        if ((e = make_row_map(&a.kmap, K, d)) != cudaSuccess) return e;
+        if ((e = make_row_map(&a.vmap, V, d)) != cudaSuccess) return e;
+    }
+    a.q = static_cast<const __nv_bfloat16*>(Q);
+    a.k = static_cast<const __nv_bfloat16*>(K);
+    a.v = static_cast<const __nv_bfloat16*>(V);
+    a.lens = lens;
+    a.idx = idx;
+    a.kreq = kreq;
+    a.k_max = k_max;
+    a.block = block;
+    a.Hkv = d.Hkv;
+    a.Ncap = d.Ncap;
+    a.sl2 = scale * kLog2e;
+    a.splits = splits;
+    a.partials = partials;
+    a.counters = counters;
+    a.O = O;
+    a.flag = flag;
     dim3 grid(splits, d.units());
-    const float sl2 = scale * kLog2e;
-    const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(Q);
-    const __nv_bfloat16* k = static_cast<const __nv_bfloat16*>(K);
-    const __nv_bfloat16* v = static_cast<const __nv_bfloat16*>(V);
     switch (d.G) {
-        case 1: e = attn_dispatch<1>(one_tile, cluster, grid, st, q, k, v, lens, idx, kreq, k_max, block, d, sl2, splits, partials, counters, O, flag); break;
-        case 2: e = attn_dispatch<2>(one_tile, cluster, grid, st, q, k, v, lens, idx, kreq, k_max, block, d, sl2, splits, partials, counters, O, flag); break;
-        case 4: e = attn_dispatch<4>(one_tile, cluster, grid, st, q, k, v, lens, idx, kreq, k_max, block, d, sl2, splits, partials, counters, O, flag); break;
-        case 8: e = attn_dispatch<8>(one_tile, cluster, grid, st, q, k, v, lens, idx, kreq, k_max, block, d, sl2, splits, partials, counters, O, flag); break;
+        case 1: e = attn_dispatch<1>(contig, one_tile, cluster, grid, st, a); break;
+        case 2: e = attn_dispatch<2>(contig, one_tile, cluster, grid, st, a); break;
+        case 4: e = attn_dispatch<4>(contig, one_tile, cluster, grid, st, a); break;
+        case 8: e = attn_dispatch<8>(contig, one_tile, cluster, grid, st, a); break;
         default: return cudaErrorInvalidValue;
     }
     note_launch();

@@ -1,15 +1,15 @@
-// score.cu -- step 1 of the decode path: score every cached key (or block mean)
-// against the current query group, and the block summaries of block mode.
+// score.cu -- block mode's step 1: score every block's mean key against the
+// current query group, and the block summaries (the means) themselves.  The
+// per-token scan of token mode is score_tc.cu.
 //
 // "inference-time context sparsity: illusion or opportunity?", sec. 2 (oracle
-// Top-K): the k most important tokens are chosen exactly; importance here is
-// the scaled logit, reduced over the GQA group by max.  "Flash Attention vs
-// Sparse Attention", DSA stage 1: the indexer pass that reads the whole context.
+// Top-K): importance is the scaled logit, reduced over the GQA group by max.
 // HyLRA sec. 2.4: 128-token blocks, scored through their mean key.
 //
-// The pass is bound by HBM: every K byte is read once.  Each warp streams rows
-// with coalesced 16-byte loads (a half-warp per 256-byte row, 8 dims per lane),
-// keeps the g query heads of the kv-head in registers, so one K read serves the
+// The means are fp32 rows (512 B) and 128x fewer than the keys, so this is a
+// short HBM-bound pass that must not run out of CTAs: each warp takes one step
+// of rows with coalesced 16-byte loads (a half-warp per row, 8 dims per lane),
+// keeps the g query heads of the kv-head in registers, so one read serves the
 // whole GQA group, and reduces the per-lane partial dot products with a
 // reduce-scatter across the half-warp.
 #include "common.cuh"
@@ -19,16 +19,15 @@ namespace tsa {
 
 constexpr int kScoreThreads = 256;
 constexpr int kScoreWarps = kScoreThreads / 32;
-constexpr int kScoreSteps = 8;  // warp steps per CTA
 
-template <int G, bool kMeans>
+template <int G>
 __global__ void __launch_bounds__(kScoreThreads)
-score_kernel(const __nv_bfloat16* __restrict__ Q, const void* __restrict__ keys,
+score_kernel(const __nv_bfloat16* __restrict__ Q, const float* __restrict__ means,
              const int32_t* __restrict__ lens, int Hkv, int Ncap, int rows_cap, int block,
              float scale, float* __restrict__ scores, unsigned* __restrict__ flag) {
-    constexpr int R = 16 / G;          // rows per half-warp per step (R*G = 16 partial dots)
-    constexpr int kRowsStep = 2 * R;   // rows per warp per step
-    constexpr int kRowsCta = kRowsStep * kScoreWarps * kScoreSteps;
+    constexpr int R = 16 / G;          // rows per half-warp (R*G = 16 partial dots)
+    constexpr int kRowsWarp = 2 * R;   // rows per warp
+    constexpr int kRowsCta = kRowsWarp * kScoreWarps;
     const int unit = blockIdx.y;
     const int b = unit / Hkv, kvh = unit - b * Hkv;
     griddep_wait();
@@ -38,12 +37,11 @@ score_kernel(const __nv_bfloat16* __restrict__ Q, const void* __restrict__ keys,
         if (threadIdx.x == 0) atomicOr(flag, kFlagBounds);
         len = len < 0 ? 0 : Ncap;
     }
-    const int n = kMeans ? ceil_div(len, block) : len;
-    const int row0 = blockIdx.x * kRowsCta;
-    if (row0 >= n) return;
-
+    const int n = ceil_div(len, block);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int half = lane >> 4, c = lane & 15;
+    const int base = blockIdx.x * kRowsCta + warp * kRowsWarp;
+    if (base >= n) return;
 
     float q[G][8];
 #pragma unroll
@@ -51,66 +49,38 @@ score_kernel(const __nv_bfloat16* __restrict__ Q, const void* __restrict__ keys,
         const __nv_bfloat16* qp = Q + ((size_t)(b * Hkv + kvh) * G + h) * kD + 8 * c;
         unpack8(*reinterpret_cast<const uint4*>(qp), q[h]);
     }
-    float* out = scores + (size_t)unit * rows_cap;
-
-    for (int it = 0; it < kScoreSteps; ++it) {
-        const int base = row0 + (it * kScoreWarps + warp) * kRowsStep;
-        if (base >= n) break;
-        float v[16];
-        if constexpr (!kMeans) {
-            const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(keys) + (size_t)unit * Ncap * kD;
-            uint4 raw[R];
+    const float* kb = means + (size_t)unit * rows_cap * kD;
+    uint4 raw[R][2];
 #pragma unroll
-            for (int r = 0; r < R; ++r) {
-                const int row = base + 2 * r + half;
-                raw[r] = row < n ? ld_stream(kb + (size_t)row * kD + 8 * c) : make_uint4(0, 0, 0, 0);
-            }
-#pragma unroll
-            for (int r = 0; r < R; ++r) {
-                float kf[8];
-                unpack8(raw[r], kf);
-#pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    float s = 0.f;
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) s = fmaf(kf[e], q[h][e], s);
-                    v[r * G + h] = s;
-                }
-            }
-        } else {
-            const float* kb = static_cast<const float*>(keys) + (size_t)unit * rows_cap * kD;
-            uint4 raw[R][2];
-#pragma unroll
-            for (int r = 0; r < R; ++r) {
-                const int row = base + 2 * r + half;
-                const float* p = kb + (size_t)row * kD + 8 * c;
-                raw[r][0] = row < n ? ld_stream(p) : make_uint4(0, 0, 0, 0);
-                raw[r][1] = row < n ? ld_stream(p + 4) : make_uint4(0, 0, 0, 0);
-            }
-#pragma unroll
-            for (int r = 0; r < R; ++r) {
-                const float kf[8] = {__uint_as_float(raw[r][0].x), __uint_as_float(raw[r][0].y),
-                                     __uint_as_float(raw[r][0].z), __uint_as_float(raw[r][0].w),
-                                     __uint_as_float(raw[r][1].x), __uint_as_float(raw[r][1].y),
-                                     __uint_as_float(raw[r][1].z), __uint_as_float(raw[r][1].w)};
-#pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    float s = 0.f;
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) s = fmaf(kf[e], q[h][e], s);
-                    v[r * G + h] = s;
-                }
-            }
-        }
-        // lane c of each half now gets the full dot of (row 2*(c/G)+half, head c%G)
-        halfwarp_reduce_scatter16(v, c);
-        float m = v[0];
-#pragma unroll
-        for (int o = 1; o < G; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        const int row = base + 2 * (c / G) + half;
-        // scale > 0, so scale * max_h(z_h) = max_h(scale * z_h) exactly (rounding is monotone)
-        if ((c % G) == 0 && row < n) out[row] = m * scale;
+    for (int r = 0; r < R; ++r) {
+        const int row = base + 2 * r + half;
+        const float* p = kb + (size_t)row * kD + 8 * c;
+        raw[r][0] = row < n ? ld_stream(p) : make_uint4(0, 0, 0, 0);
+        raw[r][1] = row < n ? ld_stream(p + 4) : make_uint4(0, 0, 0, 0);
     }
+    float v[16];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const float kf[8] = {__uint_as_float(raw[r][0].x), __uint_as_float(raw[r][0].y),
+                             __uint_as_float(raw[r][0].z), __uint_as_float(raw[r][0].w),
+                             __uint_as_float(raw[r][1].x), __uint_as_float(raw[r][1].y),
+                             __uint_as_float(raw[r][1].z), __uint_as_float(raw[r][1].w)};
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            float s = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) s = fmaf(kf[e], q[h][e], s);
+            v[r * G + h] = s;
+        }
+    }
+    // lane c of each half now gets the full dot of (row 2*(c/G)+half, head c%G)
+    halfwarp_reduce_scatter16(v, c);
+    float m = v[0];
+#pragma unroll
+    for (int o = 1; o < G; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const int row = base + 2 * (c / G) + half;
+    // scale > 0, so scale * max_h(z_h) = max_h(scale * z_h) exactly (rounding is monotone)
+    if ((c % G) == 0 && row < n) scores[(size_t)unit * rows_cap + row] = m * scale;
 }
 
 // One CTA per (block, unit); thread t owns dimension t and sums the block's
@@ -135,39 +105,32 @@ block_mean_kernel(const __nv_bfloat16* __restrict__ K, const int32_t* __restrict
     Kmean[((size_t)unit * NB + beta) * kD + t] = s / (float)(t1 - t0);
 }
 
-template <bool kMeans>
-static cudaError_t score_dispatch(const void* Q, const void* keys, const int32_t* lens,
-                                  const Dims& d, int block, float scale, float* scores,
-                                  unsigned* flag, cudaStream_t st) {
+cudaError_t launch_score(const void* Q, const void* keys, const int32_t* lens, const Dims& d,
+                         int block, float scale, float* scores, unsigned* flag, cudaStream_t st) {
+    if (d.units() == 0 || d.Ncap == 0) return cudaSuccess;
+    if (block == 1) return launch_score_tc(Q, keys, lens, d, scale, scores, flag, st);
     const int rows_cap = rows_cap_of(d, block);
-    const int rows_cta = 2 * (16 / d.G) * kScoreWarps * kScoreSteps;
-    dim3 grid(ceil_div(rows_cap, rows_cta), d.units());
-    const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(Q);
+    const int rows_cta = 2 * (16 / d.G) * kScoreWarps;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
+    cfg.gridDim = dim3(ceil_div(rows_cap, rows_cta), d.units());
     cfg.blockDim = dim3(kScoreThreads);
     cfg.stream = st;
     cudaLaunchAttribute attr[1] = {pdl_attr()};
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(Q);
+    const float* m = static_cast<const float*>(keys);
     cudaError_t e;
     switch (d.G) {
-        case 1: e = cudaLaunchKernelEx(&cfg, score_kernel<1, kMeans>, q, keys, lens, d.Hkv, d.Ncap, rows_cap, block, scale, scores, flag); break;
-        case 2: e = cudaLaunchKernelEx(&cfg, score_kernel<2, kMeans>, q, keys, lens, d.Hkv, d.Ncap, rows_cap, block, scale, scores, flag); break;
-        case 4: e = cudaLaunchKernelEx(&cfg, score_kernel<4, kMeans>, q, keys, lens, d.Hkv, d.Ncap, rows_cap, block, scale, scores, flag); break;
-        case 8: e = cudaLaunchKernelEx(&cfg, score_kernel<8, kMeans>, q, keys, lens, d.Hkv, d.Ncap, rows_cap, block, scale, scores, flag); break;
+        case 1: e = cudaLaunchKernelEx(&cfg, score_kernel<1>, q, m, lens, d.Hkv, d.Ncap, rows_cap, block, scale, scores, flag); break;
+        case 2: e = cudaLaunchKernelEx(&cfg, score_kernel<2>, q, m, lens, d.Hkv, d.Ncap, rows_cap, block, scale, scores, flag); break;
+        case 4: e = cudaLaunchKernelEx(&cfg, score_kernel<4>, q, m, lens, d.Hkv, d.Ncap, rows_cap, block, scale, scores, flag); break;
+        case 8: e = cudaLaunchKernelEx(&cfg, score_kernel<8>, q, m, lens, d.Hkv, d.Ncap, rows_cap, block, scale, scores, flag); break;
         default: return cudaErrorInvalidValue;
     }
     note_launch();
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
-}
-
-cudaError_t launch_score(const void* Q, const void* keys, const int32_t* lens, const Dims& d,
-                         int block, float scale, float* scores, unsigned* flag, cudaStream_t st) {
-    if (d.units() == 0 || d.Ncap == 0) return cudaSuccess;
-    if (block == 1) return launch_score_tc(Q, keys, lens, d, scale, scores, flag, st);
-    return score_dispatch<true>(Q, keys, lens, d, block, scale, scores, flag, st);
 }
 
 cudaError_t launch_block_summarize(const void* K, const int32_t* lens, const Dims& d, int block,
