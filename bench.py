@@ -305,10 +305,44 @@ def run_ours(args, rank, world, dev):
     return res
 
 
+class L2Flush:
+    """Reads a 256 MB buffer (twice L2) into one scalar: afterwards L2 holds only
+    clean lines of that buffer, so the next launch reads its data from HBM."""
+
+    def __init__(self, dev):
+        self.buf = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+        self.out = torch.empty((), dtype=torch.float32, device=dev)
+
+    def __call__(self):
+        torch.sum(self.buf, dim=0, out=self.out)
+
+
+def graph_us(fn, stream, reps):
+    """Device time of `reps` calls of fn captured in one CUDA graph, per call."""
+    with torch.cuda.stream(stream):
+        fn()
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for _ in range(reps):
+            fn()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        g.replay()
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+    stream.synchronize()
+    del g
+    return e0.elapsed_time(e1) * 1e3 / reps
+
+
 def stage_times(tsa, w, plan, layers, Kmean, ws, kreq_t, idx, O, stream, reps=10):
-    """Average device time of each stage, each launched `reps` times back to back in a
-    CUDA graph.  The score stage streams more than L2 per launch; the top-k and the
-    attention stages read L2-sized data, so their repeated launches run L2-warm."""
+    """Device time of each stage two ways, each in a CUDA graph of `reps` launches:
+    back to back ("warm": the top-k and attention stages read L2-sized data, so
+    their repeats hit L2), and each launch after an L2 flush, minus the flushes
+    alone ("cold": HBM reads, as inside a step; it includes the launch latency
+    that programmatic dependent launch hides inside a step)."""
     from top_sparse_attention_02_b200 import binding as _b
 
     shape = _b.shape_of(layers[0].Q, layers[0].K)
@@ -333,28 +367,18 @@ def stage_times(tsa, w, plan, layers, Kmean, ws, kreq_t, idx, O, stream, reps=10
         else:
             calls[f"L{li}_attn"] = lambda L=L, li=li: tsa.sparse_decode_attn(
                 L.Q, L.K, L.V, L.seq_lens, None, None, 0, 1, w.scale, O[li], ws, stream)
-    out = {}
+    flush = L2Flush(layers[0].Q.device)
+    flush_us = graph_us(flush, stream, reps)
+    warm, cold = {}, {}
     for name, fn in calls.items():
-        with torch.cuda.stream(stream):
-            fn()
-        stream.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            for _ in range(reps):
-                fn()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            g.replay()
-            e0.record(stream)
-            g.replay()
-            e1.record(stream)
-        stream.synchronize()
-        out[name] = e0.elapsed_time(e1) * 1e3 / reps
-        del g
+        warm[name] = graph_us(fn, stream, reps)
+        cold[name] = graph_us(lambda fn=fn: (flush(), fn()), stream, reps) - flush_us
+    del flush
     sel = [li for li, m in enumerate(w.route) if m == tsa.SELECT]
-    out["score_us"] = statistics.mean(out[f"L{li}_score"] for li in sel) if sel else float("nan")
-    out["note"] = "each stage alone, %d launches back to back in a CUDA graph" % reps
-    return out
+    return {"warm": warm, "cold": cold,
+            "score_us": statistics.mean(warm[f"L{li}_score"] for li in sel) if sel else float("nan"),
+            "note": f"per launch, {reps} launches per CUDA graph; warm = back to back, cold = after an L2 "
+                    "flush (minus the flush alone)"}
 
 
 def copy_probe(tsa, dev, stream, nbytes=2 << 30):
@@ -376,7 +400,9 @@ def copy_probe(tsa, dev, stream, nbytes=2 << 30):
 def gather_probe(tsa, w, plan, layers, idx, ws, stream, reps=10):
     """Random-row gather ceiling on the attention stage's own rows: the rows layer 0
     selected, fetched from a reuse layer's K and V by tsa_hbm_gather (bulk copies
-    into shared memory, nothing kept).  Returns GB/s over the bytes fetched."""
+    into shared memory, nothing kept), each pair of launches after an L2 flush
+    (minus the flush alone), as the cold attention stage is timed.  Returns GB/s
+    over the bytes fetched."""
     sel = [li for li, m in enumerate(w.route) if m == 1]
     if not sel or w.block != 1:
         return None
@@ -386,40 +412,34 @@ def gather_probe(tsa, w, plan, layers, idx, ws, stream, reps=10):
     rows = (ix + base)[ix >= 0].to(torch.int32).contiguous()
     K2 = src_layer.K.view(torch.uint8).reshape(-1)
     V2 = src_layer.V.view(torch.uint8).reshape(-1)
-    with torch.cuda.stream(stream):
+
+    def both():
         tsa.hbm_gather(K2, rows, ws, stream)
         tsa.hbm_gather(V2, rows, ws, stream)
-    stream.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=stream):
-        for _ in range(reps):
-            tsa.hbm_gather(K2, rows, ws, stream)
-            tsa.hbm_gather(V2, rows, ws, stream)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        g.replay()
-        e0.record(stream)
-        g.replay()
-        e1.record(stream)
-    stream.synchronize()
+
+    flush = L2Flush(ix.device)
+    us = graph_us(lambda: (flush(), both()), stream, reps) - graph_us(flush, stream, reps)
+    warm_us = graph_us(both, stream, reps)
+    del flush
     tsa.check_device_status(ws, stream)
-    us = e0.elapsed_time(e1) * 1e3 / reps
     nbytes = 2 * rows.numel() * 256
-    del g
     return {"gbs": nbytes / (us * 1e-6) / 1e9, "us": us, "bytes": nbytes,
-            "rows": "the K and V rows layer 0 selected, in another layer's cache"}
+            "warm_gbs": nbytes / (warm_us * 1e-6) / 1e9,
+            "rows": "the K and V rows layer 0 selected, in another layer's cache; after an L2 flush"}
 
 
 def attn_roofline(w, plan, stages, gather):
     """The attention stage against the random-row gather ceiling measured in this run."""
     if gather is None:
         return None
-    reuse = [k for k in stages if k.endswith("_attn") and not k.startswith("L0")]
-    us = statistics.mean(stages[k] for k in reuse) if reuse else stages.get("L0_attn")
+    cold = stages["cold"]
+    reuse = [k for k in cold if k.endswith("_attn") and not k.startswith("L0")]
+    us = statistics.mean(cold[k] for k in reuse) if reuse else cold.get("L0_attn")
     achieved = plan.bytes["gather"] / (us * 1e-6) / 1e9
     return {"kernel": "attn_kernel (one reuse layer)", "bound": "hbm random-row gather",
             "achieved": achieved, "peak": gather["gbs"], "unit": "GB/s", "frac": achieved / gather["gbs"],
-            "peak_source": "tsa_hbm_gather on the same rows in this run", "algorithmic_bytes_per_launch":
+            "peak_source": "tsa_hbm_gather on the same rows in this run, both timed after an L2 flush",
+            "algorithmic_bytes_per_launch":
             plan.bytes["gather"]}
 
 

@@ -76,6 +76,24 @@ def test_topk_ties_signed_zeros_and_duplicates(cuda_dev):
     _topk_case(cuda_dev, S2, [5000], [100], 100)
 
 
+def test_topk_many_units_and_wide_clusters(cuda_dev):
+    """Launch shapes of the top-k: many units, a unit wider than 8 slices (a
+    non-portable cluster of 16), and exact ties across a cluster of 3 (the
+    boundary bin overflows rank 0's buffer)."""
+    rng = np.random.default_rng(23)
+    S = rng.standard_normal((40, 8, 20000))
+    lens = rng.integers(1, 20001, size=40).tolist()
+    kreq = [int(x) for x in rng.integers(1, 70, size=40)]
+    _topk_case(cuda_dev, S, lens, kreq, 69, Hq=32)
+    S = rng.standard_normal((1, 1, 250000))
+    for k in (1, 6000, 249999):
+        _topk_case(cuda_dev, S, [250000], [k], k, Hq=4)
+    S = np.zeros((2, 1, 40000))
+    S[1, 0, 20000:] = 1.0
+    for k in (5, 12345, 30000):
+        _topk_case(cuda_dev, S, [40000, 39000], [k, k], k, Hq=2)
+
+
 def test_topk_ragged_per_sequence_k(cuda_dev):
     rng = np.random.default_rng(11)
     B, Hkv, rows = 6, 3, 9000

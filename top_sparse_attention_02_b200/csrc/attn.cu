@@ -28,16 +28,15 @@
 //               bits; V fragments by ldmatrix.trans).
 // tcgen05's smallest M is 64, so there 87-94% of every MMA would be padding;
 // the m16 warp MMA fits a GQA group.  The 8 warps are merged at the end into
-// the CTA's partial (M, L, acc[128]) per head.  With at most 8 splits per unit
-// the splits of a unit form one thread-block cluster: each CTA pushes the slices
-// of its partial to the CTAs that own those output slices (posted
-// distributed-shared-memory stores), one cluster barrier, and each CTA combines
-// its slice locally (no scratch).  Clusters stay at <= 8 CTAs: on B200 only 7
-// clusters of 16 are co-resident, so 8 units of 16 would run in two waves.
-// With more splits (few units, or a long dense range)
-// each CTA writes its partial to the workspace and the last CTA of the unit to
-// arrive (an atomic counter in the workspace, reset by that CTA) combines the
-// partials into O.
+// the CTA's partial (M, L, acc[128]) per head.  When a unit has at most 8
+// splits and every unit's cluster can be resident at once, the splits of a unit
+// form one thread-block cluster: each CTA pushes the slices of its partial to
+// the CTAs that own those output slices (posted distributed-shared-memory
+// stores), one cluster barrier, and each CTA combines its slice locally (no
+// scratch).  Otherwise (more splits, or more clusters than fit: a B200 holds
+// only 15 clusters of 8 CTAs of ~226 KB) each CTA writes its partial to the
+// workspace and the last CTA of the unit to arrive (an atomic counter in the
+// workspace, reset by that CTA) combines the partials into O.
 #include <cooperative_groups.h>
 #include <cstring>
 #include <cuda.h>
@@ -590,15 +589,15 @@ int attn_splits(const Dims& d, int k_max, int block, bool dense) {
             }
         }
     } else {
-        // latency-bound gather: splits of at most kRing tiles (all in flight at
-        // once), one tile each where the GPU has room, at most 8 splits (one
-        // cluster) unless fewer than 4 units would leave most SMs idle
+        // latency-bound gather: one tile per split where the GPU has room
+        // (a wave of at most one CTA per SM), else longer splits whose first
+        // kRing tiles are all in flight at once; whether the splits of a unit
+        // combine in a cluster is decided at launch (attn_cluster_fits)
         const long long nbmax = block == 1 ? d.Ncap : ceil_div(d.Ncap, block);
         rows = (long long)(k_max < nbmax ? k_max : nbmax) * block;
         s = (int)((rows + kTileRows - 1) / kTileRows);
         const int room = kSms / units > 1 ? kSms / units : 1;
         if (s > room) s = room;
-        if (s > kClusterMax && units >= 4) s = kClusterMax;
     }
     const long long smax = (rows + 31) / 32;  // at least 32 positions per split
     if (s > smax) s = (int)smax;
@@ -613,7 +612,61 @@ size_t attn_partials_floats(const Dims& d, int splits) {
 
 static int g_attn_configured[64];
 
-bool attn_uses_cluster(int splits) { return splits <= kClusterMax; }
+// Clusters of S CTAs need S free SMs in one GPC at once: with ~226 KB of shared
+// memory per CTA a B200 holds only 15 clusters of 8 (not 148 / 8), and a 16th
+// would wait for a whole wave.  The count comes from the occupancy API, per
+// device and kernel configuration, and the cluster combine is used only when
+// every unit's cluster is co-resident; otherwise the splits combine through the
+// workspace (sized for them in either case).
+static int g_max_clusters[64][4][2][2][kClusterMax + 1];  // dev, log2 G, one-tile, contig, S; 0 = unknown
+
+template <int G, int STAGES, bool CONTIG>
+static int max_active_clusters(int S) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)S, 1);
+    cfg.blockDim = dim3(kAttnThreads);
+    cfg.dynamicSmemBytes = AttnCfg<G>::smem_bytes(STAGES, true);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)S;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, attn_kernel<G, STAGES, true, CONTIG>, &cfg) != cudaSuccess) {
+        cudaGetLastError();  // clear it: the workspace combine is always available
+        return -1;
+    }
+    return n;
+}
+
+template <int G>
+static bool attn_cluster_fits_g(int dev, bool one_tile, bool contig, int S, int units) {
+    const int lg = G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : 3;
+    int& slot = g_max_clusters[dev][lg][one_tile][contig][S];
+    if (slot == 0) {
+        int n;
+        if (one_tile) n = contig ? max_active_clusters<G, 1, true>(S) : max_active_clusters<G, 1, false>(S);
+        else n = contig ? max_active_clusters<G, kRing, true>(S) : max_active_clusters<G, kRing, false>(S);
+        slot = n;
+    }
+    return slot > 0 && units <= slot;
+}
+
+static bool attn_cluster_fits(int G, bool one_tile, bool contig, int S, int units) {
+    if (S > kClusterMax) return false;
+    if (S == 1) return true;  // a cluster of one: no co-scheduling constraint
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    switch (G) {
+        case 1: return attn_cluster_fits_g<1>(dev, one_tile, contig, S, units);
+        case 2: return attn_cluster_fits_g<2>(dev, one_tile, contig, S, units);
+        case 4: return attn_cluster_fits_g<4>(dev, one_tile, contig, S, units);
+        case 8: return attn_cluster_fits_g<8>(dev, one_tile, contig, S, units);
+        default: return false;
+    }
+}
 
 struct AttnArgs {
     CUtensorMap kmap, vmap;
@@ -734,7 +787,7 @@ cudaError_t launch_attn(const void* Q, const void* K, const void* V, const int32
     const long long per_split = contig ? ((rows + splits - 1) / splits + kTileRows - 1) / kTileRows * kTileRows
                                        : (rows + splits - 1) / splits;
     const bool one_tile = per_split <= kTileRows;
-    const bool cluster = attn_uses_cluster(splits);
+    const bool cluster = attn_cluster_fits(d.G, one_tile, contig, splits, d.units());
     AttnArgs a;
     memset(&a.kmap, 0, sizeof a.kmap);
     memset(&a.vmap, 0, sizeof a.vmap);
