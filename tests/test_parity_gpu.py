@@ -94,6 +94,22 @@ def test_topk_many_units_and_wide_clusters(cuda_dev):
         _topk_case(cuda_dev, S, [40000, 39000], [k, k], k, Hq=2)
 
 
+def test_topk_one_cta_per_unit_ties_and_overflow(cuda_dev):
+    """The one-CTA-per-unit top-k (many units, or units of <= 8192 rows): heavy
+    exact ties, where the candidate list overflows and every later pass streams
+    the scores again, and k close to the unit's length."""
+    rng = np.random.default_rng(29)
+    S = rng.integers(-2, 3, size=(2, 2, 6000)).astype(np.float64)
+    S[0, 1] = 0.0
+    S[1, 0, ::5] = -0.0
+    for k in (1, 10, 1234, 5999):
+        _topk_case(cuda_dev, S, [6000, 4321], [k, k], k, Hq=4)
+    S = rng.integers(-1, 2, size=(20, 8, 3000)).astype(np.float64)  # 160 units
+    lens = rng.integers(1, 3001, size=20).tolist()
+    kreq = [int(x) for x in rng.integers(1, 3001, size=20)]
+    _topk_case(cuda_dev, S, lens, kreq, 3000, Hq=16)
+
+
 def test_topk_ragged_per_sequence_k(cuda_dev):
     rng = np.random.default_rng(11)
     B, Hkv, rows = 6, 3, 9000
@@ -329,3 +345,23 @@ def test_select_steps_share_one_workspace(cuda_dev):
         compare_idx(idx.cpu().numpy(), S, lens, kreq)
         ref = oracle.attn(L.Q, L.K, L.V, L.seq_lens, idx.cpu().numpy(), kreq, k_max, 1, SCALE)
         check_output(O.cpu().numpy(), ref, f"step with seed {seed}")
+
+
+def test_block_select_steps_share_one_workspace(cuda_dev):
+    """Block mode: the block-mean scorer also leaves the first-pass histogram for
+    the top-k; consecutive block-mode steps on one workspace each match the oracle."""
+    B, Hq, Hkv, N, k = 2, 16, 4, 6000, 8
+    lens = [6000, 1000]
+    ws = G.ws_for(torch.empty(B, Hq, 128, device=cuda_dev, dtype=torch.bfloat16),
+                  torch.empty(B, Hkv, N, 128, device=cuda_dev, dtype=torch.bfloat16), k, 128, tsa.SELECT)
+    for seed in (61, 62):
+        L = layer(B, Hq, Hkv, N, lens, seed=seed)
+        Q, K, V, ln = G.to_dev(L, cuda_dev)
+        Km = G.block_means(K, ln, 128)
+        O, idx = G.step(Q, K, V, ln, mode=tsa.SELECT, scale=SCALE, k_max=k, block=128, kreq=[k, k],
+                        Kmean=Km, ws=ws)
+        nb = oracle.nblocks_of(L.seq_lens, 128)
+        S = oracle.block_scores(L.Q, oracle.block_means(L.K, L.seq_lens, 128), nb, SCALE)
+        compare_idx(idx.cpu().numpy(), S, nb, [k, k])
+        ref = oracle.attn(L.Q, L.K, L.V, L.seq_lens, idx.cpu().numpy(), [k, k], k, 128, SCALE)
+        check_output(O.cpu().numpy(), ref, f"block step with seed {seed}")

@@ -74,9 +74,10 @@ size_t a256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 constexpr size_t kFlagBytes = 256;
 
-// Workspace: [flag 256 B][split counters][split partials][scores (SELECT only)]
+// Workspace: [flag 256 B][split counters][split partials][scores, top-digit
+// histograms (SELECT only)]
 struct Layout {
-    size_t counters = 0, partials = 0, scores = 0, total = kFlagBytes;
+    size_t counters = 0, partials = 0, scores = 0, hist = 0, total = kFlagBytes;
     int splits = 0;
 };
 
@@ -93,6 +94,8 @@ Layout layout(const tsa::Dims& d, int k_max, int block, bool attn, bool dense, b
     if (scores) {
         L.scores = off;
         off += a256((size_t)d.units() * tsa::rows_cap_of(d, block) * sizeof(float));
+        L.hist = off;
+        off += a256((size_t)d.units() * tsa::kHistBins * sizeof(uint32_t));
     }
     L.total = off;
     return L;
@@ -167,7 +170,7 @@ tsa_status sparse_decode_score(const void* Q, const void* keys, const int32_t* s
     if (!Q || !keys || !seq_lens || !scores) return fail(TSA_ERR_INVALID_ARG, "sparse_decode_score: NULL pointer");
     if (!aligned16(Q) || !aligned16(keys)) return fail(TSA_ERR_INVALID_ARG, "sparse_decode_score: Q and keys must be 16-byte aligned");
     TSA_TRY(check_ws(ws, ws_bytes, kFlagBytes));
-    cudaError_t e = tsa::launch_score(Q, keys, seq_lens, d, block, scale, scores, flag_of(ws),
+    cudaError_t e = tsa::launch_score(Q, keys, seq_lens, d, block, scale, scores, nullptr, flag_of(ws),
                                       static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "sparse_decode_score");
     return TSA_OK;
@@ -185,7 +188,7 @@ tsa_status topk_select(const float* scores, const int32_t* seq_lens, const int32
     if (!tsa::topk_plan(tsa::rows_cap_of(d, block), &C, &chunk))
         return fail(TSA_ERR_UNSUPPORTED, "topk_select: %d rows per unit exceed the cluster capacity", tsa::rows_cap_of(d, block));
     TSA_TRY(check_ws(ws, ws_bytes, kFlagBytes));
-    cudaError_t e = tsa::launch_topk(scores, seq_lens, k_per_seq, k_max, d, block, idx,
+    cudaError_t e = tsa::launch_topk(scores, seq_lens, k_per_seq, k_max, d, block, idx, nullptr,
                                      flag_of(ws), static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "topk_select");
     return TSA_OK;
@@ -246,12 +249,23 @@ tsa_status tsa_decode_step(const tsa_step_args* a, void* stream) {
                             tsa::rows_cap_of(d, a->block));
             const Layout L = layout(d, a->k_max, a->block, true, false, true);
             TSA_TRY(check_ws(a->ws, a->ws_bytes, L.total));
-            float* scores = reinterpret_cast<float*>(static_cast<char*>(a->ws) + L.scores);
+            char* w = static_cast<char*>(a->ws);
+            float* scores = reinterpret_cast<float*>(w + L.scores);
+            // the scorer also histograms the top digit of its keys; the top-k
+            // starts from that histogram and zeroes it for the next step
+            uint32_t* hist = reinterpret_cast<uint32_t*>(w + L.hist);
             const void* keys = a->block == 1 ? a->K : static_cast<const void*>(a->Kmean);
-            TSA_TRY(sparse_decode_score(a->Q, keys, a->seq_lens, a->shape, a->block, a->scale, scores,
-                                        a->ws, a->ws_bytes, stream));
-            TSA_TRY(topk_select(scores, a->seq_lens, a->k_per_seq, a->k_max, a->shape, a->block,
-                                a->idx_out, a->ws, a->ws_bytes, stream));
+            cudaStream_t st = static_cast<cudaStream_t>(stream);
+            cudaError_t e = tsa::launch_score(a->Q, keys, a->seq_lens, d, a->block, a->scale, scores, hist,
+                                              flag_of(a->ws), st);
+            if (e != cudaSuccess) return cuda_fail(e, "tsa_decode_step (score)");
+            e = tsa::launch_topk(scores, a->seq_lens, a->k_per_seq, a->k_max, d, a->block, a->idx_out, hist,
+                                 flag_of(a->ws), st);
+            if (e != cudaSuccess) {
+                // leave no partial histogram behind for the next step (best effort)
+                cudaMemsetAsync(hist, 0, (size_t)d.units() * tsa::kHistBins * sizeof(uint32_t), st);
+                return cuda_fail(e, "tsa_decode_step (top-k)");
+            }
             return sparse_decode_attn(a->Q, a->K, a->V, a->seq_lens, a->idx_out, a->k_per_seq, a->k_max,
                                       a->block, a->shape, a->scale, a->O, a->ws, a->ws_bytes, stream);
         }

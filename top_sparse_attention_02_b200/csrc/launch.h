@@ -35,16 +35,31 @@ void set_error_message(const char* msg);
 cudaError_t launch_block_summarize(const void* K, const int32_t* lens, const Dims& d, int block,
                                    float* Kmean, unsigned* flag, cudaStream_t st);
 
+// Top-digit histogram of a unit's score keys (the top 11 bits of the order key):
+// [units][kHistBins] u32, accumulated by the scorer when it is given one and
+// read and then zeroed by the top-k that follows it (the decode step pairs them).
+constexpr int kHistBins = 2048;
+
 cudaError_t launch_score(const void* Q, const void* keys, const int32_t* lens, const Dims& d,
-                         int block, float scale, float* scores, unsigned* flag, cudaStream_t st);
+                         int block, float scale, float* scores, uint32_t* hist, unsigned* flag,
+                         cudaStream_t st);
 // token mode on the tensor cores (TMA + tcgen05); used by launch_score for bf16 keys
 cudaError_t launch_score_tc(const void* Q, const void* K, const int32_t* lens, const Dims& d, float scale,
-                            float* scores, unsigned* flag, cudaStream_t st);
+                            float* scores, uint32_t* hist, unsigned* flag, cudaStream_t st);
 
 // top-k plan: cluster size and keys per CTA for a row count; false if too large
 bool topk_plan(int rows_cap, int* cluster, int* chunk);
+// hist: NULL (the kernel histograms the top digit itself) or the scorer's
+// histogram of these scores, which the kernel zeroes after reading it
 cudaError_t launch_topk(const float* scores, const int32_t* lens, const int32_t* kreq, int k_max,
-                        const Dims& d, int block, int32_t* idx, unsigned* flag, cudaStream_t st);
+                        const Dims& d, int block, int32_t* idx, uint32_t* hist, unsigned* flag,
+                        cudaStream_t st);
+
+// one CTA per unit, no cluster (topk_stream.cu): for many units or short ones
+bool topk_stream_fits(int units, int rows_cap);
+cudaError_t launch_topk_stream(const float* scores, const int32_t* lens, const int32_t* kreq, int k_max,
+                               const Dims& d, int block, int32_t* idx, uint32_t* hist, unsigned* flag,
+                               cudaStream_t st);
 
 // split-K plan for the attention stage (a pure function of the arguments, so
 // that workspace sizing and launch agree)

@@ -24,7 +24,8 @@ template <int G>
 __global__ void __launch_bounds__(kScoreThreads)
 score_kernel(const __nv_bfloat16* __restrict__ Q, const float* __restrict__ means,
              const int32_t* __restrict__ lens, int Hkv, int Ncap, int rows_cap, int block,
-             float scale, float* __restrict__ scores, unsigned* __restrict__ flag) {
+             float scale, float* __restrict__ scores, uint32_t* __restrict__ hist,
+             unsigned* __restrict__ flag) {
     constexpr int R = 16 / G;          // rows per half-warp (R*G = 16 partial dots)
     constexpr int kRowsWarp = 2 * R;   // rows per warp
     constexpr int kRowsCta = kRowsWarp * kScoreWarps;
@@ -80,7 +81,12 @@ score_kernel(const __nv_bfloat16* __restrict__ Q, const float* __restrict__ mean
     for (int o = 1; o < G; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     const int row = base + 2 * (c / G) + half;
     // scale > 0, so scale * max_h(z_h) = max_h(scale * z_h) exactly (rounding is monotone)
-    if ((c % G) == 0 && row < n) scores[(size_t)unit * rows_cap + row] = m * scale;
+    if ((c % G) == 0 && row < n) {
+        const float v = m * scale;
+        scores[(size_t)unit * rows_cap + row] = v;
+        // the top-k's first digit (one global atomic per block: 128x fewer than tokens)
+        if (hist) atomicAdd(&hist[(size_t)unit * kHistBins + (order_key(v) >> 21)], 1u);
+    }
 }
 
 // One CTA per (block, unit); thread t owns dimension t and sums the block's
@@ -106,9 +112,10 @@ block_mean_kernel(const __nv_bfloat16* __restrict__ K, const int32_t* __restrict
 }
 
 cudaError_t launch_score(const void* Q, const void* keys, const int32_t* lens, const Dims& d,
-                         int block, float scale, float* scores, unsigned* flag, cudaStream_t st) {
+                         int block, float scale, float* scores, uint32_t* hist, unsigned* flag,
+                         cudaStream_t st) {
     if (d.units() == 0 || d.Ncap == 0) return cudaSuccess;
-    if (block == 1) return launch_score_tc(Q, keys, lens, d, scale, scores, flag, st);
+    if (block == 1) return launch_score_tc(Q, keys, lens, d, scale, scores, hist, flag, st);
     const int rows_cap = rows_cap_of(d, block);
     const int rows_cta = 2 * (16 / d.G) * kScoreWarps;
     cudaLaunchConfig_t cfg = {};
@@ -122,10 +129,10 @@ cudaError_t launch_score(const void* Q, const void* keys, const int32_t* lens, c
     const float* m = static_cast<const float*>(keys);
     cudaError_t e;
     switch (d.G) {
-        case 1: e = cudaLaunchKernelEx(&cfg, score_kernel<1>, q, m, lens, d.Hkv, d.Ncap, rows_cap, block, scale, scores, flag); break;
-        case 2: e = cudaLaunchKernelEx(&cfg, score_kernel<2>, q, m, lens, d.Hkv, d.Ncap, rows_cap, block, scale, scores, flag); break;
-        case 4: e = cudaLaunchKernelEx(&cfg, score_kernel<4>, q, m, lens, d.Hkv, d.Ncap, rows_cap, block, scale, scores, flag); break;
-        case 8: e = cudaLaunchKernelEx(&cfg, score_kernel<8>, q, m, lens, d.Hkv, d.Ncap, rows_cap, block, scale, scores, flag); break;
+        case 1: e = cudaLaunchKernelEx(&cfg, score_kernel<1>, q, m, lens, d.Hkv, d.Ncap, rows_cap, block, scale, scores, hist, flag); break;
+        case 2: e = cudaLaunchKernelEx(&cfg, score_kernel<2>, q, m, lens, d.Hkv, d.Ncap, rows_cap, block, scale, scores, hist, flag); break;
+        case 4: e = cudaLaunchKernelEx(&cfg, score_kernel<4>, q, m, lens, d.Hkv, d.Ncap, rows_cap, block, scale, scores, hist, flag); break;
+        case 8: e = cudaLaunchKernelEx(&cfg, score_kernel<8>, q, m, lens, d.Hkv, d.Ncap, rows_cap, block, scale, scores, hist, flag); break;
         default: return cudaErrorInvalidValue;
     }
     note_launch();

@@ -21,7 +21,10 @@
 //           K = 16 x 8 steps, into one of two TMEM accumulators; tcgen05.commit
 //           frees the ring stage and publishes the accumulator;
 //   warps 2-5 epilogue: tcgen05.ld of their 32 TMEM lanes (= rows), max over the
-//           g heads, times the scale, coalesced store of the scores.
+//           g heads, times the scale, coalesced store of the scores; when asked,
+//           also a shared-memory histogram of the scores' top 11 key bits,
+//           added into the unit's histogram at the end (the top-k's first
+//           digit, counted here where the ALUs idle behind HBM).
 // Q is written once per CTA into shared memory in the same swizzled K-major
 // layout (the B operand).  Every mbarrier wait is bounded: on expiry the kernel
 // raises the device timeout flag and moves on; TMEM is always freed.
@@ -87,10 +90,12 @@ template <int G>
 __global__ void __launch_bounds__(kTcThreads, 2)
 score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16* __restrict__ Q,
                 const int32_t* __restrict__ lens, int Hkv, int Ncap, float scale,
-                float* __restrict__ scores, unsigned* __restrict__ flag) {
+                float* __restrict__ scores, uint32_t* __restrict__ hist, int tiles_per_cta,
+                unsigned* __restrict__ flag) {
     extern __shared__ unsigned char tc_smem_raw[];
     __shared__ __align__(8) uint64_t s_full[kTcStages], s_empty[kTcStages], s_tfull[2], s_tempty[2];
     __shared__ uint32_t s_tmem;
+    __shared__ uint32_t s_hist[kHistBins];  // this CTA's counts of the keys' top digit (when hist != NULL)
 
     const int unit = blockIdx.y;
     const int b = unit / Hkv;
@@ -102,8 +107,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16* _
         len = len < 0 ? 0 : Ncap;
     }
     const int ntiles_unit = ceil_div(len, kTcTileRows);
-    const int t0 = blockIdx.x * kTcTilesPerCta;
-    const int t1 = min(t0 + kTcTilesPerCta, ntiles_unit);
+    const int t0 = blockIdx.x * tiles_per_cta;
+    const int t1 = min(t0 + tiles_per_cta, ntiles_unit);
     if (t0 >= t1) return;  // uniform: before any barrier or TMEM use
     const int nt = t1 - t0;
 
@@ -114,6 +119,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16* _
     const unsigned qbase = base + kTcStages * kTcStageBytes;
 
     // ---- set-up: barriers (thread 0), TMEM (warp 1), Q as the swizzled B operand (warps 2-5)
+    if (hist)
+        for (int i = tid; i < kHistBins; i += kTcThreads) s_hist[i] = 0u;
     if (tid == 0) {
         for (int i = 0; i < kTcStages; ++i) {
             tc_mbar_init(su32(&s_full[i]), 1);
@@ -225,7 +232,11 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16* _
             for (int h = 1; h < G; ++h) m = fmaxf(m, __uint_as_float(r[h]));
             const int row = (t0 + i) * kTcTileRows + q * 32 + lane;
             // scale > 0, so scale * max_h(z_h) = max_h(scale * z_h) exactly (rounding is monotone)
-            if (ok && row < len) out[row] = m * scale;
+            if (ok && row < len) {
+                const float v = m * scale;
+                out[row] = v;
+                if (hist) atomicAdd(&s_hist[order_key(v) >> 21], 1u);
+            }
             asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
             tc_arrive(su32(&s_tempty[bsel]));
         }
@@ -236,6 +247,13 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16* _
     if (warp == 1) {
         asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(32) : "memory");
+    }
+    // this CTA's top-digit counts into the unit's histogram (the dependent top-k
+    // reads it only once this grid has completed)
+    if (hist) {
+        uint32_t* hu = hist + (size_t)unit * kHistBins;
+        for (int i = tid; i < kHistBins; i += kTcThreads)
+            if (const uint32_t c = s_hist[i]) atomicAdd(&hu[i], c);
     }
 }
 
@@ -256,7 +274,7 @@ static cudaError_t get_encode() {
 static int g_tc_configured[64];
 
 cudaError_t launch_score_tc(const void* Q, const void* K, const int32_t* lens, const Dims& d, float scale,
-                            float* scores, unsigned* flag, cudaStream_t st) {
+                            float* scores, uint32_t* hist, unsigned* flag, cudaStream_t st) {
     if (d.units() == 0 || d.Ncap == 0) return cudaSuccess;
     cudaError_t e = get_encode();
     if (e != cudaSuccess) return e;
@@ -282,7 +300,8 @@ cudaError_t launch_score_tc(const void* Q, const void* K, const int32_t* lens, c
         g_tc_configured[dev] = 1;
     }
     const int tiles = ceil_div(d.Ncap, kTcTileRows);
-    dim3 grid(ceil_div(tiles, kTcTilesPerCta), d.units());
+    const int per = kTcTilesPerCta;
+    dim3 grid(ceil_div(tiles, per), d.units());
     const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(Q);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
@@ -293,10 +312,10 @@ cudaError_t launch_score_tc(const void* Q, const void* K, const int32_t* lens, c
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     switch (d.G) {
-        case 1: e = cudaLaunchKernelEx(&cfg, score_tc_kernel<1>, map, q, lens, d.Hkv, d.Ncap, scale, scores, flag); break;
-        case 2: e = cudaLaunchKernelEx(&cfg, score_tc_kernel<2>, map, q, lens, d.Hkv, d.Ncap, scale, scores, flag); break;
-        case 4: e = cudaLaunchKernelEx(&cfg, score_tc_kernel<4>, map, q, lens, d.Hkv, d.Ncap, scale, scores, flag); break;
-        case 8: e = cudaLaunchKernelEx(&cfg, score_tc_kernel<8>, map, q, lens, d.Hkv, d.Ncap, scale, scores, flag); break;
+        case 1: e = cudaLaunchKernelEx(&cfg, score_tc_kernel<1>, map, q, lens, d.Hkv, d.Ncap, scale, scores, hist, per, flag); break;
+        case 2: e = cudaLaunchKernelEx(&cfg, score_tc_kernel<2>, map, q, lens, d.Hkv, d.Ncap, scale, scores, hist, per, flag); break;
+        case 4: e = cudaLaunchKernelEx(&cfg, score_tc_kernel<4>, map, q, lens, d.Hkv, d.Ncap, scale, scores, hist, per, flag); break;
+        case 8: e = cudaLaunchKernelEx(&cfg, score_tc_kernel<8>, map, q, lens, d.Hkv, d.Ncap, scale, scores, hist, per, flag); break;
         default: return cudaErrorInvalidValue;
     }
     note_launch();
