@@ -360,6 +360,13 @@ def stage_times(tsa, w, plan, layers, Kmean, ws, kreq_t, idx, O, stream, reps=10
                 scores, L.seq_lens, kreq_t, plan.k_max, shape, w.block, idx[li], ws, stream)
             calls[f"L{li}_attn"] = lambda L=L, li=li: tsa.sparse_decode_attn(
                 L.Q, L.K, L.V, L.seq_lens, idx[li], kreq_t, plan.k_max, w.block, w.scale, O[li], ws, stream)
+            # the whole SELECT step, as the decode step runs it (its top-k starts
+            # from the scorer's first-digit histogram, which the stand-alone
+            # stages above do not have)
+            sa = tsa.step_args(L.Q, L.K, L.V, L.seq_lens, O[li], ws, mode=tsa.SELECT, scale=w.scale,
+                               k_max=plan.k_max, block=w.block, k_per_seq=kreq_t, Kmean=Kmean[li],
+                               idx_out=idx[li])
+            calls[f"L{li}_select_step"] = lambda sa=sa: tsa.decode_step(sa, stream)
         elif m == tsa.REUSE:
             calls[f"L{li}_attn"] = lambda L=L, li=li: tsa.sparse_decode_attn(
                 L.Q, L.K, L.V, L.seq_lens, idx[w.reuse_from[li]], kreq_t, plan.k_max, w.block, w.scale,

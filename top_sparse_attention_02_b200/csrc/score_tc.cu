@@ -159,6 +159,10 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16* _
         // ---- TMA producer
         if (lane == 0) {
             const int row_base = unit * Ncap;
+            // K is read once: evict it from L2 first, so the scores (kept with
+            // evict_last below) are still there when the top-k reads them
+            uint64_t pol;
+            asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(pol));
             for (int i = 0; i < nt; ++i) {
                 const int s = i % kTcStages;
                 if (i >= kTcStages && !tc_wait(su32(&s_empty[s]), (unsigned)((i / kTcStages) - 1) & 1u, flag)) break;
@@ -169,9 +173,9 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16* _
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     asm volatile(
-                        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::"r"(
+                        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;\n" ::"r"(
                             dst + half * kTcHalfBytes),
-                        "l"(&kmap), "r"(half * 64), "r"(y), "r"(full)
+                        "l"(&kmap), "r"(half * 64), "r"(y), "r"(full), "l"(pol)
                         : "memory");
                 }
             }
@@ -212,6 +216,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16* _
         // ---- epilogue: warp quarter q reads TMEM lanes 32q..32q+31 (tile rows)
         const int q = warp & 3;
         float* out = scores + (size_t)unit * Ncap;
+        uint64_t keep;  // the scores are read again right after this kernel: keep them in L2
+        asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;\n" : "=l"(keep));
         for (int i = 0; i < nt; ++i) {
             const int bsel = i & 1;
             const bool ok = tc_wait(su32(&s_tfull[bsel]), (unsigned)(i >> 1) & 1u, flag);
@@ -234,7 +240,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16* _
             // scale > 0, so scale * max_h(z_h) = max_h(scale * z_h) exactly (rounding is monotone)
             if (ok && row < len) {
                 const float v = m * scale;
-                out[row] = v;
+                asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;\n" ::"l"(out + row), "f"(v), "l"(keep)
+                             : "memory");
                 if (hist) atomicAdd(&s_hist[order_key(v) >> 21], 1u);
             }
             asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");

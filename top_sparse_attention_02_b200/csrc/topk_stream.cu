@@ -62,8 +62,9 @@ __device__ __forceinline__ uint32_t ts_block_scan(uint32_t x, uint32_t* wsum, ui
     return ex;
 }
 
+// 256 threads: at most 64 registers, so that 4 CTAs (units) share an SM
 template <int THREADS>
-__global__ void __launch_bounds__(THREADS)
+__global__ void __launch_bounds__(THREADS, THREADS <= 256 ? 4 : 1)
 topk_stream_kernel(const float* __restrict__ scores, const int32_t* __restrict__ lens,
                    const int32_t* __restrict__ kreq, int k_max, int Hkv, int Ncap, int rows_cap, int block,
                    int wcap, int32_t* __restrict__ idx, uint32_t* __restrict__ hist,
