@@ -46,6 +46,9 @@
  *    tsa_workspace_size(...) bytes, 256-byte aligned, set to zero once with
  *    tsa_workspace_init before first use.  Calls that share a workspace must be
  *    ordered on one stream; calls that overlap on the GPU with the same `ws` race.
+ *    Between its scorer and its top-k a SELECT decode step keeps per-unit
+ *    counts in the workspace, which the top-k returns to zero; after any call
+ *    that returned TSA_ERR_CUDA, run tsa_workspace_init again before reusing it.
  */
 #ifndef TSA_H
 #define TSA_H

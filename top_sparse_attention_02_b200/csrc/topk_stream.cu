@@ -175,22 +175,42 @@ topk_stream_kernel(const float* __restrict__ scores, const int32_t* __restrict__
     const uint32_t kept = s_sel[1] + h[d0];  // keys whose top digit is >= d0, exactly
     const uint32_t lt = (1u << lane) - 1u;
 
-    // ---- filter into the per-warp lists (index order within each warp)
+    // ---- filter into the per-warp lists (index order within each warp).  Most
+    // keys fail, so a batch is first tested as raw floats against the smallest
+    // float whose key reaches digit d0 (the key order is the float order, -0 =
+    // +0; NaN passes and is sorted out by its key), one vote for the batch.
     uint32_t* lkey = ts_list + warp * wcap;
     uint32_t* lrow = ts_list + W * wcap + warp * wcap;
     bool list_mode = kept <= (uint32_t)(W * wcap);
     if (list_mode) {
+        const uint32_t kthr = d0 << 21;
+        const float fthr = __uint_as_float((kthr & 0x80000000u) ? (kthr & 0x7fffffffu) : ~kthr);
         uint32_t cnt = 0;
-        stream([&](int i, uint32_t k, bool v) {
-            const bool keep = v && (k >> 21) >= d0;
-            const uint32_t bal = __ballot_sync(0xffffffffu, keep);
-            const uint32_t pos = cnt + __popc(bal & lt);
-            if (keep && pos < (uint32_t)wcap) {
-                lkey[pos] = k;
-                lrow[pos] = (uint32_t)i;
+        for (int base = wb; base < we; base += 32 * kTsNB) {
+            float v[kTsNB];
+#pragma unroll
+            for (int j = 0; j < kTsNB; ++j) {
+                const int i = base + j * 32 + lane;
+                v[j] = i < we ? __ldcg(su + i) : 0.f;
             }
-            cnt += __popc(bal);
-        });
+            bool any = false;
+#pragma unroll
+            for (int j = 0; j < kTsNB; ++j) any |= (base + j * 32 + lane < we) && !(v[j] < fthr);
+            if (!__any_sync(0xffffffffu, any)) continue;
+#pragma unroll
+            for (int j = 0; j < kTsNB; ++j) {
+                const int i = base + j * 32 + lane;
+                const uint32_t k = order_key(v[j]);
+                const bool keep = i < we && (k >> 21) >= d0;
+                const uint32_t bal = __ballot_sync(0xffffffffu, keep);
+                const uint32_t pos = cnt + __popc(bal & lt);
+                if (keep && pos < (uint32_t)wcap) {
+                    lkey[pos] = k;
+                    lrow[pos] = (uint32_t)i;
+                }
+                cnt += __popc(bal);
+            }
+        }
         if (lane == 0) {
             s_cnt[warp] = cnt;
             if (cnt > (uint32_t)wcap) s_over = 1;
