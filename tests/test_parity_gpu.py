@@ -365,3 +365,34 @@ def test_block_select_steps_share_one_workspace(cuda_dev):
         compare_idx(idx.cpu().numpy(), S, nb, [k, k])
         ref = oracle.attn(L.Q, L.K, L.V, L.seq_lens, idx.cpu().numpy(), [k, k], k, 128, SCALE)
         check_output(O.cpu().numpy(), ref, f"block step with seed {seed}")
+
+
+@pytest.mark.parametrize("case", ["plain", "tied_top", "k_near_len"])
+def test_decode_step_topk_from_the_scorers_histogram(cuda_dev, case):
+    """Inside a decode step the top-k of long units starts from the scorer's
+    first-digit histogram (a cluster per unit, lists in registers and shared
+    memory).  Its paths: the plain one; 7000 identical top keys (exact ties at T:
+    the lists overflow and every later pass runs over all keys); k one short of
+    the length.  Two steps on one workspace check that the histogram is zeroed."""
+    B, Hq, Hkv, N = 2, 16, 4, 20000
+    lens = [20000, 15000]
+    L = layer(B, Hq, Hkv, N, lens, seed=71)
+    if case == "tied_top":
+        S0 = oracle.scores(L.Q, L.K, L.seq_lens, SCALE)
+        for b in range(B):
+            for h in range(Hkv):
+                top = int(np.argmax(S0[b, h, :lens[b]]))
+                L.K[b, h, 5000:12000] = L.K[b, h, top]
+        kreq, k_max = [100, 6000], 6000
+    elif case == "k_near_len":
+        kreq, k_max = [19999, 14999], 19999
+    else:
+        kreq, k_max = [400, 300], 400
+    Q, K, V, ln = G.to_dev(L, cuda_dev)
+    ws = G.ws_for(Q, K, k_max, 1, tsa.SELECT)
+    S = oracle.scores(L.Q, L.K, L.seq_lens, SCALE)
+    for rep in range(2):
+        O, idx = G.step(Q, K, V, ln, mode=tsa.SELECT, scale=SCALE, k_max=k_max, kreq=kreq, ws=ws)
+        compare_idx(idx.cpu().numpy(), S, lens, kreq)
+        ref = oracle.attn(L.Q, L.K, L.V, L.seq_lens, idx.cpu().numpy(), kreq, k_max, 1, SCALE)
+        check_output(O.cpu().numpy(), ref, f"{case} step {rep}")

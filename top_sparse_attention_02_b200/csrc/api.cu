@@ -266,8 +266,13 @@ tsa_status tsa_decode_step(const tsa_step_args* a, void* stream) {
                 cudaMemsetAsync(hist, 0, (size_t)d.units() * tsa::kHistBins * sizeof(uint32_t), st);
                 return cuda_fail(e, "tsa_decode_step (top-k)");
             }
-            return sparse_decode_attn(a->Q, a->K, a->V, a->seq_lens, a->idx_out, a->k_per_seq, a->k_max,
-                                      a->block, a->shape, a->scale, a->O, a->ws, a->ws_bytes, stream);
+            // the attention follows this step's own top-k, which wrote only the
+            // indices: it may read the lengths, k's and Q before waiting on it
+            e = tsa::launch_attn(a->Q, a->K, a->V, a->seq_lens, a->idx_out, a->k_per_seq, a->k_max, a->block, d,
+                                 a->scale, L.splits, reinterpret_cast<float*>(w + L.partials),
+                                 reinterpret_cast<unsigned*>(w + L.counters), a->O, flag_of(a->ws), st, true);
+            if (e != cudaSuccess) return cuda_fail(e, "tsa_decode_step (attention)");
+            return TSA_OK;
         }
         default:
             return fail(TSA_ERR_INVALID_ARG, "tsa_decode_step: unknown mode %d", a->mode);

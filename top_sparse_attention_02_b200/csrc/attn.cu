@@ -139,7 +139,7 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
             const __nv_bfloat16* __restrict__ V, const int32_t* __restrict__ lens,
             const int32_t* __restrict__ idx, const int32_t* __restrict__ kreq, int k_max,
             int block, int Hkv, int Ncap, float scale_log2, int S, float* __restrict__ part,
-            unsigned* __restrict__ counters, float* __restrict__ O, unsigned* __restrict__ flag) {
+            unsigned* __restrict__ counters, float* __restrict__ O, unsigned* __restrict__ flag, int early) {
     using Cfg = AttnCfg<G>;
     extern __shared__ __align__(128) unsigned char smem_raw[];
     // 1024-byte aligned work area (the swizzled layout needs it)
@@ -156,10 +156,19 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
     const int b = unit / Hkv;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t4 = lane & 3;  // mma fragment coordinates
+    // early: the kernel before this one did not write the lengths, the k's or Q
+    // (the decode step's own top-k), so they are read before waiting on it
+    int len = 0, kreq_b = k_max;
+    if (early) {
+        len = lens[b];
+        if (kreq) kreq_b = kreq[b];
+    }
     griddep_wait();
     griddep_launch();
-
-    int len = lens[b];
+    if (!early) {
+        len = lens[b];
+        if (kreq) kreq_b = kreq[b];
+    }
     if (len < 0 || len > Ncap) {
         if (tid == 0 && s == 0) atomicOr(flag, kFlagBounds);
         len = len < 0 ? 0 : Ncap;
@@ -169,8 +178,7 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
         npos = len;
     } else {
         nb = block == 1 ? len : ceil_div(len, block);
-        int kb = kreq ? kreq[b] : k_max;
-        kb = max(0, min(kb, nb));
+        int kb = max(0, min(kreq_b, nb));
         if (kb > k_max) {
             if (tid == 0 && s == 0) atomicOr(flag, kFlagBounds);
             kb = k_max;
@@ -679,6 +687,7 @@ struct AttnArgs {
     unsigned* counters;
     float* O;
     unsigned* flag;
+    int early;
 };
 
 template <int G, int STAGES, bool CLUSTER, bool CONTIG>
@@ -698,7 +707,7 @@ static cudaError_t attn_launch_g(dim3 grid, cudaStream_t st, const AttnArgs& a) 
     cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, attn_kernel<G, STAGES, CLUSTER, CONTIG>, a.kmap, a.vmap, a.q, a.k, a.v, a.lens,
                               a.idx, a.kreq, a.k_max, a.block, a.Hkv, a.Ncap, a.sl2, a.splits, a.partials, a.counters,
-                              a.O, a.flag);
+                              a.O, a.flag, a.early);
 }
 
 template <int G, int STAGES, bool CLUSTER, bool CONTIG>
@@ -762,7 +771,7 @@ static cudaError_t make_row_map(CUtensorMap* map, const void* base, const Dims& 
 cudaError_t launch_attn(const void* Q, const void* K, const void* V, const int32_t* lens,
                         const int32_t* idx, const int32_t* kreq, int k_max, int block,
                         const Dims& d, float scale, int splits, float* partials,
-                        unsigned* counters, float* O, unsigned* flag, cudaStream_t st) {
+                        unsigned* counters, float* O, unsigned* flag, cudaStream_t st, bool early) {
     if (d.units() == 0) return cudaSuccess;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -811,6 +820,7 @@ cudaError_t launch_attn(const void* Q, const void* K, const void* V, const int32
     a.counters = counters;
     a.O = O;
     a.flag = flag;
+    a.early = early ? 1 : 0;
     dim3 grid(splits, d.units());
     switch (d.G) {
         case 1: e = attn_dispatch<1>(contig, one_tile, cluster, grid, st, a); break;

@@ -61,6 +61,13 @@ cudaError_t launch_topk_stream(const float* scores, const int32_t* lens, const i
                                const Dims& d, int block, int32_t* idx, uint32_t* hist, unsigned* flag,
                                cudaStream_t st);
 
+// inside a decode step, for few long units (topk_hist.cu): starts from the
+// scorer's histogram; false when the shape is not one it serves
+bool topk_hist_plan(int units, int rows_cap, int* cluster, int* kpt);
+cudaError_t launch_topk_hist(int C, int kpt, const float* scores, const int32_t* lens, const int32_t* kreq,
+                             int k_max, const Dims& d, int block, int32_t* idx, uint32_t* hist, unsigned* flag,
+                             cudaStream_t st);
+
 // split-K plan for the attention stage (a pure function of the arguments, so
 // that workspace sizing and launch agree)
 int attn_splits(const Dims& d, int k_max, int block, bool dense);
@@ -68,7 +75,8 @@ size_t attn_partials_floats(const Dims& d, int splits);
 cudaError_t launch_attn(const void* Q, const void* K, const void* V, const int32_t* lens,
                         const int32_t* idx, const int32_t* kreq, int k_max, int block,
                         const Dims& d, float scale, int splits, float* partials,
-                        unsigned* counters, float* O, unsigned* flag, cudaStream_t st);
+                        unsigned* counters, float* O, unsigned* flag, cudaStream_t st,
+                        bool early = false);  // early: lens, k's and Q not written by the previous kernel
 
 cudaError_t launch_copy(const void* src, void* dst, size_t bytes, cudaStream_t st);
 cudaError_t launch_gather(const void* base, size_t base_bytes, const int32_t* rows, int nrows, unsigned* flag,

@@ -418,6 +418,9 @@ cudaError_t launch_topk(const float* scores, const int32_t* lens, const int32_t*
     const int rows_cap = rows_cap_of(d, block);
     if (topk_stream_fits(d.units(), rows_cap))
         return launch_topk_stream(scores, lens, kreq, k_max, d, block, idx, hist, flag, st);
+    int hc = 1, hk = 16;
+    if (hist && topk_hist_plan(d.units(), rows_cap, &hc, &hk))
+        return launch_topk_hist(hc, hk, scores, lens, kreq, k_max, d, block, idx, hist, flag, st);
     int C = 1, chunk = 32;
     if (!topk_plan(rows_cap, &C, &chunk)) return cudaErrorInvalidValue;
     int dev = 0;
