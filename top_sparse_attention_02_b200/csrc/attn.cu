@@ -144,7 +144,6 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
     extern __shared__ __align__(128) unsigned char smem_raw[];
     // 1024-byte aligned work area (the swizzled layout needs it)
     unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    __shared__ int s_row[STAGES][kTileRows];
     __shared__ float s_wm[kAttnWarps][G], s_wl[kAttnWarps][G];
     __shared__ float s_M[G], s_L[G];
     __shared__ float s_Mr[kClusterMax][G], s_Lr[kClusterMax][G];  // cluster path: received (M, L)
@@ -213,14 +212,6 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
         const int r = e * block + (pos - slot * block);
         return r < len ? r : -1;
     };
-    // thread slot (< 128) owns row `slot` of every tile: two 256-byte bulk copies
-    // (K and V) per valid row, each thread arriving once per tile on that
-    // stage's mbarrier (with the bytes it expects); unused rows are zero-filled.
-    const int my_slot = tid;
-    auto row_for_tile = [&](int t) -> int {
-        const int pos = p0 + t * kTileRows + my_slot;
-        return (my_slot < kTileRows && t < ntiles && pos < p1) ? row_of(pos) : -1;
-    };
     // CONTIG: the tile's first cache row (dense: its position; block mode: the
     // chosen block's first row), or -1 when the block entry is absent
     auto tile_first = [&](int t) -> int {
@@ -263,34 +254,13 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
             mbar_arrive(&s_bar[st]);
         }
     };
-    auto stage_tile = [&](int t, int row) {
-        if (t >= ntiles || my_slot >= kTileRows) return;
-        const int st = t % STAGES;
-        s_row[st][my_slot] = row;
-        unsigned char* kd = smem + st * kStageBytes + my_slot * kRowStride;
-        unsigned char* vd = kd + kTileRows * kRowStride;
-        if (row >= 0) {
-            fence_proxy_async();  // earlier generic accesses of this stage come first
-            mbar_arrive_expect_tx(&s_bar[st], 2 * kD * 2);
-            bulk_g2s(kd, Ku + (size_t)row * kD, kD * 2, &s_bar[st]);
-            bulk_g2s(vd, Vu + (size_t)row * kD, kD * 2, &s_bar[st]);
-        } else {  // an unused row must hold zeros: its weight is 0 and 0 * garbage may be NaN
-#pragma unroll
-            for (int ch = 0; ch < 16; ++ch) {
-                *reinterpret_cast<uint4*>(kd + 16 * ch) = make_uint4(0, 0, 0, 0);
-                *reinterpret_cast<uint4*>(vd + 16 * ch) = make_uint4(0, 0, 0, 0);
-            }
-            mbar_arrive(&s_bar[st]);
-        }
-    };
-
     if (tid == 0) {
 #pragma unroll
         for (int i = 0; i < STAGES; ++i) mbar_init(&s_bar[i], CONTIG ? 1 : kTileRows);
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
     __syncthreads();
-    // the first STAGES tiles: index reads in one round, then every copy
+    // CONTIG: the first STAGES tiles' block indices in one round, then their loads
     int next_first = -1;  // CONTIG, thread 0: first row of the tile that refills the stage next
     if constexpr (CONTIG) {
         if (tid == 0) {
@@ -300,13 +270,36 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
 #pragma unroll
             for (int t = 0; t < STAGES; ++t) stage_contig(t, f[t]);
         }
-    } else {
-        int pre[STAGES];
-#pragma unroll
-        for (int t = 0; t < STAGES; ++t) pre[t] = row_for_tile(t);
-#pragma unroll
-        for (int t = 0; t < STAGES; ++t) stage_tile(t, pre[t]);
     }
+
+    const int r0 = warp * 16;  // this warp's rows in a tile
+    // Gather: each warp fetches its own 16 rows of a tile with 16-byte vector
+    // loads (a half-warp per 256-byte row; lane l takes chunk l & 15 of rows
+    // (l >> 4), +2, ..., +14), one tile ahead in registers, and stores them
+    // into its rows of the padded tile: no TMA queue (one 256-byte bulk copy
+    // per row issued at ~13 ns a copy per SM, which bounded short gathers) and
+    // no CTA barrier per tile.  Rows not in the set are zeros (0 x NaN = NaN).
+    unsigned char* kw = smem + r0 * kRowStride;
+    unsigned char* vw = smem + (kTileRows + r0) * kRowStride;
+    const int hl = lane >> 4, c16 = lane & 15;
+    uint4 pk[8], pv[8];
+    uint32_t vm_next = 0;
+    auto fetch = [&](int t) {
+        if constexpr (CONTIG) return;
+        int myrow = -1;
+        if (lane < 16) {
+            const int pos = p0 + t * kTileRows + r0 + lane;
+            if (pos < p1) myrow = row_of(pos);
+        }
+        vm_next = __ballot_sync(0xffffffffu, myrow >= 0) & 0xffffu;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int rr = __shfl_sync(0xffffffffu, myrow, hl + 2 * j);
+            pk[j] = rr >= 0 ? ld_stream(Ku + (size_t)rr * kD + 8 * c16) : make_uint4(0, 0, 0, 0);
+            pv[j] = rr >= 0 ? ld_stream(Vu + (size_t)rr * kD + 8 * c16) : make_uint4(0, 0, 0, 0);
+        }
+    };
+    if (!CONTIG && ntiles > 0) fetch(0);  // in flight while Q is read
 
     // A fragments of Q (bf16, unscaled: the scale is applied to S in fp32).
     // Row g of A = query head g of the group (zero for g >= G); rows g+8 are zero.
@@ -327,15 +320,88 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
     float m_run = -INFINITY, l_run = 0.f;  // this warp's running max / sum for head g
 
     const unsigned sbase = smem_u32(smem);
-    for (int t = 0; t < ntiles; ++t) {
-        if (CONTIG && tid == 0) next_first = tile_first(t + STAGES);  // in flight during this tile
-        mbar_wait(&s_bar[t % STAGES], (unsigned)(t / STAGES) & 1u, flag);  // tile t has landed
-        const int st = t % STAGES;
-        int tile_rows = min(kTileRows, p1 - p0 - t * kTileRows);
-        if constexpr (CONTIG) {
+    // The two contractions of flash decoding on this warp's 16 rows of a tile
+    // (K at kt, V at vt); bit i of vm: row r0 + i is in the set.
+    auto warp_tile = [&](unsigned kt, unsigned vt, uint32_t vm) {
+        // byte offset of 16-byte chunk c of tile row r (padded rows, or the
+        // 128-byte swizzle of the TMA tensor loads: two 64-dim halves)
+        auto off = [&](int r, int c) -> unsigned {
+            if constexpr (CONTIG)
+                return (unsigned)((c >> 3) * 64 * kTileRows * 2 + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+            else
+                return (unsigned)roff(r, c);
+        };
+        // ---- S = Q K^T over this warp's 16 rows (two n-tiles of 8 rows)
+        float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        {
+            const int m = lane >> 3, i = lane & 7;  // ldmatrix: matrix m, row i
+            const int row = r0 + (m >> 1) * 8 + i;   // n-tile (m>>1), k-half (m&1)
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4(kt + off(row, 2 * ks + (m & 1)), b0, b1, b2, b3);
+                mma_bf16(sc[0], qa[ks][0], qa[ks][1], b0, b1);
+                mma_bf16(sc[1], qa[ks][0], qa[ks][1], b2, b3);
+            }
+        }
+        // ---- online softmax for head g (columns = rows of the tile)
+        float z[4];
+        {
+            const int ia = 2 * t4;  // local rows of sc[0][0..1]; sc[1] adds 8
+            z[0] = (vm >> ia) & 1u ? sc[0][0] * scale_log2 : -INFINITY;
+            z[1] = (vm >> (ia + 1)) & 1u ? sc[0][1] * scale_log2 : -INFINITY;
+            z[2] = (vm >> (ia + 8)) & 1u ? sc[1][0] * scale_log2 : -INFINITY;
+            z[3] = (vm >> (ia + 9)) & 1u ? sc[1][1] * scale_log2 : -INFINITY;
+        }
+        float mt = fmaxf(fmaxf(z[0], z[1]), fmaxf(z[2], z[3]));
+        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
+        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
+        const float mnew = fmaxf(m_run, mt);
+        if (mnew != -INFINITY) {  // uniform across the 4 lanes of head g
+            const float alpha = m_run == -INFINITY ? 0.f : exp2f(m_run - mnew);
+            float p[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) p[e] = z[e] == -INFINITY ? 0.f : exp2f(z[e] - mnew);
+            float ps = (p[0] + p[1]) + (p[2] + p[3]);
+            ps += __shfl_xor_sync(0xffffffffu, ps, 1);
+            ps += __shfl_xor_sync(0xffffffffu, ps, 2);
+            l_run = l_run * alpha + ps;
+            m_run = mnew;
+#pragma unroll
+            for (int n = 0; n < 16; ++n) {
+                o[n][0] *= alpha;
+                o[n][1] *= alpha;
+            }
+            // P as the A operand (row g, k = tile rows), split hi + lo
+            const uint32_t ph0 = pack_bf16(p[0], p[1]), ph1 = pack_bf16(p[2], p[3]);
+            const __nv_bfloat162 h0 = *reinterpret_cast<const __nv_bfloat162*>(&ph0);
+            const __nv_bfloat162 h1 = *reinterpret_cast<const __nv_bfloat162*>(&ph1);
+            const uint32_t pl0 = pack_bf16(p[0] - __low2float(h0), p[1] - __high2float(h0));
+            const uint32_t pl1 = pack_bf16(p[2] - __low2float(h1), p[3] - __high2float(h1));
+            // ---- O += P V over 16 dim n-tiles
+            const int m = lane >> 3, i = lane & 7;  // ldmatrix.trans: matrix m, row i
+            const int row = r0 + (m & 1) * 8 + i;    // k-half (m&1), dim n-tile (m>>1)
+#pragma unroll
+            for (int np = 0; np < 8; ++np) {
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4_t(vt + off(row, 2 * np + (m >> 1)), b0, b1, b2, b3);
+                mma_bf16(o[2 * np], ph0, ph1, b0, b1);
+                mma_bf16(o[2 * np], pl0, pl1, b0, b1);
+                mma_bf16(o[2 * np + 1], ph0, ph1, b2, b3);
+                mma_bf16(o[2 * np + 1], pl0, pl1, b2, b3);
+            }
+        }
+    };
+
+    if constexpr (CONTIG) {
+        for (int t = 0; t < ntiles; ++t) {
+            if (tid == 0) next_first = tile_first(t + STAGES);  // in flight during this tile
+            mbar_wait(&s_bar[t % STAGES], (unsigned)(t / STAGES) & 1u, flag);  // tile t has landed
+            const int st = t % STAGES;
             // the valid rows are a prefix: the range's and the sequence's ends cut it;
             // an absent block (first < 0) has none and nothing landed
             const int first = s_first[st];
+            int tile_rows = min(kTileRows, p1 - p0 - t * kTileRows);
             tile_rows = first < 0 ? 0 : max(0, min(tile_rows, len - first));
             // rows past it hold real cache data, which may be anything: give V
             // there zeros, since their weight 0 times NaN is NaN
@@ -350,89 +416,28 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
                 fence_proxy_async();  // before the stage's next tensor load overwrites them
             }
             __syncthreads();  // every thread, every tile (never a divergent barrier)
-        }
-        const int r0 = warp * 16;  // this warp's rows in the tile
-        if (r0 < tile_rows) {      // warp-uniform
-            const unsigned kt = sbase + st * kStageBytes;
-            const unsigned vt = kt + (CONTIG ? 2 * 64 * kTileRows * 2 : kTileRows * kRowStride);
-            // byte offset of 16-byte chunk c of tile row r (padded rows, or the
-            // 128-byte swizzle of the TMA tensor loads: two 64-dim halves)
-            auto off = [&](int r, int c) -> unsigned {
-                if constexpr (CONTIG)
-                    return (unsigned)((c >> 3) * 64 * kTileRows * 2 + r * 128 + (((c & 7) ^ (r & 7)) << 4));
-                else
-                    return (unsigned)roff(r, c);
-            };
-            // ---- S = Q K^T over this warp's 16 rows (two n-tiles of 8 rows)
-            float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-            {
-                const int m = lane >> 3, i = lane & 7;  // ldmatrix: matrix m, row i
-                const int row = r0 + (m >> 1) * 8 + i;   // n-tile (m>>1), k-half (m&1)
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    uint32_t b0, b1, b2, b3;
-                    ldsm_x4(kt + off(row, 2 * ks + (m & 1)), b0, b1, b2, b3);
-                    mma_bf16(sc[0], qa[ks][0], qa[ks][1], b0, b1);
-                    mma_bf16(sc[1], qa[ks][0], qa[ks][1], b2, b3);
-                }
+            const int nv = tile_rows - r0;
+            const uint32_t vm = nv >= 16 ? 0xffffu : (nv > 0 ? (1u << nv) - 1u : 0u);
+            if (vm) {  // warp-uniform
+                const unsigned kt = sbase + st * kStageBytes;
+                warp_tile(kt, kt + 2 * 64 * kTileRows * 2, vm);
             }
-            // ---- online softmax for head g (columns = rows of the tile)
-            float z[4];
-            {
-                const int ra = r0 + 2 * t4;  // rows of sc[0][0..1]; sc[1] adds 8
-                const bool v0 = ra < tile_rows && (CONTIG || s_row[st][ra] >= 0);
-                const bool v1 = ra + 1 < tile_rows && (CONTIG || s_row[st][ra + 1] >= 0);
-                const bool v2 = ra + 8 < tile_rows && (CONTIG || s_row[st][ra + 8] >= 0);
-                const bool v3 = ra + 9 < tile_rows && (CONTIG || s_row[st][ra + 9] >= 0);
-                z[0] = v0 ? sc[0][0] * scale_log2 : -INFINITY;
-                z[1] = v1 ? sc[0][1] * scale_log2 : -INFINITY;
-                z[2] = v2 ? sc[1][0] * scale_log2 : -INFINITY;
-                z[3] = v3 ? sc[1][1] * scale_log2 : -INFINITY;
-            }
-            float mt = fmaxf(fmaxf(z[0], z[1]), fmaxf(z[2], z[3]));
-            mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
-            mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
-            const float mnew = fmaxf(m_run, mt);
-            if (mnew != -INFINITY) {  // uniform across the 4 lanes of head g
-                const float alpha = m_run == -INFINITY ? 0.f : exp2f(m_run - mnew);
-                float p[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) p[e] = z[e] == -INFINITY ? 0.f : exp2f(z[e] - mnew);
-                float ps = (p[0] + p[1]) + (p[2] + p[3]);
-                ps += __shfl_xor_sync(0xffffffffu, ps, 1);
-                ps += __shfl_xor_sync(0xffffffffu, ps, 2);
-                l_run = l_run * alpha + ps;
-                m_run = mnew;
-#pragma unroll
-                for (int n = 0; n < 16; ++n) {
-                    o[n][0] *= alpha;
-                    o[n][1] *= alpha;
-                }
-                // P as the A operand (row g, k = tile rows), split hi + lo
-                const uint32_t ph0 = pack_bf16(p[0], p[1]), ph1 = pack_bf16(p[2], p[3]);
-                const __nv_bfloat162 h0 = *reinterpret_cast<const __nv_bfloat162*>(&ph0);
-                const __nv_bfloat162 h1 = *reinterpret_cast<const __nv_bfloat162*>(&ph1);
-                const uint32_t pl0 = pack_bf16(p[0] - __low2float(h0), p[1] - __high2float(h0));
-                const uint32_t pl1 = pack_bf16(p[2] - __low2float(h1), p[3] - __high2float(h1));
-                // ---- O += P V over 16 dim n-tiles
-                const int m = lane >> 3, i = lane & 7;  // ldmatrix.trans: matrix m, row i
-                const int row = r0 + (m & 1) * 8 + i;    // k-half (m&1), dim n-tile (m>>1)
-#pragma unroll
-                for (int np = 0; np < 8; ++np) {
-                    uint32_t b0, b1, b2, b3;
-                    ldsm_x4_t(vt + off(row, 2 * np + (m >> 1)), b0, b1, b2, b3);
-                    mma_bf16(o[2 * np], ph0, ph1, b0, b1);
-                    mma_bf16(o[2 * np], pl0, pl1, b0, b1);
-                    mma_bf16(o[2 * np + 1], ph0, ph1, b2, b3);
-                    mma_bf16(o[2 * np + 1], pl0, pl1, b2, b3);
-                }
-            }
-        }
-        __syncthreads();               // every warp is done with this stage
-        if constexpr (CONTIG) {
+            __syncthreads();  // every warp is done with this stage
             if (tid == 0) stage_contig(t + STAGES, next_first);  // refill it (nothing past the end)
         }
-        else stage_tile(t + STAGES, row_for_tile(t + STAGES));
+    } else {
+        for (int t = 0; t < ntiles; ++t) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                *reinterpret_cast<uint4*>(kw + (hl + 2 * j) * kRowStride + 16 * c16) = pk[j];
+                *reinterpret_cast<uint4*>(vw + (hl + 2 * j) * kRowStride + 16 * c16) = pv[j];
+            }
+            const uint32_t vm = vm_next;
+            __syncwarp();
+            if (t + 1 < ntiles) fetch(t + 1);  // the next tile's loads fly during this tile's math
+            if (vm) warp_tile(sbase, sbase + kTileRows * kRowStride, vm);
+            __syncwarp();  // the math has read these rows before the next store
+        }
     }
     __syncthreads();
 
@@ -598,14 +603,17 @@ int attn_splits(const Dims& d, int k_max, int block, bool dense) {
         }
     } else {
         // latency-bound gather: one tile per split where the GPU has room
-        // (a wave of at most one CTA per SM), else longer splits whose first
-        // kRing tiles are all in flight at once; whether the splits of a unit
+        // (a wave of at most one CTA per SM); whether the splits of a unit
         // combine in a cluster is decided at launch (attn_cluster_fits)
         const long long nbmax = block == 1 ? d.Ncap : ceil_div(d.Ncap, block);
         rows = (long long)(k_max < nbmax ? k_max : nbmax) * block;
         s = (int)((rows + kTileRows - 1) / kTileRows);
         const int room = kSms / units > 1 ? kSms / units : 1;
         if (s > room) s = room;
+        // past 8 splits the partials combine through the workspace (the last CTA
+        // of a unit reads them all), which costs more than the extra splits save
+        // unless there are too few units to fill the GPU
+        if (s > kClusterMax && units >= 4) s = kClusterMax;
     }
     const long long smax = (rows + 31) / 32;  // at least 32 positions per split
     if (s > smax) s = (int)smax;
@@ -795,7 +803,8 @@ cudaError_t launch_attn(const void* Q, const void* K, const void* V, const int32
     const bool contig = idx == nullptr || block == kTileRows;
     const long long per_split = contig ? ((rows + splits - 1) / splits + kTileRows - 1) / kTileRows * kTileRows
                                        : (rows + splits - 1) / splits;
-    const bool one_tile = per_split <= kTileRows;
+    // one stage: a tile at a time (contiguous tiles), or the warp-private gather
+    const bool one_tile = !contig || per_split <= kTileRows;
     const bool cluster = attn_cluster_fits(d.G, one_tile, contig, splits, d.units());
     AttnArgs a;
     memset(&a.kmap, 0, sizeof a.kmap);
