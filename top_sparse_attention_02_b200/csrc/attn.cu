@@ -612,7 +612,8 @@ int attn_splits(const Dims& d, int k_max, int block, bool dense) {
         if (s > room) s = room;
         // past 8 splits the partials combine through the workspace (the last CTA
         // of a unit reads them all), which costs more than the extra splits save
-        // unless there are too few units to fill the GPU
+        // unless there are too few units to fill the GPU (16-CTA clusters measured
+        // no faster than 8: the per-launch chain of dependent loads dominates)
         if (s > kClusterMax && units >= 4) s = kClusterMax;
     }
     const long long smax = (rows + 31) / 32;  // at least 32 positions per split
@@ -663,8 +664,8 @@ static bool attn_cluster_fits_g(int dev, bool one_tile, bool contig, int S, int 
     int& slot = g_max_clusters[dev][lg][one_tile][contig][S];
     if (slot == 0) {
         int n;
-        if (one_tile) n = contig ? max_active_clusters<G, 1, true>(S) : max_active_clusters<G, 1, false>(S);
-        else n = contig ? max_active_clusters<G, kRing, true>(S) : max_active_clusters<G, kRing, false>(S);
+        if (!contig) n = max_active_clusters<G, 1, false>(S);
+        else n = one_tile ? max_active_clusters<G, 1, true>(S) : max_active_clusters<G, kRing, true>(S);
         slot = n;
     }
     return slot > 0 && units <= slot;
@@ -730,10 +731,9 @@ static cudaError_t attn_configure_one() {
 template <int G>
 static cudaError_t attn_configure() {
     cudaError_t e = cudaSuccess;
+    // the gather runs one stage; contiguous tiles one or kRing
     if (e == cudaSuccess) e = attn_configure_one<G, 1, true, false>();
-    if (e == cudaSuccess) e = attn_configure_one<G, kRing, true, false>();
     if (e == cudaSuccess) e = attn_configure_one<G, 1, false, false>();
-    if (e == cudaSuccess) e = attn_configure_one<G, kRing, false, false>();
     if (e == cudaSuccess) e = attn_configure_one<G, 1, true, true>();
     if (e == cudaSuccess) e = attn_configure_one<G, kRing, true, true>();
     if (e == cudaSuccess) e = attn_configure_one<G, 1, false, true>();
@@ -743,9 +743,13 @@ static cudaError_t attn_configure() {
 
 template <int G, bool CONTIG>
 static cudaError_t attn_dispatch2(bool one_tile, bool cluster, dim3 grid, cudaStream_t st, const AttnArgs& a) {
-    if (cluster)
-        return one_tile ? attn_launch_g<G, 1, true, CONTIG>(grid, st, a) : attn_launch_g<G, kRing, true, CONTIG>(grid, st, a);
-    return one_tile ? attn_launch_g<G, 1, false, CONTIG>(grid, st, a) : attn_launch_g<G, kRing, false, CONTIG>(grid, st, a);
+    if constexpr (!CONTIG) {  // the gather: one stage (each warp keeps the next tile in registers)
+        return cluster ? attn_launch_g<G, 1, true, false>(grid, st, a) : attn_launch_g<G, 1, false, false>(grid, st, a);
+    } else {
+        if (cluster)
+            return one_tile ? attn_launch_g<G, 1, true, true>(grid, st, a) : attn_launch_g<G, kRing, true, true>(grid, st, a);
+        return one_tile ? attn_launch_g<G, 1, false, true>(grid, st, a) : attn_launch_g<G, kRing, false, true>(grid, st, a);
+    }
 }
 
 template <int G>
