@@ -14,7 +14,7 @@
 //
 // Design (per CTA: one unit, a range of 128-row tiles; 6 warps):
 //   warp 0  TMA producer: 2-D tensor loads (box 64 dims x 128 rows, 128-byte
-//           swizzle) of K into a 3-stage shared-memory ring, completing on
+//           swizzle) of K into a 2-stage shared-memory ring, completing on
 //           "full" mbarriers;
 //   warp 1  MMA issuer: tcgen05.mma kind::f16 (bf16 in, fp32 accumulate),
 //           M = 128 rows, N = 16 (the g <= 8 query heads, zero-padded),
@@ -39,11 +39,12 @@ namespace tsa {
 constexpr int kTcThreads = 192;         // 6 warps
 constexpr int kTcTileRows = 128;        // M
 constexpr int kTcN = 16;                // N: query heads padded to 16
-constexpr int kTcStages = 3;
+constexpr int kTcStages = 2;  // 2 x 32 KB in flight per CTA, 2 CTAs per SM (measured: 2 >= 3 > 4)
 constexpr int kTcHalfBytes = kTcTileRows * 128;       // 64 dims x 128 rows x 2 B = 16 KB
 constexpr int kTcStageBytes = 2 * kTcHalfBytes;       // the full 128-dim tile: 32 KB
 constexpr int kTcQHalfBytes = kTcN * 128;             // 16 rows x 128 B = 2 KB
-constexpr int kTcTilesPerCta = 16;                    // 2048 rows per CTA
+constexpr int kTcTilesPerCta = 32;                    // 4096 rows per CTA (the 128K scan: 256 CTAs, one wave)
+constexpr int kTcSms = 148;
 constexpr int kTcSmem = 1024 /*align slack*/ + kTcStages * kTcStageBytes + 2 * kTcQHalfBytes;
 constexpr long kTcSpins = 1L << 22;
 // instruction descriptor: D f32 (bits 4-5 = 1), A bf16 (7-9 = 1), B bf16 (10-12 = 1),
@@ -306,8 +307,12 @@ cudaError_t launch_score_tc(const void* Q, const void* K, const int32_t* lens, c
         }
         g_tc_configured[dev] = 1;
     }
+    // 32 tiles a CTA, unless that leaves SMs idle (short or few units): then
+    // about two CTAs per SM
     const int tiles = ceil_div(d.Ncap, kTcTileRows);
-    const int per = kTcTilesPerCta;
+    int per = kTcTilesPerCta;
+    if ((long long)d.units() * ceil_div(tiles, per) < kTcSms)
+        per = max(1, ceil_div(tiles * d.units(), 2 * kTcSms));
     dim3 grid(ceil_div(tiles, per), d.units());
     const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(Q);
     cudaLaunchConfig_t cfg = {};
