@@ -132,8 +132,10 @@ __device__ __forceinline__ int roff(int row, int chunk) { return row * kRowStrid
 // one 128-token block in block mode) and arrives by 2-D TMA tensor loads in the
 // 128-byte-swizzled layout (4 loads per tile); otherwise each row is its own
 // 256-byte bulk copy into rows padded to 272 bytes.
-template <int G, int STAGES, bool CLUSTER, bool CONTIG>
-__global__ void __launch_bounds__(kAttnThreads)
+// ONE (gather only): every CTA's range is one tile; rows are copied straight into
+// shared memory (cp.async) instead of through registers, so two CTAs fit an SM.
+template <int G, int STAGES, bool CLUSTER, bool CONTIG, bool ONE>
+__global__ void __launch_bounds__(kAttnThreads, ONE ? 2 : 1)
 attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
             const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
             const __nv_bfloat16* __restrict__ V, const int32_t* __restrict__ lens,
@@ -299,7 +301,38 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
             pv[j] = rr >= 0 ? ld_stream(Vu + (size_t)rr * kD + 8 * c16) : make_uint4(0, 0, 0, 0);
         }
     };
-    if (!CONTIG && ntiles > 0) fetch(0);  // in flight while Q is read
+    // ONE: cp.async copies of tile t's rows of this warp (zeros for rows not in the set)
+    uint32_t vm_one = 0;
+    auto issue_one = [&](int t) {
+        int myrow = -1;
+        if (lane < 16) {
+            const int pos = p0 + t * kTileRows + r0 + lane;
+            if (pos < p1) myrow = row_of(pos);
+        }
+        vm_one = __ballot_sync(0xffffffffu, myrow >= 0) & 0xffffu;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int rr = __shfl_sync(0xffffffffu, myrow, hl + 2 * j);
+            unsigned char* kd = kw + (hl + 2 * j) * kRowStride + 16 * c16;
+            unsigned char* vd = vw + (hl + 2 * j) * kRowStride + 16 * c16;
+            if (rr >= 0) {
+                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(kd)),
+                             "l"(Ku + (size_t)rr * kD + 8 * c16) : "memory");
+                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(vd)),
+                             "l"(Vu + (size_t)rr * kD + 8 * c16) : "memory");
+            } else {
+                *reinterpret_cast<uint4*>(kd) = make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4*>(vd) = make_uint4(0, 0, 0, 0);
+            }
+        }
+        asm volatile("cp.async.commit_group;\n" ::: "memory");
+    };
+    if constexpr (!CONTIG) {
+        if (ntiles > 0) {  // in flight while Q is read
+            if constexpr (ONE) issue_one(0);
+            else fetch(0);
+        }
+    }
 
     // A fragments of Q (bf16, unscaled: the scale is applied to S in fp32).
     // Row g of A = query head g of the group (zero for g >= G); rows g+8 are zero.
@@ -424,6 +457,14 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
             }
             __syncthreads();  // every warp is done with this stage
             if (tid == 0) stage_contig(t + STAGES, next_first);  // refill it (nothing past the end)
+        }
+    } else if constexpr (ONE) {
+        for (int t = 0; t < ntiles; ++t) {  // one tile (any count stays correct, unpipelined)
+            if (t > 0) issue_one(t);
+            asm volatile("cp.async.wait_all;\n" ::: "memory");
+            __syncwarp();
+            if (vm_one) warp_tile(sbase, sbase + kTileRows * kRowStride, vm_one);
+            __syncwarp();  // the math has read these rows before the next copies land
         }
     } else {
         for (int t = 0; t < ntiles; ++t) {
@@ -637,7 +678,7 @@ static int g_attn_configured[64];
 // workspace (sized for them in either case).
 static int g_max_clusters[64][4][2][2][kClusterMax + 1];  // dev, log2 G, one-tile, contig, S; 0 = unknown
 
-template <int G, int STAGES, bool CONTIG>
+template <int G, int STAGES, bool CONTIG, bool ONE>
 static int max_active_clusters(int S) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)S, 1);
@@ -651,7 +692,7 @@ static int max_active_clusters(int S) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, attn_kernel<G, STAGES, true, CONTIG>, &cfg) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveClusters(&n, attn_kernel<G, STAGES, true, CONTIG, ONE>, &cfg) != cudaSuccess) {
         cudaGetLastError();  // clear it: the workspace combine is always available
         return -1;
     }
@@ -664,8 +705,8 @@ static bool attn_cluster_fits_g(int dev, bool one_tile, bool contig, int S, int 
     int& slot = g_max_clusters[dev][lg][one_tile][contig][S];
     if (slot == 0) {
         int n;
-        if (!contig) n = max_active_clusters<G, 1, false>(S);
-        else n = one_tile ? max_active_clusters<G, 1, true>(S) : max_active_clusters<G, kRing, true>(S);
+        if (!contig) n = one_tile ? max_active_clusters<G, 1, false, true>(S) : max_active_clusters<G, 1, false, false>(S);
+        else n = one_tile ? max_active_clusters<G, 1, true, false>(S) : max_active_clusters<G, kRing, true, false>(S);
         slot = n;
     }
     return slot > 0 && units <= slot;
@@ -699,7 +740,7 @@ struct AttnArgs {
     int early;
 };
 
-template <int G, int STAGES, bool CLUSTER, bool CONTIG>
+template <int G, int STAGES, bool CLUSTER, bool CONTIG, bool ONE = false>
 static cudaError_t attn_launch_g(dim3 grid, cudaStream_t st, const AttnArgs& a) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
@@ -714,14 +755,14 @@ static cudaError_t attn_launch_g(dim3 grid, cudaStream_t st, const AttnArgs& a) 
     attr[1] = pdl_attr();
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, attn_kernel<G, STAGES, CLUSTER, CONTIG>, a.kmap, a.vmap, a.q, a.k, a.v, a.lens,
+    return cudaLaunchKernelEx(&cfg, attn_kernel<G, STAGES, CLUSTER, CONTIG, ONE>, a.kmap, a.vmap, a.q, a.k, a.v, a.lens,
                               a.idx, a.kreq, a.k_max, a.block, a.Hkv, a.Ncap, a.sl2, a.splits, a.partials, a.counters,
                               a.O, a.flag, a.early);
 }
 
-template <int G, int STAGES, bool CLUSTER, bool CONTIG>
+template <int G, int STAGES, bool CLUSTER, bool CONTIG, bool ONE = false>
 static cudaError_t attn_configure_one() {
-    const void* f = (const void*)attn_kernel<G, STAGES, CLUSTER, CONTIG>;
+    const void* f = (const void*)attn_kernel<G, STAGES, CLUSTER, CONTIG, ONE>;
     cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          AttnCfg<G>::smem_bytes(STAGES, CLUSTER));
     if (e == cudaSuccess && CLUSTER) e = cudaFuncSetAttribute(f, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
@@ -734,6 +775,8 @@ static cudaError_t attn_configure() {
     // the gather runs one stage; contiguous tiles one or kRing
     if (e == cudaSuccess) e = attn_configure_one<G, 1, true, false>();
     if (e == cudaSuccess) e = attn_configure_one<G, 1, false, false>();
+    if (e == cudaSuccess) e = attn_configure_one<G, 1, true, false, true>();
+    if (e == cudaSuccess) e = attn_configure_one<G, 1, false, false, true>();
     if (e == cudaSuccess) e = attn_configure_one<G, 1, true, true>();
     if (e == cudaSuccess) e = attn_configure_one<G, kRing, true, true>();
     if (e == cudaSuccess) e = attn_configure_one<G, 1, false, true>();
@@ -743,7 +786,10 @@ static cudaError_t attn_configure() {
 
 template <int G, bool CONTIG>
 static cudaError_t attn_dispatch2(bool one_tile, bool cluster, dim3 grid, cudaStream_t st, const AttnArgs& a) {
-    if constexpr (!CONTIG) {  // the gather: one stage (each warp keeps the next tile in registers)
+    if constexpr (!CONTIG) {  // the gather: one stage; one tile a CTA -> the cp.async instance
+        if (one_tile)
+            return cluster ? attn_launch_g<G, 1, true, false, true>(grid, st, a)
+                           : attn_launch_g<G, 1, false, false, true>(grid, st, a);
         return cluster ? attn_launch_g<G, 1, true, false>(grid, st, a) : attn_launch_g<G, 1, false, false>(grid, st, a);
     } else {
         if (cluster)
@@ -807,8 +853,9 @@ cudaError_t launch_attn(const void* Q, const void* K, const void* V, const int32
     const bool contig = idx == nullptr || block == kTileRows;
     const long long per_split = contig ? ((rows + splits - 1) / splits + kTileRows - 1) / kTileRows * kTileRows
                                        : (rows + splits - 1) / splits;
-    // one stage: a tile at a time (contiguous tiles), or the warp-private gather
-    const bool one_tile = !contig || per_split <= kTileRows;
+    // one tile a CTA: the single-stage kernel (contiguous tiles), or the gather's
+    // two-CTAs-an-SM instance
+    const bool one_tile = per_split <= kTileRows;
     const bool cluster = attn_cluster_fits(d.G, one_tile, contig, splits, d.units());
     AttnArgs a;
     memset(&a.kmap, 0, sizeof a.kmap);
