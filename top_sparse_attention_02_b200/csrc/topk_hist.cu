@@ -55,6 +55,8 @@ struct ThSmem {
     uint32_t ncand;                            // rank 0: keys posted
     uint32_t over;                             // rank 0: some list overflowed
     uint32_t Tk[3];                            // rank 0 -> all: T, krem, fallback
+    uint32_t small[64];                        // rank 0: keys sharing the first two digits
+    uint32_t nsmall;
 };
 
 __device__ __forceinline__ uint32_t th_block_scan(uint32_t x, uint32_t* wsum, uint32_t* total) {
@@ -254,15 +256,53 @@ topk_hist_kernel(const float* __restrict__ scores, const int32_t* __restrict__ l
             pre |= sm.sel[0] << 10;
             pm |= 0x7ffu << 10;
             kr -= sm.sel[1];
-            // digit 3 over the few keys that share the first two
+            // digit 3: the keys sharing the first two are usually a handful, so
+            // one warp ranks them directly; more (ties) take a histogram pass
+            if (tid == 0) sm.nsmall = 0u;
+            __syncthreads();
             for (uint32_t i = tid; i < nc; i += kThThreads) {
                 const uint32_t k = sm.cand[i];
-                if ((k & pm) == pre) atomicAdd(&sm.gh[k & 0x3ffu], 1u);
+                if ((k & pm) == pre) {
+                    const uint32_t q = atomicAdd(&sm.nsmall, 1u);
+                    if (q < 64u) sm.small[q] = k;
+                }
             }
             __syncthreads();
-            select_bin(sm.gh, 1024, kr);
-            pre |= sm.sel[0];
-            kr -= sm.sel[1];
+            const uint32_t ns = sm.nsmall;  // >= kr >= 1
+            if (ns <= 64u) {
+                if (warp == 0) {
+                    // T is the key x with #{y > x} < kr <= #{y >= x}; krem = kr - #{y > x}
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const uint32_t me = (uint32_t)(lane + 32 * h);
+                        if (me < ns) {
+                            const uint32_t x = sm.small[me];
+                            uint32_t gt = 0, ge = 0;
+                            for (uint32_t j = 0; j < ns; ++j) {
+                                const uint32_t y = sm.small[j];
+                                gt += y > x;
+                                ge += y >= x;
+                            }
+                            if (gt < kr && kr <= ge) {  // every lane holding T writes the same
+                                sm.sel[0] = x;
+                                sm.sel[1] = gt;
+                            }
+                        }
+                    }
+                }
+                __syncthreads();
+                pre = sm.sel[0];
+                kr -= sm.sel[1];
+            } else {
+                for (uint32_t i = tid; i < nc; i += kThThreads) {
+                    const uint32_t k = sm.cand[i];
+                    if ((k & pm) == pre) atomicAdd(&sm.gh[k & 0x3ffu], 1u);
+                }
+                __syncthreads();
+                select_bin(sm.gh, 1024, kr);
+                pre |= sm.sel[0];
+                kr -= sm.sel[1];
+            }
         }
         if (tid < C) {
             uint32_t* d = cluster.map_shared_rank(sm.Tk, tid);
