@@ -10,15 +10,19 @@
 // Flux Attention router or a HyLRA sensitive layer chooses).
 //
 // Design: grid = (split, unit); a CTA is 8 warps and owns a contiguous range of
-// the unit's index list, walked in tiles of 128 rows (16 per warp).  The rows' K
-// and V (256 B each) are gathered into shared memory by the TMA engine, one
-// 256-byte bulk copy (cp.async.bulk) per K or V row completing on the stage's
-// mbarrier; rows are padded to 272 B so the tensor-core fragment loads below are
-// free of bank conflicts.  (16-byte cp.async copies issue from the load/store
-// unit, whose in-flight capacity held a gather to ~33 GB/s per SM.)  The index reads of the first three
-// tiles go out in one round, then all their copies, so a split of up to 384
-// rows has every gather in flight at once; a longer range refills each stage
-// as soon as its tile is consumed (one stage when the range fits in a tile).  Each warp then runs, on its
+// the unit's index list, walked in tiles of 128 rows (16 per warp).  Two ways
+// of bringing a tile's K and V (256 B a row) into shared memory:
+//   - gather (an index list of tokens): each warp fetches its own 16 rows with
+//     16-byte vector loads (a half-warp per row) one tile ahead in registers,
+//     or, when the CTA's range is a single tile, with cp.async straight into
+//     shared memory (no registers held, so two CTAs fit an SM); rows are padded
+//     to 272 B so the fragment loads below are free of bank conflicts, and no
+//     barrier wider than a warp is needed per tile.  (One TMA bulk copy per
+//     256-byte row was the first design: issuing them cost ~13 ns a copy.)
+//   - contiguous tiles (full attention, or a 128-token block): four 2-D TMA
+//     tensor loads a tile in the 128-byte swizzle into a 3-stage ring, each
+//     stage completing on an mbarrier, refilled as soon as it is consumed.
+// Each warp then runs, on its
 // 16 rows, the two contractions of flash decoding on the tensor cores
 // (mma.sync m16n8k16, bf16 in, fp32 accumulate), with the g <= 8 query heads as
 // the M dimension padded to 16:
