@@ -176,9 +176,9 @@ topk_stream_kernel(const float* __restrict__ scores, const int32_t* __restrict__
     const uint32_t lt = (1u << lane) - 1u;
 
     // ---- filter into the per-warp lists (index order within each warp).  Most
-    // keys fail, so a batch is first tested as raw floats against the smallest
-    // float whose key reaches digit d0 (the key order is the float order, -0 =
-    // +0; NaN passes and is sorted out by its key), one vote for the batch.
+    // keys fail, so each 32 rows are first tested as raw floats against the
+    // smallest float whose key reaches digit d0 (the key order is the float
+    // order, -0 = +0; NaN passes and is sorted out by its key), one vote each.
     uint32_t* lkey = ts_list + warp * wcap;
     uint32_t* lrow = ts_list + W * wcap + warp * wcap;
     bool list_mode = kept <= (uint32_t)(W * wcap);
@@ -193,15 +193,15 @@ topk_stream_kernel(const float* __restrict__ scores, const int32_t* __restrict__
                 const int i = base + j * 32 + lane;
                 v[j] = i < we ? __ldcg(su + i) : 0.f;
             }
-            bool any = false;
-#pragma unroll
-            for (int j = 0; j < kTsNB; ++j) any |= (base + j * 32 + lane < we) && !(v[j] < fthr);
-            if (!__any_sync(0xffffffffu, any)) continue;
 #pragma unroll
             for (int j = 0; j < kTsNB; ++j) {
                 const int i = base + j * 32 + lane;
+                // one vote per 32 rows: with k a fraction of a percent of the rows,
+                // most steps have no candidate and end here
+                const bool maybe = i < we && !(v[j] < fthr);
+                if (__ballot_sync(0xffffffffu, maybe) == 0u) continue;
                 const uint32_t k = order_key(v[j]);
-                const bool keep = i < we && (k >> 21) >= d0;
+                const bool keep = maybe && (k >> 21) >= d0;
                 const uint32_t bal = __ballot_sync(0xffffffffu, keep);
                 const uint32_t pos = cnt + __popc(bal & lt);
                 if (keep && pos < (uint32_t)wcap) {
