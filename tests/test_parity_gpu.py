@@ -396,3 +396,21 @@ def test_decode_step_topk_from_the_scorers_histogram(cuda_dev, case):
         compare_idx(idx.cpu().numpy(), S, lens, kreq)
         ref = oracle.attn(L.Q, L.K, L.V, L.seq_lens, idx.cpu().numpy(), kreq, k_max, 1, SCALE)
         check_output(O.cpu().numpy(), ref, f"{case} step {rep}")
+
+
+@pytest.mark.parametrize("N,lens,kreq", [(12000, [12000, 9000], [150, 2]),
+                                         (200000, [200000, 123457], [4000, 2469])])
+def test_decode_step_topk_cluster_shapes(cuda_dev, N, lens, kreq):
+    """The decode step's top-k on a cluster of one CTA (12000 rows) and on 32
+    scores a thread in a cluster of 7 (200000 rows); both steps on one workspace."""
+    B, Hq, Hkv = 2, 8, 2
+    L = layer(B, Hq, Hkv, N, lens, seed=83)
+    Q, K, V, ln = G.to_dev(L, cuda_dev)
+    k_max = max(kreq)
+    ws = G.ws_for(Q, K, k_max, 1, tsa.SELECT)
+    S = oracle.scores(L.Q, L.K, L.seq_lens, SCALE)
+    for rep in range(2):
+        O, idx = G.step(Q, K, V, ln, mode=tsa.SELECT, scale=SCALE, k_max=k_max, kreq=kreq, ws=ws)
+        compare_idx(idx.cpu().numpy(), S, lens, kreq)
+        ref = oracle.attn(L.Q, L.K, L.V, L.seq_lens, idx.cpu().numpy(), kreq, k_max, 1, SCALE)
+        check_output(O.cpu().numpy(), ref, f"N={N} step {rep}")
