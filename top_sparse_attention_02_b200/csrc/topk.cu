@@ -13,10 +13,9 @@
 //           and adds its non-zero bins into every cluster member's copy of the
 //           cluster histogram (remote atomic adds over distributed shared
 //           memory); after one cluster barrier each CTA holds the full
-//           histogram and finds the bin of T with a block-wide scan from the top.
-//           Inside a decode step the scorer has already counted this digit
-//           (its epilogue, hidden behind HBM): every CTA copies the unit's
-//           histogram instead, and rank 0 zeroes it for the next step;
+//           histogram and finds the bin of T with a block-wide scan from the top
+//           (inside a decode step, where the scorer has counted this digit
+//           already, topk_hist.cu and topk_stream.cu start from its histogram);
 //   filter: one pass over the keys keeps, in index order, those whose top digit
 //           is at or above that bin (every selected key plus the candidates of
 //           the boundary bin: ~2-10% of the keys);
@@ -75,8 +74,7 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t x, uint32_t* wsum, 
 __global__ void __launch_bounds__(kTkThreads, 1)
 topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ lens,
             const int32_t* __restrict__ kreq, int k_max, int Hkv, int Ncap, int rows_cap, int block,
-            int chunk, int32_t* __restrict__ idx, uint32_t* __restrict__ hist,
-            unsigned* __restrict__ flag) {
+            int chunk, int32_t* __restrict__ idx, unsigned* __restrict__ flag) {
     cg::cluster_group cluster = cg::this_cluster();
     const int C = (int)cluster.num_blocks();
     const int rank = (int)cluster.block_rank();
@@ -117,18 +115,14 @@ topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ lens,
     int32_t* out = idx + (size_t)unit * k_max;
     const int lo = rank * chunk;
     const int nloc = max(0, min(chunk, n - lo));
-    uint32_t* hu = hist ? hist + (size_t)unit * kHistBins : nullptr;  // the scorer's top-digit counts
 
     // Degenerate units need no selection; every CTA of the cluster takes the
     // same branch, so no cluster barrier is left waiting.
     if (kb == 0 || kb == n) {
         for (int i = tid; i < nloc; i += kTkThreads)
             if (lo + i < kb) out[lo + i] = lo + i;
-        if (rank == 0) {
+        if (rank == 0)
             for (int p = kb + tid; p < k_max; p += kTkThreads) out[p] = -1;
-            if (hu)
-                for (int i = tid; i < kHistBins; i += kTkThreads) hu[i] = 0u;  // ready for the next step
-        }
         return;
     }
 
@@ -167,61 +161,32 @@ topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ lens,
         }
         __syncthreads();
     };
-    if (hu) {
-        // the scorer counted the top digit already: its histogram is the
-        // cluster histogram (every CTA takes a copy; rank 0 zeroes it once all
-        // have, below)
-        if (tid < kTkHist / 4) reinterpret_cast<uint4*>(gh)[tid] = __ldcg(reinterpret_cast<const uint4*>(hu) + tid);
-        for (int i = tid; i < kTkHist; i += kTkThreads) gh[kTkHist + i] = 0u;
-        if (tid == 0) s_ncand = 0u;
-        // split cluster barrier: arrive now (copy taken, s_ncand zero), wait
-        // before the first remote access
-        asm volatile("barrier.cluster.arrive.aligned;\n" ::: "memory");
-        for (int i0 = 0; i0 < nloc; i0 += kBatch * kTkThreads) {
-            if (i0 > 0) {
-#pragma unroll
-                for (int j = 0; j < kBatch; ++j) {
-                    const int i = i0 + tid + j * kTkThreads;
-                    f[j] = i < nloc ? __ldcg(su + i) : 0.f;
-                }
-            }
+    for (int i = tid; i < 3 * kTkHist; i += kTkThreads) lh[i] = 0u;  // lh, gh[0], gh[1]
+    if (tid == 0) s_ncand = 0u;
+    cluster.sync();  // every CTA's cluster histograms are zero before anyone adds to them
+
+    // ---- pass 0: keys to shared memory, local histogram of the top digit
+    for (int i0 = 0; i0 < nloc; i0 += kBatch * kTkThreads) {
+        if (i0 > 0) {
 #pragma unroll
             for (int j = 0; j < kBatch; ++j) {
                 const int i = i0 + tid + j * kTkThreads;
-                if (i < nloc) keys[i] = order_key(f[j]);
+                f[j] = i < nloc ? __ldcg(su + i) : 0.f;
             }
         }
-        asm volatile("barrier.cluster.wait.aligned;\n" ::: "memory");
-        if (rank == 0)
-            for (int i = tid; i < kHistBins; i += kTkThreads) hu[i] = 0u;  // every member has its copy
-    } else {
-        for (int i = tid; i < 3 * kTkHist; i += kTkThreads) lh[i] = 0u;  // lh, gh[0], gh[1]
-        if (tid == 0) s_ncand = 0u;
-        cluster.sync();  // every CTA's cluster histograms are zero before anyone adds to them
-
-        // ---- pass 0: keys to shared memory, local histogram of the top digit
-        for (int i0 = 0; i0 < nloc; i0 += kBatch * kTkThreads) {
-            if (i0 > 0) {
 #pragma unroll
-                for (int j = 0; j < kBatch; ++j) {
-                    const int i = i0 + tid + j * kTkThreads;
-                    f[j] = i < nloc ? __ldcg(su + i) : 0.f;
-                }
+        for (int j = 0; j < kBatch; ++j) {
+            const int i = i0 + tid + j * kTkThreads;
+            if (i < nloc) {
+                const uint32_t k = order_key(f[j]);
+                keys[i] = k;
+                atomicAdd(&lh[k >> 21], 1u);
             }
-#pragma unroll
-            for (int j = 0; j < kBatch; ++j) {
-                const int i = i0 + tid + j * kTkThreads;
-                if (i < nloc) {
-                    const uint32_t k = order_key(f[j]);
-                    keys[i] = k;
-                    atomicAdd(&lh[k >> 21], 1u);
-                }
-            }
-    }
-        __syncthreads();
-        push_hist(gh, kTkHist);
-        cluster.sync();  // every CTA now holds the cluster histogram of the top digit
-    }
+        }
+}
+    __syncthreads();
+    push_hist(gh, kTkHist);
+    cluster.sync();  // every CTA now holds the cluster histogram of the top digit
     select_bin(gh, kTkHist, (uint32_t)kb);
     const uint32_t d0 = s_sel[0];
     uint32_t krem = (uint32_t)kb - s_sel[1];
@@ -421,6 +386,10 @@ cudaError_t launch_topk(const float* scores, const int32_t* lens, const int32_t*
     int hc = 1, hk = 16;
     if (hist && topk_hist_plan(d.units(), rows_cap, &hc, &hk))
         return launch_topk_hist(hc, hk, scores, lens, kreq, k_max, d, block, idx, hist, flag, st);
+    if (hist) {  // a shape neither histogram-fed kernel takes: count afresh, leave the counts zero
+        const cudaError_t e = cudaMemsetAsync(hist, 0, (size_t)d.units() * kHistBins * sizeof(uint32_t), st);
+        if (e != cudaSuccess) return e;
+    }
     int C = 1, chunk = 32;
     if (!topk_plan(rows_cap, &C, &chunk)) return cudaErrorInvalidValue;
     int dev = 0;
@@ -447,7 +416,7 @@ cudaError_t launch_topk(const float* scores, const int32_t* lens, const int32_t*
     cfg.attrs = attr;
     cfg.numAttrs = 2;
     e = cudaLaunchKernelEx(&cfg, topk_kernel, scores, lens, kreq, k_max, d.Hkv, d.Ncap, rows_cap,
-                           block, chunk, idx, hist, flag);
+                           block, chunk, idx, flag);
     note_launch();
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
