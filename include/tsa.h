@@ -165,23 +165,57 @@ typedef struct {
     const void* Q;            /* [B, Hq, d] bf16 */
     const void* K;            /* [B, Hkv, Ncap, d] bf16 */
     const void* V;            /* [B, Hkv, Ncap, d] bf16 */
-    const float* Kmean;       /* block mode SELECT only: output of tsa_block_summarize */
+    const float* Kmean;       /* block mode SELECT (and FULL with idx_out): from tsa_block_summarize */
     const int32_t* seq_lens;  /* [B] */
     const int32_t* k_per_seq; /* [B] or NULL (= k_max) */
-    int32_t k_max;            /* columns of idx; ignored for TSA_FULL */
+    int32_t k_max;            /* columns of idx; TSA_FULL: used only with idx_out */
     int32_t block;            /* 1 = token mode, > 1 = block mode (128 in the pages) */
     int32_t mode;             /* TSA_FULL, TSA_SELECT or TSA_REUSE */
     float scale;              /* softmax scale, > 0 (1/sqrt(d) usually) */
     const int32_t* idx_in;    /* TSA_REUSE: the earlier layer's idx [B, Hkv, k_max] */
-    int32_t* idx_out;         /* TSA_SELECT: this layer's idx [B, Hkv, k_max] */
+    int32_t* idx_out;         /* TSA_SELECT: this layer's idx [B, Hkv, k_max];
+                               * TSA_FULL: NULL, or where the layer's own top-k goes */
     float* O;                 /* [B, Hq, d] fp32 */
     void* ws;                 /* workspace */
     size_t ws_bytes;
 } tsa_step_args;
 
 /* One decode step of one layer: TSA_SELECT = score -> top-k -> attention;
- * TSA_REUSE = attention over idx_in; TSA_FULL = attention over every valid row. */
+ * TSA_REUSE = attention over idx_in; TSA_FULL = attention over every valid row.
+ * A TSA_FULL layer given idx_out (and k_max > 0) also writes the top-k that a
+ * SELECT step would have chosen, so that the tolerant layers after it can reuse
+ * it (HyLRA, sec. 2.3: the indices of a sensitive, fully attended layer are
+ * handed on).  Token mode: the full attention writes each row's group-max
+ * scaled score as it forms the logits, then the top-k runs on those; block
+ * mode: the block means (Kmean) are scored first.  O is unchanged by idx_out;
+ * the workspace must then be sized with tsa_workspace_size(shape, k_max,
+ * block, TSA_FULL), k_max > 0. */
 tsa_status tsa_decode_step(const tsa_step_args* args, void* stream);
+
+/* ------------------------------------------------------------------ reuse profiling */
+
+/* Overlap of the top-k index sets of n_layers layers: the similarity matrix
+ * that HyLRA's offline policy search runs on (HyLRA sec. 2.2; M[i][j] there is
+ * the overlap ratio of the top-k indices of source layer i and target layer j).
+ *  - idx [n_layers, units, k_max] int32 (device): layer l's index lists for the
+ *    units (b, kvh), units = B * Hkv, each in the form of `idx` above
+ *    (ascending, then -1), e.g. the idx_out of n_layers decode steps.
+ *  - counts [n_layers, n_layers, units] int32 (device) or NULL:
+ *    counts[(i*n_layers + j)*units + u] = |I_i(u) ∩ I_j(u)| for every i, j
+ *    (symmetric; the diagonal holds the list lengths |I_i(u)|).  Exact.
+ *  - M [n_layers, n_layers] double (device) or NULL: for source i <= target j,
+ *    M[j*n_layers + i] = the mean over the units with |I_j(u)| > 0 of
+ *    |I_i(u) ∩ I_j(u)| / |I_j(u)| (the share of the target layer's top-k that
+ *    reusing layer i's indices keeps), summed in unit order; 1 when every
+ *    target list is empty; M[i*n_layers + j] = 0 for i < j.  So M is lower
+ *    triangular with row = target layer, column = source layer.
+ *  - Not both counts and M NULL; 1 <= n_layers <= 1024; ws: the first 256
+ *    bytes (the device flag) are used.
+ *  - A list that is not strictly ascending before its first -1, or holds
+ *    anything but -1 after it, sets the device bounds flag
+ *    (tsa_check_device_status); the results for that pair are then unspecified. */
+tsa_status tsa_index_overlap(const int32_t* idx, int32_t n_layers, int32_t units, int32_t k_max,
+                             int32_t* counts, double* M, void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------ status */
 

@@ -182,6 +182,33 @@ def attn(Q, K, V, seq_lens, idx, kreq, k_max: int, block: int, scale: float,
     return O
 
 
+def index_overlap(idx):
+    """Overlap of L layers' index sets (HyLRA, sec. 2.2: the similarity matrix M of
+    top-k overlap ratios between a source layer i and a target layer j).
+
+    idx: int [L, B, Hkv, k_max] (or [L, units, k_max]), each list ascending then -1.
+    Returns (counts, M): counts int64 [L, L, units] = |I_i(u) ∩ I_j(u)| by numpy's
+    set intersection; M float64 [L, L] lower triangular (row = target j, column =
+    source i <= j): the mean, over the units whose target set is non-empty, of
+    |I_i ∩ I_j| / |I_j| (1 if there is no such unit), 0 above the diagonal."""
+    a = np.asarray(idx)
+    L, k_max = a.shape[0], a.shape[-1]
+    units = int(np.prod(a.shape[1:-1]))
+    a = a.reshape(L, units, k_max)
+    sets = [[a[l, u][a[l, u] >= 0] for u in range(units)] for l in range(L)]
+    counts = np.zeros((L, L, units), dtype=np.int64)
+    for i in range(L):
+        for j in range(L):
+            for u in range(units):
+                counts[i, j, u] = np.intersect1d(sets[i][u], sets[j][u]).size
+    M = np.zeros((L, L))
+    for j in range(L):
+        for i in range(j + 1):
+            ratios = [counts[i, j, u] / sets[j][u].size for u in range(units) if sets[j][u].size > 0]
+            M[j, i] = float(np.mean(ratios)) if ratios else 1.0
+    return counts, M
+
+
 def nblocks_of(seq_lens, block: int) -> np.ndarray:
     L = _i32(seq_lens)
     return ((L.astype(np.int64) + block - 1) // block).astype(np.int32)

@@ -25,15 +25,15 @@ def block_means(K, lens, block):
 
 
 def step(Q, K, V, lens, *, mode, scale, k_max=0, block=1, kreq=None, Kmean=None, idx_in=None,
-         ws=None, check=True):
-    """One decode step; returns (O, idx) with idx None unless SELECT."""
+         ws=None, check=True, emit=False):
+    """One decode step; returns (O, idx) with idx None unless SELECT (or FULL with emit)."""
     B, Hq, d = Q.shape
     Hkv = K.shape[1]
     if ws is None:
         ws = ws_for(Q, K, k_max, block, mode)
     O = torch.full((B, Hq, d), float("nan"), dtype=torch.float32, device=Q.device)
     idx = None
-    if mode == tsa.SELECT:
+    if mode == tsa.SELECT or emit:
         idx = torch.full((B, Hkv, k_max), -7, dtype=torch.int32, device=Q.device)
     kr = None if kreq is None else torch.as_tensor(kreq, dtype=torch.int32).to(Q.device)
     a = tsa.step_args(Q, K, V, lens, O, ws, mode=mode, scale=scale, k_max=k_max, block=block,

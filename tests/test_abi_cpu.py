@@ -32,7 +32,8 @@ def declared_functions():
 def test_header_declares_the_boundary():
     names = declared_functions()
     for want in ("sparse_decode_score", "topk_select", "sparse_decode_attn", "tsa_decode_step",
-                 "tsa_block_summarize", "tsa_workspace_size", "tsa_check_device_status"):
+                 "tsa_block_summarize", "tsa_workspace_size", "tsa_check_device_status",
+                 "tsa_index_overlap"):
         assert want in names
 
 
@@ -60,6 +61,9 @@ def test_workspace_size_is_host_only_and_ordered(tsa):
     # SELECT adds the fp32 score buffer (units * Ncap * 4 bytes) and the scorer's
     # top-digit histograms (units * 2048 * 4 bytes), each 256-aligned
     assert sel - reu == 2 * 4096 * 4 + 2 * 2048 * 4
+    # a full layer that also hands on its top-k adds the same score and histogram room
+    assert tsa.workspace_size(s, 128, 1, tsa.FULL) - full == 2 * 4096 * 4 + 2 * 2048 * 4
+    assert tsa.workspace_size(s, 128, 128, tsa.FULL) - full == 256 + 2 * 2048 * 4
     big = tsa.tsa_shape(1, 32, 8, 131072, 128)
     assert tsa.workspace_size(big, 2621, 1, tsa.SELECT) >= 8 * 131072 * 4
 
@@ -141,9 +145,28 @@ def test_decode_step_argument_errors(tsa):
     a = tsa.step_args(Q, K, T(0x3000), T(0x4000), T(0x5000), ws, mode=tsa.SELECT, scale=0.1,
                       k_max=16, block=128, idx_out=T(0x7000))
     assert tsa.lib().tsa_decode_step(ctypes.byref(a), None) == 1 and "Kmean" in tsa.last_error()
+    a = tsa.step_args(Q, K, T(0x3000), T(0x4000), T(0x5000), ws, mode=tsa.FULL, scale=0.1, k_max=0,
+                      idx_out=T(0x7000))
+    assert tsa.lib().tsa_decode_step(ctypes.byref(a), None) == 1 and "k_max > 0" in tsa.last_error()
+    a = tsa.step_args(Q, K, T(0x3000), T(0x4000), T(0x5000), ws, mode=tsa.FULL, scale=0.1, k_max=16,
+                      block=128, idx_out=T(0x7000))
+    assert tsa.lib().tsa_decode_step(ctypes.byref(a), None) == 1 and "Kmean" in tsa.last_error()
     a = tsa.step_args(Q, K, T(0x3000), T(0x4000), T(0x5000), ws, mode=9, scale=0.1, k_max=16)
     assert tsa.lib().tsa_decode_step(ctypes.byref(a), None) == 1 and "mode" in tsa.last_error()
     assert tsa.lib().tsa_decode_step(None, None) == 1
+
+
+def test_index_overlap_argument_errors(tsa):
+    L = tsa.lib()
+    assert L.tsa_index_overlap(0x1000, 0, 4, 8, 0x2000, 0x3000, 0x10000, 256, None) == 1
+    assert "n_layers" in tsa.last_error()
+    assert L.tsa_index_overlap(0x1000, 1025, 4, 8, 0x2000, 0x3000, 0x10000, 256, None) == 1
+    assert L.tsa_index_overlap(0x1000, 3, -1, 8, 0x2000, 0x3000, 0x10000, 256, None) == 1
+    assert L.tsa_index_overlap(None, 3, 4, 8, 0x2000, 0x3000, 0x10000, 256, None) == 1
+    assert L.tsa_index_overlap(0x1000, 3, 4, 8, None, None, 0x10000, 256, None) == 1
+    assert "NULL" in tsa.last_error()
+    assert L.tsa_index_overlap(0x1000, 3, 4, 8, 0x2000, None, None, 256, None) == 3
+    assert L.tsa_index_overlap(0x1000, 3, 4, 8, 0x2000, None, 0x10000, 100, None) == 3
 
 
 def test_hbm_copy_argument_errors(tsa):

@@ -315,3 +315,102 @@ def test_empty_sequence_gives_zero_output_and_no_indices():
     Of, _, _ = oracle.decode_step(L.Q, L.K, L.V, L.seq_lens, None, 0, 0.2, mode=0)
     assert (Of[1] == 0).all()
     np.testing.assert_allclose(Of[0], _sdpa_fp64(L.Q[:1], L.K[:1], L.V[:1], [16], 0.2)[0], atol=1e-12)
+
+
+# ------------------------------------------------------------------ layer overlap (HyLRA sec. 2.2)
+
+def _lists(sets, k_max):
+    """Index lists in the library's form: ascending, then -1."""
+    out = np.full((len(sets), len(sets[0]), k_max), -1, dtype=np.int32)
+    for l, per_unit in enumerate(sets):
+        for u, s in enumerate(per_unit):
+            v = sorted(s)
+            out[l, u, :len(v)] = v
+    return out
+
+
+def test_overlap_identical_and_disjoint_layers():
+    """Layers 0 and 1 hold the same sets (ratio 1); layer 2 the odd rows where they
+    hold even ones (ratio 0); the diagonal counts are the set sizes."""
+    even = [set(range(0, 64, 2)), set(range(10, 40, 2))]
+    odd = [set(range(1, 64, 2)), set(range(11, 41, 2))]
+    counts, M = oracle.index_overlap(_lists([even, even, odd], 40))
+    assert (counts[0, 1] == [32, 15]).all() and (counts[0, 2] == 0).all() and (counts[1, 2] == 0).all()
+    assert (np.diagonal(counts, axis1=0, axis2=1).T == [[32, 15], [32, 15], [32, 15]]).all()
+    assert np.allclose(np.diag(M), 1.0) and M[1, 0] == 1.0 and M[2, 0] == 0.0 and M[2, 1] == 0.0
+    assert (M[np.triu_indices(3, 1)] == 0).all()
+
+
+def test_overlap_shifted_window_closed_form():
+    """I_0 = [0, k), I_1 = [s, s + k): |I_0 ∩ I_1| = k - s for 0 <= s <= k."""
+    k = 50
+    for s in (0, 1, 17, 49, 50, 80):
+        counts, M = oracle.index_overlap(_lists([[set(range(k))], [set(range(s, s + k))]], k))
+        assert counts[0, 1, 0] == counts[1, 0, 0] == max(k - s, 0)
+        assert M[1, 0] == max(k - s, 0) / k
+
+
+def test_overlap_normalises_by_the_target_set_and_orients_rows_as_targets():
+    """Source layer 0 holds 4 rows, target layer 1 holds 2 of which 1 is shared:
+    reusing layer 0's indices keeps 1 of the target's 2 (0.5), not 1 of 4 (0.25).
+    With the roles swapped (layer 1 is the source of nothing, as it comes later)
+    M[0, 1] stays 0: the matrix is lower triangular, rows are targets."""
+    counts, M = oracle.index_overlap(_lists([[{3, 5, 7, 9}], [{5, 100}]], 4))
+    assert counts[0, 1, 0] == 1
+    assert M[1, 0] == 0.5 and M[0, 1] == 0.0
+
+
+def test_overlap_mean_over_units_skips_empty_targets():
+    """Units with an empty target list leave the mean; with none left M is 1."""
+    src = [{1, 2, 3, 4}, {1, 2}, {7}]
+    tgt = [{1, 2, 9, 10}, set(), {7}]  # ratios 0.5, (skipped), 1.0
+    counts, M = oracle.index_overlap(_lists([src, tgt], 4))
+    assert M[1, 0] == 0.75
+    _, M0 = oracle.index_overlap(_lists([[set(), set()], [set(), set()]], 3))
+    assert (M0[np.tril_indices(2)] == 1.0).all()
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_overlap_brute_force_tiny(seed):
+    """Random small sets of rows in [0, 30): every count equals the size of the
+    Python set intersection and every M entry the plain mean of the ratios."""
+    rng = np.random.default_rng(seed)
+    L, units, k_max = 4, 5, 9
+    sets = [[set(rng.choice(30, size=int(rng.integers(0, k_max + 1)), replace=False).tolist())
+             for _ in range(units)] for _ in range(L)]
+    counts, M = oracle.index_overlap(_lists(sets, k_max))
+    for i in range(L):
+        for j in range(L):
+            for u in range(units):
+                assert counts[i, j, u] == len(sets[i][u] & sets[j][u])
+            if i <= j:
+                r = [len(sets[i][u] & sets[j][u]) / len(sets[j][u]) for u in range(units) if sets[j][u]]
+                want = sum(r) / len(r) if r else 1.0
+                assert abs(M[j, i] - want) < 1e-15
+            else:  # above the diagonal: a later layer is no source for an earlier one
+                assert M[j, i] == 0.0
+
+
+def test_layer_index_lists_form_and_drift():
+    """The generator's lists have the library's form, and keep = 1 / 0 give
+    identical / (for n >= 2k) disjoint consecutive layers."""
+    lists = inputs.layer_index_lists(3, [100, 7, 0], [20, 20, 5], 24, 1.0, seed=3)
+    a = lists.numpy()
+    for l in range(3):
+        for u, (n, k) in enumerate([(100, 20), (7, 7), (0, 0)]):
+            v = a[l, u]
+            assert (np.diff(v[:k]) > 0).all() and (v[:k] >= 0).all() and (v[:k] < max(n, 1)).all()
+            assert (v[k:] == -1).all()
+    counts, M = oracle.index_overlap(a)
+    assert (M[np.tril_indices(3)] == 1.0).all()
+    _, M0 = oracle.index_overlap(inputs.layer_index_lists(2, [100], [20], 20, 0.0, seed=4).numpy())
+    assert M0[1, 0] == 0.0
+
+
+def test_overlap_degenerate_shapes():
+    """No units, or lists of width 0: every count is 0 and M is 1 on and below
+    the diagonal (no unit has a non-empty target)."""
+    for shape in ((2, 0, 5), (2, 3, 0), (1, 1, 1)):
+        counts, M = oracle.index_overlap(np.full(shape, -1, dtype=np.int32))
+        assert counts.shape == (shape[0], shape[0], shape[1]) and (counts == 0).all()
+        assert (M == np.tril(np.ones((shape[0], shape[0])))).all()

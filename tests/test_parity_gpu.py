@@ -414,3 +414,144 @@ def test_decode_step_topk_cluster_shapes(cuda_dev, N, lens, kreq):
         compare_idx(idx.cpu().numpy(), S, lens, kreq)
         ref = oracle.attn(L.Q, L.K, L.V, L.seq_lens, idx.cpu().numpy(), kreq, k_max, 1, SCALE)
         check_output(O.cpu().numpy(), ref, f"N={N} step {rep}")
+
+
+# ------------------------------------------------------------------ full layers that hand on their top-k
+
+@pytest.mark.parametrize("case", ["ragged", "long", "k_gt_len", "g1"])
+def test_full_step_emits_topk(cuda_dev, case):
+    """A fully attended layer (HyLRA, sec. 2.3: a sensitive layer) also writes
+    the top-k a SELECT step would choose: O is the dense attention, idx the
+    exact top-k of the group-max scaled scores (formed inside the attention);
+    a REUSE step then attends over it."""
+    if case == "ragged":
+        L, kreq = layer(4, 32, 8, 3000, [3000, 1, 129, 0], seed=91, tail_fill=float("nan")), [60] * 4
+    elif case == "long":  # several splits per unit, the top-k from the one-CTA-per-unit kernel
+        L, kreq = layer(2, 16, 4, 70000, [70000, 41234], seed=92), [1400, 800]
+    elif case == "k_gt_len":
+        L, kreq = layer(2, 8, 2, 256, [100, 256], seed=93), [150, 150]
+    else:  # one query head per KV head
+        L, kreq = layer(2, 8, 8, 5000, [5000, 4999], seed=94), [77, 1]
+    k_max = max(kreq)
+    Q, K, V, ln = G.to_dev(L, cuda_dev)
+    ws = G.ws_for(Q, K, k_max, 1, tsa.FULL)
+    assert ws.numel() > G.ws_for(Q, K, 0, 1, tsa.FULL).numel()
+    S = oracle.scores(L.Q, L.K, L.seq_lens, SCALE)
+    ref = oracle.attn(L.Q, L.K, L.V, L.seq_lens, None, None, 0, 1, SCALE)
+    for rep in range(2):
+        O, idx = G.step(Q, K, V, ln, mode=tsa.FULL, scale=SCALE, k_max=k_max, kreq=kreq, ws=ws, emit=True)
+        check_output(O.cpu().numpy(), ref, f"{case} full step {rep}")
+        compare_idx(idx.cpu().numpy(), S, L.seq_lens.numpy(), kreq)
+    O1, _ = G.step(Q, K, V, ln, mode=tsa.REUSE, scale=SCALE, k_max=k_max, kreq=kreq, idx_in=idx)
+    ref1 = oracle.attn(L.Q, L.K, L.V, L.seq_lens, idx.cpu().numpy(), kreq, k_max, 1, SCALE)
+    check_output(O1.cpu().numpy(), ref1, f"{case} reuse of the full layer's top-k")
+
+
+def test_full_step_emits_block_topk(cuda_dev):
+    """Block mode: the full layer scores the block means (HyLRA, sec. 2.4) and
+    hands on the top-k blocks; O is still the dense attention over every row."""
+    L = layer(2, 32, 8, 9000, [9000, 4100], seed=95, plant=0.01)
+    kreq, k_max, block = [32, 20], 32, 128
+    Q, K, V, ln = G.to_dev(L, cuda_dev)
+    Kmean = G.block_means(K, ln, block)
+    ws = G.ws_for(Q, K, k_max, block, tsa.FULL)
+    nrows = oracle.nblocks_of(L.seq_lens, block)
+    S = oracle.block_scores(L.Q, oracle.block_means(L.K, L.seq_lens, block), nrows, SCALE)
+    ref = oracle.attn(L.Q, L.K, L.V, L.seq_lens, None, None, 0, 1, SCALE)
+    for rep in range(2):
+        O, idx = G.step(Q, K, V, ln, mode=tsa.FULL, scale=SCALE, k_max=k_max, block=block, kreq=kreq,
+                        Kmean=Kmean, ws=ws, emit=True)
+        check_output(O.cpu().numpy(), ref, f"block full step {rep}")
+        compare_idx(idx.cpu().numpy(), S, nrows, kreq)
+
+
+# ------------------------------------------------------------------ layer overlap (HyLRA sec. 2.2)
+
+def _overlap_gpu(idx_dev):
+    L = idx_dev.shape[0]
+    units = math.prod(idx_dev.shape[1:-1])
+    counts = torch.full((L, L, units), -7, dtype=torch.int32, device=idx_dev.device)
+    M = torch.full((L, L), float("nan"), dtype=torch.float64, device=idx_dev.device)
+    ws = torch.zeros(256, dtype=torch.uint8, device=idx_dev.device)
+    tsa.index_overlap(idx_dev, counts, M, ws)
+    tsa.check_device_status(ws)
+    torch.cuda.synchronize()
+    return counts.cpu().numpy(), M.cpu().numpy()
+
+
+def _check_overlap(idx):
+    counts, M = _overlap_gpu(idx)
+    c_ref, M_ref = oracle.index_overlap(idx.cpu().numpy())
+    assert (counts == c_ref).all(), "overlap counts differ"
+    assert np.allclose(M, M_ref, rtol=1e-12, atol=0), f"M differs: {np.abs(M - M_ref).max()}"
+    return counts, M
+
+
+@pytest.mark.parametrize("keep", [0.0, 0.7, 1.0])
+def test_index_overlap_random_layers(cuda_dev, keep):
+    """Exact counts for 6 layers x 32 units: ragged k, an empty unit, a full one."""
+    rng = np.random.default_rng(7)
+    n = rng.integers(1, 3000, 32).tolist()
+    n[3] = 0
+    k = [int(min(x, rng.integers(1, 700))) for x in n]
+    k[5] = 700
+    n[5] = max(n[5], 700)
+    idx = inputs.layer_index_lists(6, n, k, 700, keep, seed=11).to(cuda_dev)
+    counts, M = _check_overlap(idx)
+    if keep == 1.0:
+        assert (M[np.tril_indices(6)] == 1.0).all()
+
+
+def test_index_overlap_long_lists_and_degenerate_sizes(cuda_dev):
+    """Lists longer than the shared-memory stage (13000 rows of 40000), one layer,
+    no units, and k_max = 0."""
+    idx = inputs.layer_index_lists(3, [40000, 30000], [13000, 12000], 13000, 0.5, seed=12).to(cuda_dev)
+    _check_overlap(idx)
+    _check_overlap(inputs.layer_index_lists(1, [50], [10], 10, 0.5, seed=13).to(cuda_dev))
+    counts, M = _check_overlap(torch.empty(2, 0, 5, dtype=torch.int32, device=cuda_dev))
+    assert (M == [[1.0, 0.0], [1.0, 1.0]]).all()
+    counts, M = _check_overlap(torch.empty(2, 3, 0, dtype=torch.int32, device=cuda_dev))
+    assert (counts == 0).all() and (M == [[1.0, 0.0], [1.0, 1.0]]).all()
+
+
+def test_index_overlap_flags_malformed_lists(cuda_dev):
+    """A list out of order, or with an entry after its -1, sets the bounds flag."""
+    good = inputs.layer_index_lists(2, [100, 100], [10, 10], 12, 0.5, seed=14)
+    for bad in ("order", "tail"):
+        idx = good.clone()
+        if bad == "order":
+            idx[1, 0, 3], idx[1, 0, 4] = idx[1, 0, 4].item(), idx[1, 0, 3].item()
+        else:
+            idx[0, 1, 11] = 5
+        ws = torch.zeros(256, dtype=torch.uint8, device=cuda_dev)
+        counts = torch.zeros((2, 2, 2), dtype=torch.int32, device=cuda_dev)
+        tsa.index_overlap(idx.to(cuda_dev), counts, None, ws)
+        with pytest.raises(tsa.TsaError, match="BOUNDS"):
+            tsa.check_device_status(ws)
+
+
+def test_index_overlap_of_decode_steps(cuda_dev):
+    """The similarity matrix of a chain of layers as the decode steps select
+    them: a full layer that hands on its top-k, then SELECT layers whose queries
+    drift; the lists go straight from the steps into one [L, B, Hkv, k] tensor."""
+    B, Hq, Hkv, N, kreq, k_max = 2, 16, 4, 8000, [300, 200], 300
+    lens = [8000, 5123]
+    L0 = layer(B, Hq, Hkv, N, lens, seed=101)
+    Q, K, V, ln = G.to_dev(L0, cuda_dev)
+    nl = 5
+    idx = torch.full((nl, B, Hkv, k_max), -7, dtype=torch.int32, device=cuda_dev)
+    ws = G.ws_for(Q, K, k_max, 1, tsa.FULL)
+    O = torch.empty(B, Hq, 128, dtype=torch.float32, device=cuda_dev)
+    kr = torch.tensor(kreq, dtype=torch.int32, device=cuda_dev)
+    q = L0.Q
+    for l in range(nl):
+        if l > 0:
+            q = inputs.drift_query(q, 0.4, 200 + l)
+        a = tsa.step_args(q.to(cuda_dev), K, V, ln, O, ws, mode=tsa.FULL if l == 0 else tsa.SELECT,
+                          scale=SCALE, k_max=k_max, k_per_seq=kr, idx_out=idx[l])
+        tsa.decode_step(a)
+        tsa.check_device_status(ws)
+        S = oracle.scores(q, L0.K, L0.seq_lens, SCALE)
+        compare_idx(idx[l].cpu().numpy(), S, lens, kreq)
+    counts, M = _check_overlap(idx)
+    assert 0.0 < M[1, 0] < 1.0

@@ -8,6 +8,7 @@ module raises.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 
 import torch
@@ -51,6 +52,7 @@ _SIGS = {
     "sparse_decode_attn_noalloc": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, tsa_shape,
                                                   _f32, _vp, _vp]),
     "tsa_decode_step": (ctypes.c_int, [ctypes.POINTER(tsa_step_args), _vp]),
+    "tsa_index_overlap": (ctypes.c_int, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _sz, _vp]),
     "tsa_check_device_status": (ctypes.c_int, [_vp, _vp]),
     "tsa_last_error_string": (ctypes.c_char_p, []),
     "tsa_launch_count": (ctypes.c_uint64, []),
@@ -177,6 +179,14 @@ def step_args(Q, K, V, seq_lens, O, ws, *, mode: int, scale: float, k_max: int =
 
 def decode_step(args: tsa_step_args, stream=None):
     _ok(_lib.tsa_decode_step(ctypes.byref(args), _stream(stream)))
+
+
+def index_overlap(idx, counts, M, ws, stream=None):
+    """Overlap of L layers' index lists idx [L, B, Hkv, k_max] (int32, device) into
+    counts [L, L, B*Hkv] int32 and M [L, L] float64 (either may be None)."""
+    L, units, k_max = idx.shape[0], math.prod(idx.shape[1:-1]), idx.shape[-1]
+    _ok(_lib.tsa_index_overlap(_ptr(idx), L, units, k_max, _ptr(counts), _ptr(M), *_wsargs(ws),
+                               _stream(stream)))
 
 
 def check_device_status(ws, stream=None):

@@ -129,7 +129,8 @@ size_t tsa_workspace_size(tsa_shape shape, int32_t k_max, int32_t block, int32_t
     tsa::Dims d;
     if (check_shape(shape, &d) != TSA_OK || check_block(block) != TSA_OK || check_kmax(k_max) != TSA_OK) return 0;
     switch (mode) {
-        case TSA_FULL: return layout(d, 0, 1, true, true, false).total;
+        case TSA_FULL:  // k_max > 0: room for a layer that also emits its top-k
+            return k_max > 0 ? layout(d, k_max, block, true, true, true).total : layout(d, 0, 1, true, true, false).total;
         case TSA_SELECT: return layout(d, k_max, block, true, false, true).total;
         case TSA_REUSE: return layout(d, k_max, block, true, false, false).total;
         default:
@@ -157,6 +158,21 @@ tsa_status tsa_block_summarize(const void* K, const int32_t* seq_lens, tsa_shape
     cudaError_t e = tsa::launch_block_summarize(K, seq_lens, d, block, Kmean, flag_of(ws),
                                                 static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "tsa_block_summarize");
+    return TSA_OK;
+}
+
+tsa_status tsa_index_overlap(const int32_t* idx, int32_t n_layers, int32_t units, int32_t k_max,
+                             int32_t* counts, double* M, void* ws, size_t ws_bytes, void* stream) {
+    if (n_layers < 1 || n_layers > 1024)
+        return fail(TSA_ERR_INVALID_ARG, "tsa_index_overlap: n_layers must be in [1, 1024] (got %d)", n_layers);
+    if (units < 0 || k_max < 0)
+        return fail(TSA_ERR_INVALID_ARG, "tsa_index_overlap: units and k_max must be >= 0 (got %d, %d)", units, k_max);
+    if ((!idx && (size_t)units * k_max > 0) || (!counts && !M))
+        return fail(TSA_ERR_INVALID_ARG, "tsa_index_overlap: NULL pointer (idx, or both counts and M)");
+    TSA_TRY(check_ws(ws, ws_bytes, kFlagBytes));
+    cudaError_t e = tsa::launch_index_overlap(idx, n_layers, units, k_max, counts, M, flag_of(ws),
+                                              static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "tsa_index_overlap");
     return TSA_OK;
 }
 
@@ -225,9 +241,59 @@ tsa_status tsa_decode_step(const tsa_step_args* a, void* stream) {
     tsa::Dims d;
     TSA_TRY(check_shape(a->shape, &d));
     switch (a->mode) {
-        case TSA_FULL:
-            return sparse_decode_attn(a->Q, a->K, a->V, a->seq_lens, nullptr, nullptr, 0, 1, a->shape,
-                                      a->scale, a->O, a->ws, a->ws_bytes, stream);
+        case TSA_FULL: {
+            if (!a->idx_out)
+                return sparse_decode_attn(a->Q, a->K, a->V, a->seq_lens, nullptr, nullptr, 0, 1, a->shape,
+                                          a->scale, a->O, a->ws, a->ws_bytes, stream);
+            // A full layer that also hands its top-k on (HyLRA: a sensitive layer's
+            // extracted indices pass to the tolerant layers after it).  Token mode:
+            // the full attention writes each row's score as it forms S (no second
+            // read of K), then the top-k.  Block mode: the block means are scored
+            // as in a SELECT step.
+            TSA_TRY(check_block(a->block));
+            TSA_TRY(check_scale(a->scale));
+            TSA_TRY(check_kmax(a->k_max));
+            if (a->k_max == 0) return fail(TSA_ERR_INVALID_ARG, "tsa_decode_step: a TSA_FULL layer with idx_out needs k_max > 0");
+            if (a->block > 1 && !a->Kmean) return fail(TSA_ERR_INVALID_ARG, "tsa_decode_step: block mode needs Kmean");
+            if (!a->Q || !a->K || !a->V || !a->seq_lens || !a->O) return fail(TSA_ERR_INVALID_ARG, "tsa_decode_step: NULL pointer");
+            if (!aligned16(a->Q) || !aligned16(a->K) || !aligned16(a->V) || !aligned16(a->O) ||
+                (a->block > 1 && !aligned16(a->Kmean)))
+                return fail(TSA_ERR_INVALID_ARG, "tsa_decode_step: Q, K, V, Kmean and O must be 16-byte aligned");
+            int C, chunk;
+            if (!tsa::topk_plan(tsa::rows_cap_of(d, a->block), &C, &chunk))
+                return fail(TSA_ERR_UNSUPPORTED, "tsa_decode_step: %d rows per unit exceed the top-k cluster capacity",
+                            tsa::rows_cap_of(d, a->block));
+            const Layout L = layout(d, a->k_max, a->block, true, true, true);
+            TSA_TRY(check_ws(a->ws, a->ws_bytes, L.total));
+            char* w = static_cast<char*>(a->ws);
+            float* scores = reinterpret_cast<float*>(w + L.scores);
+            uint32_t* hist = reinterpret_cast<uint32_t*>(w + L.hist);
+            float* partials = reinterpret_cast<float*>(w + L.partials);
+            unsigned* counters = reinterpret_cast<unsigned*>(w + L.counters);
+            cudaStream_t st = static_cast<cudaStream_t>(stream);
+            cudaError_t e;
+            if (a->block == 1) {
+                e = tsa::launch_attn(a->Q, a->K, a->V, a->seq_lens, nullptr, nullptr, 0, 1, d, a->scale, L.splits,
+                                     partials, counters, a->O, flag_of(a->ws), st, false, scores);
+                if (e != cudaSuccess) return cuda_fail(e, "tsa_decode_step (full attention)");
+                e = tsa::launch_topk(scores, a->seq_lens, a->k_per_seq, a->k_max, d, 1, a->idx_out, nullptr,
+                                     flag_of(a->ws), st);
+                if (e != cudaSuccess) return cuda_fail(e, "tsa_decode_step (top-k)");
+                return TSA_OK;
+            }
+            e = tsa::launch_score(a->Q, a->Kmean, a->seq_lens, d, a->block, a->scale, scores, hist, flag_of(a->ws), st);
+            if (e != cudaSuccess) return cuda_fail(e, "tsa_decode_step (score)");
+            e = tsa::launch_topk(scores, a->seq_lens, a->k_per_seq, a->k_max, d, a->block, a->idx_out, hist,
+                                 flag_of(a->ws), st);
+            if (e != cudaSuccess) {
+                cudaMemsetAsync(hist, 0, (size_t)d.units() * tsa::kHistBins * sizeof(uint32_t), st);
+                return cuda_fail(e, "tsa_decode_step (top-k)");
+            }
+            e = tsa::launch_attn(a->Q, a->K, a->V, a->seq_lens, nullptr, nullptr, 0, 1, d, a->scale, L.splits,
+                                 partials, counters, a->O, flag_of(a->ws), st);
+            if (e != cudaSuccess) return cuda_fail(e, "tsa_decode_step (full attention)");
+            return TSA_OK;
+        }
         case TSA_REUSE:
             if (!a->idx_in) return fail(TSA_ERR_INVALID_ARG, "tsa_decode_step: TSA_REUSE needs idx_in");
             return sparse_decode_attn(a->Q, a->K, a->V, a->seq_lens, a->idx_in, a->k_per_seq, a->k_max,

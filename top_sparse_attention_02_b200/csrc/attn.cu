@@ -145,7 +145,8 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
             const __nv_bfloat16* __restrict__ V, const int32_t* __restrict__ lens,
             const int32_t* __restrict__ idx, const int32_t* __restrict__ kreq, int k_max,
             int block, int Hkv, int Ncap, float scale_log2, int S, float* __restrict__ part,
-            unsigned* __restrict__ counters, float* __restrict__ O, unsigned* __restrict__ flag, int early) {
+            unsigned* __restrict__ counters, float* __restrict__ O, unsigned* __restrict__ flag, int early,
+            float* __restrict__ sout, float scale) {
     using Cfg = AttnCfg<G>;
     extern __shared__ __align__(128) unsigned char smem_raw[];
     // 1024-byte aligned work area (the swizzled layout needs it)
@@ -359,7 +360,11 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
     const unsigned sbase = smem_u32(smem);
     // The two contractions of flash decoding on this warp's 16 rows of a tile
     // (K at kt, V at vt); bit i of vm: row r0 + i is in the set.
-    auto warp_tile = [&](unsigned kt, unsigned vt, uint32_t vm) {
+    // sout (full attention that also emits its top-k, contiguous tiles only): the
+    // scores of the tile's rows -- scale x the max over the group's heads of q.k,
+    // the criterion a SELECT layer scores by -- written as S is formed
+    float* const su_out = (CONTIG && sout) ? sout + (size_t)unit * Ncap : nullptr;
+    auto warp_tile = [&](unsigned kt, unsigned vt, uint32_t vm, int first) {
         // byte offset of 16-byte chunk c of tile row r (padded rows, or the
         // 128-byte swizzle of the TMA tensor loads: two 64-dim halves)
         auto off = [&](int r, int c) -> unsigned {
@@ -379,6 +384,23 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
                 ldsm_x4(kt + off(row, 2 * ks + (m & 1)), b0, b1, b2, b3);
                 mma_bf16(sc[0], qa[ks][0], qa[ks][1], b0, b1);
                 mma_bf16(sc[1], qa[ks][0], qa[ks][1], b2, b3);
+            }
+        }
+        if constexpr (CONTIG) {
+            if (su_out) {  // uniform: the max over heads g < G of each row's dot, by lanes of equal t4
+                float e[4] = {g < G ? sc[0][0] : -INFINITY, g < G ? sc[0][1] : -INFINITY,
+                              g < G ? sc[1][0] : -INFINITY, g < G ? sc[1][1] : -INFINITY};
+#pragma unroll
+                for (int o = 4; o < 32; o <<= 1)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) e[q] = fmaxf(e[q], __shfl_xor_sync(0xffffffffu, e[q], o));
+                if (g == 0) {
+                    const int ia = 2 * t4;
+                    const int lrow[4] = {ia, ia + 1, ia + 8, ia + 9};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)  // scale > 0: scale x max = max of the scaled logits
+                        if ((vm >> lrow[q]) & 1u) su_out[first + r0 + lrow[q]] = e[q] * scale;
+                }
             }
         }
         // ---- online softmax for head g (columns = rows of the tile)
@@ -457,7 +479,7 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
             const uint32_t vm = nv >= 16 ? 0xffffu : (nv > 0 ? (1u << nv) - 1u : 0u);
             if (vm) {  // warp-uniform
                 const unsigned kt = sbase + st * kStageBytes;
-                warp_tile(kt, kt + 2 * 64 * kTileRows * 2, vm);
+                warp_tile(kt, kt + 2 * 64 * kTileRows * 2, vm, first);
             }
             __syncthreads();  // every warp is done with this stage
             if (tid == 0) stage_contig(t + STAGES, next_first);  // refill it (nothing past the end)
@@ -467,7 +489,7 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
             if (t > 0) issue_one(t);
             asm volatile("cp.async.wait_all;\n" ::: "memory");
             __syncwarp();
-            if (vm_one) warp_tile(sbase, sbase + kTileRows * kRowStride, vm_one);
+            if (vm_one) warp_tile(sbase, sbase + kTileRows * kRowStride, vm_one, 0);
             __syncwarp();  // the math has read these rows before the next copies land
         }
     } else {
@@ -480,7 +502,7 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
             const uint32_t vm = vm_next;
             __syncwarp();
             if (t + 1 < ntiles) fetch(t + 1);  // the next tile's loads fly during this tile's math
-            if (vm) warp_tile(sbase, sbase + kTileRows * kRowStride, vm);
+            if (vm) warp_tile(sbase, sbase + kTileRows * kRowStride, vm, 0);
             __syncwarp();  // the math has read these rows before the next store
         }
     }
@@ -742,6 +764,8 @@ struct AttnArgs {
     float* O;
     unsigned* flag;
     int early;
+    float* sout;
+    float scale;
 };
 
 template <int G, int STAGES, bool CLUSTER, bool CONTIG, bool ONE = false>
@@ -761,7 +785,7 @@ static cudaError_t attn_launch_g(dim3 grid, cudaStream_t st, const AttnArgs& a) 
     cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, attn_kernel<G, STAGES, CLUSTER, CONTIG, ONE>, a.kmap, a.vmap, a.q, a.k, a.v, a.lens,
                               a.idx, a.kreq, a.k_max, a.block, a.Hkv, a.Ncap, a.sl2, a.splits, a.partials, a.counters,
-                              a.O, a.flag, a.early);
+                              a.O, a.flag, a.early, a.sout, a.scale);
 }
 
 template <int G, int STAGES, bool CLUSTER, bool CONTIG, bool ONE = false>
@@ -833,8 +857,10 @@ static cudaError_t make_row_map(CUtensorMap* map, const void* base, const Dims& 
 cudaError_t launch_attn(const void* Q, const void* K, const void* V, const int32_t* lens,
                         const int32_t* idx, const int32_t* kreq, int k_max, int block,
                         const Dims& d, float scale, int splits, float* partials,
-                        unsigned* counters, float* O, unsigned* flag, cudaStream_t st, bool early) {
+                        unsigned* counters, float* O, unsigned* flag, cudaStream_t st, bool early,
+                        float* scores_out) {
     if (d.units() == 0) return cudaSuccess;
+    if (scores_out && idx != nullptr) return cudaErrorInvalidValue;  // scores come with full attention only
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -885,6 +911,8 @@ cudaError_t launch_attn(const void* Q, const void* K, const void* V, const int32
     a.O = O;
     a.flag = flag;
     a.early = early ? 1 : 0;
+    a.sout = scores_out;
+    a.scale = scale;
     dim3 grid(splits, d.units());
     switch (d.G) {
         case 1: e = attn_dispatch<1>(contig, one_tile, cluster, grid, st, a); break;

@@ -32,6 +32,12 @@ inline cudaLaunchAttribute pdl_attr() {
 // set the text tsa_last_error_string() returns on this thread
 void set_error_message(const char* msg);
 
+// |I_i(u) ∩ I_j(u)| of L layers' index lists [L][units][k_max] into counts
+// [L][L][units] (may be NULL) and the mean target-normalised ratio into M [L][L]
+// (lower triangle, row = target; may be NULL)
+cudaError_t launch_index_overlap(const int32_t* idx, int L, int units, int k_max, int32_t* counts, double* M,
+                                 unsigned* flag, cudaStream_t st);
+
 cudaError_t launch_block_summarize(const void* K, const int32_t* lens, const Dims& d, int block,
                                    float* Kmean, unsigned* flag, cudaStream_t st);
 
@@ -76,7 +82,8 @@ cudaError_t launch_attn(const void* Q, const void* K, const void* V, const int32
                         const int32_t* idx, const int32_t* kreq, int k_max, int block,
                         const Dims& d, float scale, int splits, float* partials,
                         unsigned* counters, float* O, unsigned* flag, cudaStream_t st,
-                        bool early = false);  // early: lens, k's and Q not written by the previous kernel
+                        bool early = false,  // early: lens, k's and Q not written by the previous kernel
+                        float* scores_out = nullptr);  // full attention only: [units][Ncap] scores of the valid rows
 
 cudaError_t launch_copy(const void* src, void* dst, size_t bytes, cudaStream_t st);
 cudaError_t launch_gather(const void* base, size_t base_bytes, const int32_t* rows, int nrows, unsigned* flag,

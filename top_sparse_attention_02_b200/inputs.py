@@ -117,3 +117,27 @@ def drift_query(Q: torch.Tensor, sigma: float, seed: int) -> torch.Tensor:
     g = _gen(seed, Q.device)
     noise = torch.randn(Q.shape, generator=g, device=Q.device)
     return (Q.float() + sigma * noise).to(torch.bfloat16)
+
+
+def layer_index_lists(L: int, n_rows, k_rows, k_max: int, keep: float, seed: int) -> torch.Tensor:
+    """L layers' index lists for len(n_rows) units: int32 [L, units, k_max], each
+    list ascending then -1, as a decode step writes them.  Unit u draws
+    min(k_rows[u], n_rows[u]) distinct rows of [0, n_rows[u]) uniformly for layer 0;
+    each later layer keeps every row of the layer before with probability `keep`
+    and fills up with rows the layer before did not hold, drawn uniformly (then,
+    if those run out, with the rows it dropped) (CPU generator)."""
+    g = _gen(seed, "cpu")
+    units = len(n_rows)
+    out = torch.full((L, units, k_max), -1, dtype=torch.int32)
+    for u in range(units):
+        n, k = int(n_rows[u]), min(int(k_rows[u]), int(n_rows[u]))
+        cur = torch.randperm(n, generator=g)[:k]
+        for l in range(L):
+            if l > 0:
+                take = torch.rand(k, generator=g) < keep
+                kept, dropped = cur[take], cur[~take]
+                pool = torch.randperm(n, generator=g)
+                pool = torch.cat([pool[~torch.isin(pool, cur)], dropped])
+                cur = torch.cat([kept, pool[:k - kept.numel()]])
+            out[l, u, :k] = torch.sort(cur).values.to(torch.int32)
+    return out
