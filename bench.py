@@ -374,6 +374,18 @@ def stage_times(tsa, w, plan, layers, Kmean, ws, kreq_t, idx, O, stream, reps=10
         else:
             calls[f"L{li}_attn"] = lambda L=L, li=li: tsa.sparse_decode_attn(
                 L.Q, L.K, L.V, L.seq_lens, None, None, 0, 1, w.scale, O[li], ws, stream)
+            if li == w.route.index(tsa.FULL):
+                # the first full layer once more, handing on its top-k (what a
+                # sensitive layer does before reuse layers): the cost of the hand-off
+                km = None
+                if w.block > 1:
+                    km = torch.zeros(w.B, w.Hkv, NB, w.d, dtype=torch.float32, device=L.Q.device)
+                    tsa.block_summarize(L.K, L.seq_lens, w.block, km, ws, shape=shape)
+                idx_emit = torch.full_like(idx[li], -1)
+                fa = tsa.step_args(L.Q, L.K, L.V, L.seq_lens, O[li], ws, mode=tsa.FULL, scale=w.scale,
+                                   k_max=plan.k_max, block=w.block, k_per_seq=kreq_t, Kmean=km,
+                                   idx_out=idx_emit)
+                calls[f"L{li}_full_emit_step"] = lambda fa=fa, km=km, ie=idx_emit: tsa.decode_step(fa, stream)
     flush = L2Flush(layers[0].Q.device)
     flush_us = graph_us(flush, stream, reps)
     warm, cold = {}, {}
