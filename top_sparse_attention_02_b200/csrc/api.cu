@@ -74,8 +74,8 @@ size_t a256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 constexpr size_t kFlagBytes = 256;
 
-// Workspace: [flag 256 B][split counters][split partials][scores, top-digit
-// histograms (SELECT only)]
+// Workspace: [flag 256 B][top-digit histograms][split counters][split partials]
+// [scores (SELECT, and FULL handing on its top-k)]
 struct Layout {
     size_t counters = 0, partials = 0, scores = 0, hist = 0, total = kFlagBytes;
     int splits = 0;
@@ -84,6 +84,12 @@ struct Layout {
 Layout layout(const tsa::Dims& d, int k_max, int block, bool attn, bool dense, bool scores) {
     Layout L;
     size_t off = kFlagBytes;
+    // The top-digit histograms must be zero when a decode step starts (its top-k
+    // returns them to zero).  They sit at the same offset, right after the flag,
+    // in every layout, so steps of any mode that share a workspace never write
+    // over them with their split partials or scores.
+    L.hist = off;
+    off += a256((size_t)d.units() * tsa::kHistBins * sizeof(uint32_t));
     if (attn) {
         L.splits = tsa::attn_splits(d, k_max, block, dense);
         L.counters = off;
@@ -94,8 +100,6 @@ Layout layout(const tsa::Dims& d, int k_max, int block, bool attn, bool dense, b
     if (scores) {
         L.scores = off;
         off += a256((size_t)d.units() * tsa::rows_cap_of(d, block) * sizeof(float));
-        L.hist = off;
-        off += a256((size_t)d.units() * tsa::kHistBins * sizeof(uint32_t));
     }
     L.total = off;
     return L;
