@@ -302,6 +302,8 @@ def run_ours(args, rank, world, dev):
     }
     if not args.no_e2e:
         res["e2e"] = e2e_measure(tsa, w, plan, layers, step_args, O, idx, stream, args)
+    if args.offload:
+        res["offload"] = offload_probe(tsa, w, plan, layers, Kmean, ws, kreq_t, idx, O, stream)
     return res
 
 
@@ -398,6 +400,75 @@ def stage_times(tsa, w, plan, layers, Kmean, ws, kreq_t, idx, O, stream, reps=10
             "score_us": statistics.mean(warm[f"L{li}_score"] for li in sel) if sel else float("nan"),
             "note": f"per launch, {reps} launches per CUDA graph; warm = back to back, cold = after an L2 "
                     "flush (minus the flush alone)"}
+
+
+def offload_probe(tsa, w, plan, layers, Kmean, ws, kreq_t, idx, O, stream, reps=5):
+    """Index-guided offload: the first SELECT layer of a block-mode stack, and a
+    REUSE step over its blocks, with that layer's K and V in page-locked host
+    memory (the block means stay on the device).  Only the selected blocks cross
+    the host link.  Timed with CUDA events around single launches, each after an
+    L2 flush (the pointer check that the offload path makes on the host is kept
+    out of graph capture), against a 1 GiB pinned host-to-device copy."""
+    assert w.block > 1, "the offload probe needs a block-mode workload"
+    li = w.route.index(tsa.SELECT)
+    L = layers[li]
+    dev = L.Q.device
+    Kh = torch.empty(L.K.shape, dtype=L.K.dtype, pin_memory=True)
+    Vh = torch.empty(L.V.shape, dtype=L.V.dtype, pin_memory=True)
+    Kh.copy_(L.K)
+    Vh.copy_(L.V)
+    flush = L2Flush(dev)
+
+    def timed(fn):
+        ts = []
+        for _ in range(reps + 1):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                flush()
+                e0.record(stream)
+                fn()
+                e1.record(stream)
+            stream.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e3)
+        return statistics.median(ts[1:])
+
+    sel = tsa.step_args(L.Q, Kh, Vh, L.seq_lens, O[li], ws, mode=tsa.SELECT, scale=w.scale, k_max=plan.k_max,
+                        block=w.block, k_per_seq=kreq_t, Kmean=Kmean[li], idx_out=idx[li], flags=tsa.KV_HOST)
+    reu = tsa.step_args(L.Q, Kh, Vh, L.seq_lens, O[li], ws, mode=tsa.REUSE, scale=w.scale, k_max=plan.k_max,
+                        block=w.block, k_per_seq=kreq_t, idx_in=idx[li], flags=tsa.KV_HOST)
+    select_us = timed(lambda: tsa.decode_step(sel, stream))
+    reuse_us = timed(lambda: tsa.decode_step(reu, stream))
+    tsa.check_device_status(ws, stream)
+    # rows the attention fetches: every valid row of each selected block, K and V
+    lens = [int(x) for x in L.seq_lens.cpu()]
+    ix = idx[li].cpu().numpy()
+    rows = 0
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            for e in ix[b, h]:
+                if e >= 0:
+                    rows += max(0, min(w.block, lens[b] - int(e) * w.block))
+    fetched = rows * 2 * w.d * 2
+    src = torch.empty(1 << 30, dtype=torch.uint8, pin_memory=True)
+    dst = torch.empty(1 << 30, dtype=torch.uint8, device=dev)
+    h2d = []
+    for _ in range(4):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            dst.copy_(src, non_blocking=True)
+            e1.record(stream)
+        stream.synchronize()
+        h2d.append(src.numel() / (e0.elapsed_time(e1) * 1e-3) / 1e9)
+    h2d_gbs = max(h2d[1:])
+    del Kh, Vh, src, dst, flush
+    achieved = fetched / (reuse_us * 1e-6) / 1e9
+    whole = (L.K.numel() + L.V.numel()) * 2
+    return {"layer": li, "select_step_us": select_us, "reuse_step_us": reuse_us, "fetched_bytes": fetched,
+            "reuse_achieved_gbs": achieved, "h2d_copy_gbs": h2d_gbs, "frac_of_h2d_copy": achieved / h2d_gbs,
+            "whole_layer_kv_bytes": whole, "whole_layer_copy_us": whole / (h2d_gbs * 1e9) * 1e6,
+            "note": "K and V of one layer in pinned host memory; attention reads only the selected "
+                    "128-token blocks across the host link; cold L2, median of %d single launches" % reps}
 
 
 def copy_probe(tsa, dev, stream, nbytes=2 << 30):
@@ -629,6 +700,8 @@ def main():
     ap.add_argument("--workload", default="reuse128k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--offload", action="store_true",
+                    help="block-mode workloads: also time a layer whose K/V sit in pinned host memory")
     ap.add_argument("--ncap", type=int, default=0,
                     help="shrink the workload's context to this many tokens (profiler captures only)")
     args = ap.parse_args()

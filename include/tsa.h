@@ -178,7 +178,21 @@ typedef struct {
     float* O;                 /* [B, Hq, d] fp32 */
     void* ws;                 /* workspace */
     size_t ws_bytes;
+    uint32_t flags;           /* 0, or TSA_KV_HOST */
 } tsa_step_args;
+
+/* tsa_step_args.flags: K and V live in page-locked host memory that the device
+ * reads at the same address (cudaHostAlloc; or cudaHostRegister'd and mapped):
+ * a cache larger than HBM, offloaded.  The attention then fetches only the
+ * selected rows (or 128-token blocks) across the host link, with plain loads
+ * through the device's mapping of the pages (index-guided offload, HyLRA sec.
+ * 2.4: the block indices say which blocks to bring in).  Layers that select must
+ * score block means (block > 1, Kmean in device memory), since token-mode
+ * scoring reads every K row; TSA_SELECT or a TSA_FULL layer with idx_out in
+ * token mode returns TSA_ERR_UNSUPPORTED.  TSA_REUSE works in either mode; a
+ * TSA_FULL layer reads all of K and V across the link.  A K or V pointer that is
+ * not such memory returns TSA_ERR_INVALID_ARG (pageable memory would fault). */
+#define TSA_KV_HOST 1u
 
 /* One decode step of one layer: TSA_SELECT = score -> top-k -> attention;
  * TSA_REUSE = attention over idx_in; TSA_FULL = attention over every valid row.

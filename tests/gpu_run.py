@@ -25,7 +25,7 @@ def block_means(K, lens, block):
 
 
 def step(Q, K, V, lens, *, mode, scale, k_max=0, block=1, kreq=None, Kmean=None, idx_in=None,
-         ws=None, check=True, emit=False):
+         ws=None, check=True, emit=False, flags=0):
     """One decode step; returns (O, idx) with idx None unless SELECT (or FULL with emit)."""
     B, Hq, d = Q.shape
     Hkv = K.shape[1]
@@ -37,7 +37,7 @@ def step(Q, K, V, lens, *, mode, scale, k_max=0, block=1, kreq=None, Kmean=None,
         idx = torch.full((B, Hkv, k_max), -7, dtype=torch.int32, device=Q.device)
     kr = None if kreq is None else torch.as_tensor(kreq, dtype=torch.int32).to(Q.device)
     a = tsa.step_args(Q, K, V, lens, O, ws, mode=mode, scale=scale, k_max=k_max, block=block,
-                      k_per_seq=kr, Kmean=Kmean, idx_in=idx_in, idx_out=idx)
+                      k_per_seq=kr, Kmean=Kmean, idx_in=idx_in, idx_out=idx, flags=flags)
     tsa.decode_step(a)
     if check:
         tsa.check_device_status(ws)

@@ -152,6 +152,14 @@ def test_decode_step_argument_errors(tsa):
     a = tsa.step_args(Q, K, T(0x3000), T(0x4000), T(0x5000), ws, mode=tsa.FULL, scale=0.1, k_max=16,
                       block=128, idx_out=T(0x7000))
     assert tsa.lib().tsa_decode_step(ctypes.byref(a), None) == 1 and "Kmean" in tsa.last_error()
+    a = tsa.step_args(Q, K, T(0x3000), T(0x4000), T(0x5000), ws, mode=tsa.REUSE, scale=0.1, k_max=16,
+                      idx_in=T(0x7000), flags=6)
+    assert tsa.lib().tsa_decode_step(ctypes.byref(a), None) == 1 and "flags" in tsa.last_error()
+    # an offloaded cache: a layer that selects must score block means
+    for mode, idx_out in ((tsa.SELECT, T(0x7000)), (tsa.FULL, T(0x7000))):
+        a = tsa.step_args(Q, K, T(0x3000), T(0x4000), T(0x5000), ws, mode=mode, scale=0.1, k_max=16,
+                          idx_out=idx_out, flags=tsa.KV_HOST)
+        assert tsa.lib().tsa_decode_step(ctypes.byref(a), None) == 2 and "block means" in tsa.last_error()
     a = tsa.step_args(Q, K, T(0x3000), T(0x4000), T(0x5000), ws, mode=9, scale=0.1, k_max=16)
     assert tsa.lib().tsa_decode_step(ctypes.byref(a), None) == 1 and "mode" in tsa.last_error()
     assert tsa.lib().tsa_decode_step(None, None) == 1

@@ -555,3 +555,79 @@ def test_index_overlap_of_decode_steps(cuda_dev):
         compare_idx(idx[l].cpu().numpy(), S, lens, kreq)
     counts, M = _check_overlap(idx)
     assert 0.0 < M[1, 0] < 1.0
+
+
+# ------------------------------------------------------------------ index-guided offload (HyLRA sec. 2.4)
+
+def _pinned(t):
+    out = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+    out.copy_(t)
+    return out
+
+
+def test_offloaded_cache_block_select_and_reuse(cuda_dev):
+    """K and V in page-locked host memory, block means on the device: the SELECT
+    step picks the same blocks as with the cache in HBM (same scorer, same
+    top-k) and its attention, which fetches only those blocks across the host
+    link, matches the oracle; then REUSE steps over those blocks, in block and
+    in token mode, read from the host copy too."""
+    L = layer(2, 32, 8, 5000, [5000, 2100], seed=111, plant=0.01, tail_fill=float("nan"))
+    kreq, k_max, block = [12, 7], 12, 128
+    Q, K, V, ln = G.to_dev(L, cuda_dev)
+    Kh, Vh = _pinned(L.K), _pinned(L.V)
+    Kmean = G.block_means(K, ln, block)
+    O_dev, idx_dev = G.step(Q, K, V, ln, mode=tsa.SELECT, scale=SCALE, k_max=k_max, block=block, kreq=kreq,
+                            Kmean=Kmean)
+    O_h, idx_h = G.step(Q, Kh, Vh, ln, mode=tsa.SELECT, scale=SCALE, k_max=k_max, block=block, kreq=kreq,
+                        Kmean=Kmean, flags=tsa.KV_HOST)
+    assert torch.equal(idx_h, idx_dev)
+    ref = oracle.attn(L.Q, L.K, L.V, L.seq_lens, idx_h.cpu().numpy(), kreq, k_max, block, SCALE)
+    check_output(O_h.cpu().numpy(), ref, "offloaded block select")
+    O_r, _ = G.step(Q, Kh, Vh, ln, mode=tsa.REUSE, scale=SCALE, k_max=k_max, block=block, kreq=kreq,
+                    idx_in=idx_h, flags=tsa.KV_HOST)
+    check_output(O_r.cpu().numpy(), ref, "offloaded block reuse")
+    # token mode reuse over a set of rows
+    rows = np.full((2, 8, 200), -1, dtype=np.int32)
+    rng = np.random.default_rng(5)
+    for b, n in enumerate([5000, 2100]):
+        for h in range(8):
+            rows[b, h] = np.sort(rng.choice(n, 200, replace=False))
+    O_t, _ = G.step(Q, Kh, Vh, ln, mode=tsa.REUSE, scale=SCALE, k_max=200, kreq=[200, 200],
+                    idx_in=torch.from_numpy(rows).to(cuda_dev), flags=tsa.KV_HOST)
+    ref_t = oracle.attn(L.Q, L.K, L.V, L.seq_lens, rows, [200, 200], 200, 1, SCALE)
+    check_output(O_t.cpu().numpy(), ref_t, "offloaded token reuse")
+
+
+def test_offloaded_cache_full_layers(cuda_dev):
+    """A full layer over an offloaded cache reads every row across the link; in
+    block mode it can still hand on its top-k (the means are on the device)."""
+    L = layer(2, 16, 4, 3000, [3000, 1234], seed=112, tail_fill=float("nan"))
+    kreq, k_max, block = [8, 5], 8, 128
+    Q, K, V, ln = G.to_dev(L, cuda_dev)
+    Kh, Vh = _pinned(L.K), _pinned(L.V)
+    ref = oracle.attn(L.Q, L.K, L.V, L.seq_lens, None, None, 0, 1, SCALE)
+    O, _ = G.step(Q, Kh, Vh, ln, mode=tsa.FULL, scale=SCALE, flags=tsa.KV_HOST)
+    check_output(O.cpu().numpy(), ref, "offloaded full layer")
+    Kmean = G.block_means(K, ln, block)
+    ws = G.ws_for(Q, K, k_max, block, tsa.FULL)
+    O2, idx = G.step(Q, Kh, Vh, ln, mode=tsa.FULL, scale=SCALE, k_max=k_max, block=block, kreq=kreq,
+                     Kmean=Kmean, ws=ws, emit=True, flags=tsa.KV_HOST)
+    check_output(O2.cpu().numpy(), ref, "offloaded full layer handing on its blocks")
+    nrows = oracle.nblocks_of(L.seq_lens, block)
+    S = oracle.block_scores(L.Q, oracle.block_means(L.K, L.seq_lens, block), nrows, SCALE)
+    compare_idx(idx.cpu().numpy(), S, nrows, kreq)
+
+
+def test_offload_refuses_memory_the_device_cannot_read(cuda_dev):
+    """Pageable host memory is refused before anything is launched, and token-mode
+    selection over an offloaded cache is unsupported."""
+    L = layer(1, 8, 2, 512, seed=113)
+    Q, K, V, ln = G.to_dev(L, cuda_dev)
+    idx = torch.zeros(1, 2, 4, dtype=torch.int32, device=cuda_dev)
+    with pytest.raises(tsa.TsaError, match="page-locked"):
+        G.step(Q, L.K, L.V, ln, mode=tsa.REUSE, scale=SCALE, k_max=4, idx_in=idx, flags=tsa.KV_HOST)
+    with pytest.raises(tsa.TsaError, match="page-locked"):  # device memory is not host memory either
+        G.step(Q, K, V, ln, mode=tsa.REUSE, scale=SCALE, k_max=4, idx_in=idx, flags=tsa.KV_HOST)
+    with pytest.raises(tsa.TsaError, match="UNSUPPORTED"):
+        G.step(Q, _pinned(L.K), _pinned(L.V), ln, mode=tsa.SELECT, scale=SCALE, k_max=4,
+               flags=tsa.KV_HOST)

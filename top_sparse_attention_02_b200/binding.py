@@ -37,7 +37,10 @@ class tsa_step_args(ctypes.Structure):
                 ("k_per_seq", ctypes.c_void_p), ("k_max", ctypes.c_int32), ("block", ctypes.c_int32),
                 ("mode", ctypes.c_int32), ("scale", ctypes.c_float), ("idx_in", ctypes.c_void_p),
                 ("idx_out", ctypes.c_void_p), ("O", ctypes.c_void_p), ("ws", ctypes.c_void_p),
-                ("ws_bytes", ctypes.c_size_t)]
+                ("ws_bytes", ctypes.c_size_t), ("flags", ctypes.c_uint32)]
+
+
+KV_HOST = 1  # tsa_step_args.flags: K and V in mapped page-locked host memory
 
 
 _vp, _sz, _i32, _f32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_float
@@ -166,7 +169,7 @@ def sparse_decode_attn_noalloc(Q, K, V, seq_lens, idx, k_per_seq, k_max: int, bl
 
 
 def step_args(Q, K, V, seq_lens, O, ws, *, mode: int, scale: float, k_max: int = 0, block: int = 1,
-              k_per_seq=None, Kmean=None, idx_in=None, idx_out=None) -> tsa_step_args:
+              k_per_seq=None, Kmean=None, idx_in=None, idx_out=None, flags: int = 0) -> tsa_step_args:
     a = tsa_step_args()
     a.shape = shape_of(Q, K)
     a.Q, a.K, a.V, a.Kmean = _ptr(Q), _ptr(K), _ptr(V), _ptr(Kmean)
@@ -174,6 +177,7 @@ def step_args(Q, K, V, seq_lens, O, ws, *, mode: int, scale: float, k_max: int =
     a.k_max, a.block, a.mode, a.scale = k_max, block, mode, scale
     a.idx_in, a.idx_out, a.O = _ptr(idx_in), _ptr(idx_out), _ptr(O)
     a.ws, a.ws_bytes = _wsargs(ws)
+    a.flags = flags
     return a
 
 

@@ -214,11 +214,48 @@ tsa_status topk_select(const float* scores, const int32_t* seq_lens, const int32
     return TSA_OK;
 }
 
+namespace {
+
+// K and V of an offloaded cache: page-locked host memory that the device reads
+// at the same address (cudaHostAlloc, or cudaHostRegister'd and mapped).  Any
+// other host pointer (pageable memory) would fault the kernel, so it is refused.
+tsa_status check_host_kv(const void* K, const void* V) {
+    const void* ptrs[2] = {K, V};
+    for (const void* p : ptrs) {
+        cudaPointerAttributes at;
+        cudaError_t e = cudaPointerGetAttributes(&at, p);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            return cuda_fail(e, "tsa_decode_step (K/V pointer query)");
+        }
+        if (at.type != cudaMemoryTypeHost || at.devicePointer != p)
+            return fail(TSA_ERR_INVALID_ARG,
+                        "tsa_decode_step: with TSA_KV_HOST, K and V must be page-locked host memory mapped for "
+                        "the device at the same address (cudaHostAlloc, or cudaHostRegister with mapping)");
+    }
+    return TSA_OK;
+}
+
+tsa_status attn_stage(const void* Q, const void* K, const void* V, const int32_t* seq_lens, const int32_t* idx,
+                      const int32_t* k_per_seq, int32_t k_max, int32_t block, tsa_shape shape, float scale, float* O,
+                      void* ws, size_t ws_bytes, void* stream, bool host_kv);
+
+}  // namespace
+
 tsa_status sparse_decode_attn(const void* Q, const void* K, const void* V,
                               const int32_t* seq_lens, const int32_t* idx,
                               const int32_t* k_per_seq, int32_t k_max, int32_t block,
                               tsa_shape shape, float scale, float* O, void* ws, size_t ws_bytes,
                               void* stream) {
+    return attn_stage(Q, K, V, seq_lens, idx, k_per_seq, k_max, block, shape, scale, O, ws, ws_bytes, stream,
+                      false);
+}
+
+namespace {
+
+tsa_status attn_stage(const void* Q, const void* K, const void* V, const int32_t* seq_lens, const int32_t* idx,
+                      const int32_t* k_per_seq, int32_t k_max, int32_t block, tsa_shape shape, float scale, float* O,
+                      void* ws, size_t ws_bytes, void* stream, bool host_kv) {
     tsa::Dims d;
     TSA_TRY(check_shape(shape, &d));
     TSA_TRY(check_block(block));
@@ -232,23 +269,33 @@ tsa_status sparse_decode_attn(const void* Q, const void* K, const void* V,
     const Layout L = layout(d, dense ? 0 : k_max, dense ? 1 : block, true, dense, false);
     TSA_TRY(check_ws(ws, ws_bytes, L.total));
     char* w = static_cast<char*>(ws);
+    if (host_kv) TSA_TRY(check_host_kv(K, V));
     cudaError_t e = tsa::launch_attn(Q, K, V, seq_lens, idx, k_per_seq, k_max, dense ? 1 : block, d,
                                      scale, L.splits, reinterpret_cast<float*>(w + L.partials),
                                      reinterpret_cast<unsigned*>(w + L.counters), O, flag_of(ws),
-                                     static_cast<cudaStream_t>(stream));
+                                     static_cast<cudaStream_t>(stream), false, nullptr, host_kv);
     if (e != cudaSuccess) return cuda_fail(e, "sparse_decode_attn");
     return TSA_OK;
 }
+
+}  // namespace
 
 tsa_status tsa_decode_step(const tsa_step_args* a, void* stream) {
     if (!a) return fail(TSA_ERR_INVALID_ARG, "tsa_decode_step: NULL args");
     tsa::Dims d;
     TSA_TRY(check_shape(a->shape, &d));
+    if (a->flags & ~(uint32_t)TSA_KV_HOST)
+        return fail(TSA_ERR_INVALID_ARG, "tsa_decode_step: unknown flags 0x%x", a->flags);
+    const bool host_kv = (a->flags & TSA_KV_HOST) != 0;
+    if (host_kv && a->block == 1 && (a->mode == TSA_SELECT || (a->mode == TSA_FULL && a->idx_out)))
+        return fail(TSA_ERR_UNSUPPORTED,
+                    "tsa_decode_step: with TSA_KV_HOST a layer that selects must score block means (block > 1); "
+                    "token-mode scoring streams all of K");
     switch (a->mode) {
         case TSA_FULL: {
             if (!a->idx_out)
-                return sparse_decode_attn(a->Q, a->K, a->V, a->seq_lens, nullptr, nullptr, 0, 1, a->shape,
-                                          a->scale, a->O, a->ws, a->ws_bytes, stream);
+                return attn_stage(a->Q, a->K, a->V, a->seq_lens, nullptr, nullptr, 0, 1, a->shape, a->scale, a->O,
+                                  a->ws, a->ws_bytes, stream, host_kv);
             // A full layer that also hands its top-k on (HyLRA: a sensitive layer's
             // extracted indices pass to the tolerant layers after it).  Token mode:
             // the full attention writes each row's score as it forms S (no second
@@ -269,6 +316,7 @@ tsa_status tsa_decode_step(const tsa_step_args* a, void* stream) {
                             tsa::rows_cap_of(d, a->block));
             const Layout L = layout(d, a->k_max, a->block, true, true, true);
             TSA_TRY(check_ws(a->ws, a->ws_bytes, L.total));
+            if (host_kv) TSA_TRY(check_host_kv(a->K, a->V));
             char* w = static_cast<char*>(a->ws);
             float* scores = reinterpret_cast<float*>(w + L.scores);
             uint32_t* hist = reinterpret_cast<uint32_t*>(w + L.hist);
@@ -294,14 +342,14 @@ tsa_status tsa_decode_step(const tsa_step_args* a, void* stream) {
                 return cuda_fail(e, "tsa_decode_step (top-k)");
             }
             e = tsa::launch_attn(a->Q, a->K, a->V, a->seq_lens, nullptr, nullptr, 0, 1, d, a->scale, L.splits,
-                                 partials, counters, a->O, flag_of(a->ws), st);
+                                 partials, counters, a->O, flag_of(a->ws), st, false, nullptr, host_kv);
             if (e != cudaSuccess) return cuda_fail(e, "tsa_decode_step (full attention)");
             return TSA_OK;
         }
         case TSA_REUSE:
             if (!a->idx_in) return fail(TSA_ERR_INVALID_ARG, "tsa_decode_step: TSA_REUSE needs idx_in");
-            return sparse_decode_attn(a->Q, a->K, a->V, a->seq_lens, a->idx_in, a->k_per_seq, a->k_max,
-                                      a->block, a->shape, a->scale, a->O, a->ws, a->ws_bytes, stream);
+            return attn_stage(a->Q, a->K, a->V, a->seq_lens, a->idx_in, a->k_per_seq, a->k_max, a->block, a->shape,
+                              a->scale, a->O, a->ws, a->ws_bytes, stream, host_kv);
         case TSA_SELECT: {
             TSA_TRY(check_block(a->block));
             TSA_TRY(check_scale(a->scale));
@@ -319,6 +367,7 @@ tsa_status tsa_decode_step(const tsa_step_args* a, void* stream) {
                             tsa::rows_cap_of(d, a->block));
             const Layout L = layout(d, a->k_max, a->block, true, false, true);
             TSA_TRY(check_ws(a->ws, a->ws_bytes, L.total));
+            if (host_kv) TSA_TRY(check_host_kv(a->K, a->V));
             char* w = static_cast<char*>(a->ws);
             float* scores = reinterpret_cast<float*>(w + L.scores);
             // the scorer also histograms the top digit of its keys; the top-k
@@ -340,7 +389,8 @@ tsa_status tsa_decode_step(const tsa_step_args* a, void* stream) {
             // indices: it may read the lengths, k's and Q before waiting on it
             e = tsa::launch_attn(a->Q, a->K, a->V, a->seq_lens, a->idx_out, a->k_per_seq, a->k_max, a->block, d,
                                  a->scale, L.splits, reinterpret_cast<float*>(w + L.partials),
-                                 reinterpret_cast<unsigned*>(w + L.counters), a->O, flag_of(a->ws), st, true);
+                                 reinterpret_cast<unsigned*>(w + L.counters), a->O, flag_of(a->ws), st, true,
+                                 nullptr, host_kv);
             if (e != cudaSuccess) return cuda_fail(e, "tsa_decode_step (attention)");
             return TSA_OK;
         }

@@ -858,9 +858,10 @@ cudaError_t launch_attn(const void* Q, const void* K, const void* V, const int32
                         const int32_t* idx, const int32_t* kreq, int k_max, int block,
                         const Dims& d, float scale, int splits, float* partials,
                         unsigned* counters, float* O, unsigned* flag, cudaStream_t st, bool early,
-                        float* scores_out) {
+                        float* scores_out, bool host_kv) {
     if (d.units() == 0) return cudaSuccess;
-    if (scores_out && idx != nullptr) return cudaErrorInvalidValue;  // scores come with full attention only
+    // scores come with full attention on the tensor-map path only
+    if (scores_out && (idx != nullptr || host_kv)) return cudaErrorInvalidValue;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -879,13 +880,16 @@ cudaError_t launch_attn(const void* Q, const void* K, const void* V, const int32
         const long long nbmax = block == 1 ? d.Ncap : ceil_div(d.Ncap, block);
         rows = (long long)(k_max < nbmax ? k_max : nbmax) * block;
     }
-    // whole 128-row tiles of consecutive cache rows: full attention, or 128-token blocks
-    const bool contig = idx == nullptr || block == kTileRows;
+    // whole 128-row tiles of consecutive cache rows: full attention, or 128-token
+    // blocks.  K and V in host memory (index-guided offload) always take the
+    // gather, which fetches only the rows in the set, with plain vector loads
+    // through the device's mapping of the host pages (no tensor map over them).
+    const bool contig = !host_kv && (idx == nullptr || block == kTileRows);
     const long long per_split = contig ? ((rows + splits - 1) / splits + kTileRows - 1) / kTileRows * kTileRows
                                        : (rows + splits - 1) / splits;
     // one tile a CTA: the single-stage kernel (contiguous tiles), or the gather's
-    // two-CTAs-an-SM instance
-    const bool one_tile = per_split <= kTileRows;
+    // two-CTAs-an-SM instance (its cp.async copies are kept to device memory)
+    const bool one_tile = per_split <= kTileRows && !host_kv;
     const bool cluster = attn_cluster_fits(d.G, one_tile, contig, splits, d.units());
     AttnArgs a;
     memset(&a.kmap, 0, sizeof a.kmap);

@@ -83,7 +83,8 @@ cudaError_t launch_attn(const void* Q, const void* K, const void* V, const int32
                         const Dims& d, float scale, int splits, float* partials,
                         unsigned* counters, float* O, unsigned* flag, cudaStream_t st,
                         bool early = false,  // early: lens, k's and Q not written by the previous kernel
-                        float* scores_out = nullptr);  // full attention only: [units][Ncap] scores of the valid rows
+                        float* scores_out = nullptr,  // full attention: each row's group-max scaled score
+                        bool host_kv = false);        // K, V in mapped page-locked host memory: gather only  // full attention only: [units][Ncap] scores of the valid rows
 
 cudaError_t launch_copy(const void* src, void* dst, size_t bytes, cudaStream_t st);
 cudaError_t launch_gather(const void* base, size_t base_bytes, const int32_t* rows, int nrows, unsigned* flag,
