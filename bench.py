@@ -304,6 +304,9 @@ def run_ours(args, rank, world, dev):
         res["e2e"] = e2e_measure(tsa, w, plan, layers, step_args, O, idx, stream, args)
     if args.offload:
         res["offload"] = offload_probe(tsa, w, plan, layers, Kmean, ws, kreq_t, idx, O, stream)
+    if args.probes:
+        res["probes"] = {"handoff": handoff_probe(tsa, w, plan, layers, kreq_t, stream),
+                         "overlap": overlap_probe(tsa, w, plan, lens, dev, stream)}
     return res
 
 
@@ -469,6 +472,64 @@ def offload_probe(tsa, w, plan, layers, Kmean, ws, kreq_t, idx, O, stream, reps=
             "whole_layer_kv_bytes": whole, "whole_layer_copy_us": whole / (h2d_gbs * 1e9) * 1e6,
             "note": "K and V of one layer in pinned host memory; attention reads only the selected "
                     "128-token blocks across the host link; cold L2, median of %d single launches" % reps}
+
+
+def handoff_probe(tsa, w, plan, layers, kreq_t, stream, reps=10):
+    """Layer 0's tensors as a full layer (dense attention), as a full layer that
+    hands on its top-k (HyLRA's sensitive layer), and as a SELECT step: each in a
+    CUDA graph of `reps` decode steps, warm and after an L2 flush (cold)."""
+    L = layers[0]
+    dev = L.Q.device
+    shape = tsa.shape_of(L.Q, L.K)
+    ws = torch.empty(max(tsa.workspace_size(shape, plan.k_max, w.block, m) for m in (tsa.FULL, tsa.SELECT)),
+                     dtype=torch.uint8, device=dev)
+    tsa.workspace_init(ws)
+    km = None
+    if w.block > 1:
+        km = torch.zeros(w.B, w.Hkv, -(-w.Ncap // w.block), w.d, dtype=torch.float32, device=dev)
+        tsa.block_summarize(L.K, L.seq_lens, w.block, km, ws, shape=shape)
+    O = torch.empty(w.B, w.Hq, w.d, dtype=torch.float32, device=dev)
+    ix = torch.full((w.B, w.Hkv, plan.k_max), -1, dtype=torch.int32, device=dev)
+    common = dict(scale=w.scale, k_max=plan.k_max, block=w.block, k_per_seq=kreq_t, Kmean=km)
+    steps = {"full": tsa.step_args(L.Q, L.K, L.V, L.seq_lens, O, ws, mode=tsa.FULL, scale=w.scale),
+             "full_handing_on_topk": tsa.step_args(L.Q, L.K, L.V, L.seq_lens, O, ws, mode=tsa.FULL,
+                                                   idx_out=ix, **common),
+             "select": tsa.step_args(L.Q, L.K, L.V, L.seq_lens, O, ws, mode=tsa.SELECT, idx_out=ix, **common)}
+    flush = L2Flush(dev)
+    f_us = graph_us(flush, stream, reps)
+    out = {}
+    for name, a in steps.items():
+        out[name] = {"warm_us": graph_us(lambda a=a: tsa.decode_step(a, stream), stream, reps),
+                     "cold_us": graph_us(lambda a=a: (flush(), tsa.decode_step(a, stream)), stream, reps) - f_us}
+    tsa.check_device_status(ws, stream)
+    out["kv_bytes"] = (L.K.numel() + L.V.numel()) * 2
+    return out
+
+
+def overlap_probe(tsa, w, plan, lens, dev, stream, n_layers=32, keep=0.7, reps=10):
+    """tsa_index_overlap over `n_layers` layers' index lists of this workload's
+    shape (synthetic lists: each layer keeps a fraction `keep` of the previous
+    layer's rows), timed with CUDA events around `reps` launches."""
+    from top_sparse_attention_02_b200 import inputs
+
+    n = [int(lens[b]) if w.block == 1 else -(-int(lens[b]) // w.block) for b in range(w.B) for _ in range(w.Hkv)]
+    k = [int(plan.kreq[b]) for b in range(w.B) for _ in range(w.Hkv)]
+    idx = inputs.layer_index_lists(n_layers, n, k, plan.k_max, keep, seed=5).to(dev)
+    units = idx.shape[1]
+    counts = torch.empty(n_layers, n_layers, units, dtype=torch.int32, device=dev)
+    M = torch.empty(n_layers, n_layers, dtype=torch.float64, device=dev)
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    tsa.index_overlap(idx, counts, M, ws, stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(reps):
+            tsa.index_overlap(idx, counts, M, ws, stream)
+        e1.record(stream)
+    stream.synchronize()
+    tsa.check_device_status(ws, stream)
+    return {"layers": n_layers, "units": units, "k_max": plan.k_max, "us": e0.elapsed_time(e1) * 1e3 / reps,
+            "M_next_layer_mean": float(torch.diagonal(M, -1).mean()) if n_layers > 1 else 1.0}
 
 
 def copy_probe(tsa, dev, stream, nbytes=2 << 30):
@@ -700,6 +761,9 @@ def main():
     ap.add_argument("--workload", default="reuse128k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--probes", action="store_true",
+                    help="also time layer 0 as a full layer with and without handing on its top-k, "
+                         "and the layer overlap matrix over 32 layers of this shape")
     ap.add_argument("--offload", action="store_true",
                     help="block-mode workloads: also time a layer whose K/V sit in pinned host memory")
     ap.add_argument("--ncap", type=int, default=0,

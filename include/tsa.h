@@ -231,6 +231,26 @@ tsa_status tsa_decode_step(const tsa_step_args* args, void* stream);
 tsa_status tsa_index_overlap(const int32_t* idx, int32_t n_layers, int32_t units, int32_t k_max,
                              int32_t* counts, double* M, void* ws, size_t ws_bytes, void* stream);
 
+/* HyLRA's offline reuse policy (HyLRA sec. 2.2, dynamic programming over M).
+ * HOST function: M, force_full, source, n_full and total_sim are host pointers;
+ * nothing is enqueued and no GPU is needed.
+ *  - M [n_layers, n_layers] double, the layout tsa_index_overlap writes:
+ *    M[j*n_layers + i] = the similarity of source layer i to target layer j, i < j
+ *    (entries on and above the diagonal are not read).
+ *  - A policy gives every layer j a source s_j <= j: s_j = j is a full layer
+ *    (a reset: full attention that hands on its top-k, TSA_FULL with idx_out);
+ *    s_j = s_{j-1} < j reuses that source's indices (TSA_REUSE), allowed only
+ *    if M[j][s_j] > theta (strictly).  Layer 0, and every layer with
+ *    force_full[j] != 0 (force_full may be NULL), is a full layer.
+ *  - The policy returned has the fewest full layers, then the largest sum over
+ *    the reusing layers j of M[j][s_j] (added in layer order); among policies
+ *    equal in both, the smallest source sequence compared from the last layer
+ *    backwards.  source [n_layers] int32 receives it; n_full and total_sim (may
+ *    be NULL) its two costs.
+ *  - 1 <= n_layers <= 4096; theta not NaN (NaN entries of M never allow reuse). */
+tsa_status tsa_reuse_policy(const double* M, int32_t n_layers, double theta, const uint8_t* force_full,
+                            int32_t* source, int32_t* n_full, double* total_sim);
+
 /* ------------------------------------------------------------------ status */
 
 /* Wait for `stream`, then read and clear the device error flag in `ws`:

@@ -209,6 +209,43 @@ def index_overlap(idx):
     return counts, M
 
 
+def reuse_policy(M, theta: float, force_full=None):
+    """HyLRA's offline policy (HyLRA, sec. 2.2) by exhaustive search, for small L.
+
+    Every choice of full layers (layer 0 and the forced ones always full) is a
+    policy; each other layer reuses the indices of the latest full layer before it
+    and is allowed only if M[j][source] > theta.  Among the allowed policies: fewest
+    full layers, then the largest similarity of the reusing layers (summed in layer
+    order), then the smallest source sequence read from the last layer backwards.
+    M is [L, L] with row = target layer.  Returns (source, n_full, total_sim)."""
+    M = np.asarray(M, dtype=np.float64)
+    L = M.shape[0]
+    forced = [j == 0 or (force_full is not None and bool(force_full[j])) for j in range(L)]
+    free = [j for j in range(1, L) if not forced[j]]
+    best = None
+    for mask in range(1 << len(free)):
+        full = list(forced)
+        for b, j in enumerate(free):
+            if mask >> b & 1:
+                full[j] = True
+        src, cur, sim, ok = [], 0, 0.0, True
+        for j in range(L):
+            if full[j]:
+                cur = j
+            elif not M[j, cur] > theta:
+                ok = False
+                break
+            else:
+                sim += M[j, cur]
+            src.append(cur)
+        if not ok:
+            continue
+        key = (sum(full), -sim, src[::-1])
+        if best is None or key < best[0]:
+            best = (key, src, sum(full), sim)
+    return np.array(best[1], dtype=np.int32), best[2], best[3]
+
+
 def nblocks_of(seq_lens, block: int) -> np.ndarray:
     L = _i32(seq_lens)
     return ((L.astype(np.int64) + block - 1) // block).astype(np.int32)

@@ -33,7 +33,7 @@ def test_header_declares_the_boundary():
     names = declared_functions()
     for want in ("sparse_decode_score", "topk_select", "sparse_decode_attn", "tsa_decode_step",
                  "tsa_block_summarize", "tsa_workspace_size", "tsa_check_device_status",
-                 "tsa_index_overlap"):
+                 "tsa_index_overlap", "tsa_reuse_policy"):
         assert want in names
 
 
@@ -187,3 +187,36 @@ def test_binding_raises_on_error(tsa):
     with pytest.raises(tsa.TsaError) as e:
         tsa.workspace_size(tsa.tsa_shape(1, 8, 2, 64, 96), 4, 1, tsa.SELECT)
     assert "head dimension" in str(e.value)
+
+
+def test_reuse_policy_matches_exhaustive_search(tsa):
+    """The library's dynamic program (a host function) against the oracle's
+    exhaustive search over every choice of full layers."""
+    import numpy as np
+
+    import oracle
+
+    rng = np.random.default_rng(17)
+    for trial in range(300):
+        L = int(rng.integers(1, 11))
+        if trial % 3 == 0:  # coarse values: many exact ties
+            M = rng.integers(0, 5, (L, L)) / 4.0
+        else:
+            M = rng.random((L, L))
+        theta = float(rng.choice([0.0, 0.25, 0.5, 0.7, 0.9]))
+        ff = (rng.random(L) < 0.15).astype(np.uint8) if trial % 2 else None
+        got = tsa.reuse_policy(M, theta, ff)
+        want = oracle.reuse_policy(M, theta, ff)
+        assert got[0].tolist() == want[0].tolist(), (trial, M, theta, ff)
+        assert got[1] == want[1] and got[2] == want[2]
+
+
+def test_reuse_policy_argument_errors(tsa):
+    import numpy as np
+
+    L = tsa.lib()
+    assert L.tsa_reuse_policy(None, 3, 0.5, None, 0x1000, None, None) == 1
+    M = np.zeros((2, 2))
+    assert L.tsa_reuse_policy(M.ctypes.data, 0, 0.5, None, 0x1000, None, None) == 1
+    assert L.tsa_reuse_policy(M.ctypes.data, 2, float("nan"), None, 0x1000, None, None) == 1
+    assert "NaN" in tsa.last_error()

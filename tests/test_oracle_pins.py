@@ -414,3 +414,54 @@ def test_overlap_degenerate_shapes():
         counts, M = oracle.index_overlap(np.full(shape, -1, dtype=np.int32))
         assert counts.shape == (shape[0], shape[0], shape[1]) and (counts == 0).all()
         assert (M == np.tril(np.ones((shape[0], shape[0])))).all()
+
+
+# ------------------------------------------------------------------ reuse policy (HyLRA sec. 2.2)
+
+def _sim(L, entries, fill=0.0):
+    """Lower-triangular M [L, L] (row = target) from {(target, source): value}."""
+    M = np.full((L, L), fill)
+    for (j, i), v in entries.items():
+        M[j, i] = v
+    return M
+
+
+def test_policy_everything_similar_or_nothing_similar():
+    """All similarities 1 > theta: one full layer, every other reuses layer 0;
+    all 0: every layer is full."""
+    src, n, sim = oracle.reuse_policy(np.ones((6, 6)), 0.5)
+    assert src.tolist() == [0] * 6 and n == 1 and sim == 5.0
+    src, n, sim = oracle.reuse_policy(np.zeros((6, 6)), 0.5)
+    assert src.tolist() == list(range(6)) and n == 6 and sim == 0.0
+
+
+def test_policy_beats_resetting_as_late_as_possible():
+    """Layer 0 reaches layers 1-2, layer 1 reaches 2-4, layers 3 and 4 nothing
+    useful: resetting only when forced (0, 3, 4) takes 3 full layers, resetting
+    early at 1 covers the rest with 2."""
+    M = _sim(5, {(1, 0): 0.9, (2, 0): 0.9, (2, 1): 0.8, (3, 1): 0.8, (4, 1): 0.8})
+    src, n, sim = oracle.reuse_policy(M, 0.5)
+    assert src.tolist() == [0, 1, 1, 1, 1] and n == 2 and sim == 0.8 + 0.8 + 0.8
+
+
+def test_policy_prefers_more_similarity_at_equal_full_count():
+    """Two 2-full policies: layer 1 reusing layer 0 (0.6) or layer 2 reusing
+    layer 1 (0.9); the second keeps more."""
+    M = _sim(3, {(1, 0): 0.6, (2, 1): 0.9})
+    src, n, sim = oracle.reuse_policy(M, 0.5)
+    assert src.tolist() == [0, 1, 1] and n == 2 and sim == 0.9
+
+
+def test_policy_threshold_is_strict_and_forced_layers_are_full():
+    M = _sim(3, {(1, 0): 0.5, (2, 0): 0.75, (2, 1): 0.75})
+    assert oracle.reuse_policy(M, 0.5)[0].tolist() == [0, 1, 1]  # 0.5 does not exceed 0.5
+    assert oracle.reuse_policy(M, 0.49)[0].tolist() == [0, 0, 0]
+    src, n, _ = oracle.reuse_policy(M, 0.49, force_full=[0, 0, 1])
+    assert src.tolist() == [0, 0, 2] and n == 2
+
+
+def test_policy_ties_go_to_the_smaller_source_from_the_end():
+    """[0, 0, 2] and [0, 1, 1] both have 2 full layers and similarity 0.5; read
+    from the last layer, 1 < 2."""
+    M = _sim(3, {(1, 0): 0.5, (2, 1): 0.5})
+    assert oracle.reuse_policy(M, 0.25)[0].tolist() == [0, 1, 1]

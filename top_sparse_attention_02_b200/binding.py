@@ -56,6 +56,7 @@ _SIGS = {
                                                   _f32, _vp, _vp]),
     "tsa_decode_step": (ctypes.c_int, [ctypes.POINTER(tsa_step_args), _vp]),
     "tsa_index_overlap": (ctypes.c_int, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _sz, _vp]),
+    "tsa_reuse_policy": (ctypes.c_int, [_vp, _i32, ctypes.c_double, _vp, _vp, _vp, _vp]),
     "tsa_check_device_status": (ctypes.c_int, [_vp, _vp]),
     "tsa_last_error_string": (ctypes.c_char_p, []),
     "tsa_launch_count": (ctypes.c_uint64, []),
@@ -191,6 +192,23 @@ def index_overlap(idx, counts, M, ws, stream=None):
     L, units, k_max = idx.shape[0], math.prod(idx.shape[1:-1]), idx.shape[-1]
     _ok(_lib.tsa_index_overlap(_ptr(idx), L, units, k_max, _ptr(counts), _ptr(M), *_wsargs(ws),
                                _stream(stream)))
+
+
+def reuse_policy(M, theta: float, force_full=None):
+    """HyLRA's reuse policy from the similarity matrix M [L, L] (host, float64,
+    row = target layer): returns (source [L] int32 numpy array, n_full, total_sim)."""
+    import numpy as np
+
+    Mh = np.ascontiguousarray(M.cpu().numpy() if isinstance(M, torch.Tensor) else M, dtype=np.float64)
+    L = Mh.shape[0]
+    assert Mh.shape == (L, L)
+    ff = None if force_full is None else np.ascontiguousarray(np.asarray(force_full, dtype=np.uint8))
+    src = np.empty(L, dtype=np.int32)
+    nf = ctypes.c_int32()
+    sim = ctypes.c_double()
+    _ok(_lib.tsa_reuse_policy(Mh.ctypes.data, L, float(theta), None if ff is None else ff.ctypes.data,
+                              src.ctypes.data, ctypes.byref(nf), ctypes.byref(sim)))
+    return src, nf.value, sim.value
 
 
 def check_device_status(ws, stream=None):
