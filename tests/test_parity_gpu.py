@@ -631,3 +631,52 @@ def test_offload_refuses_memory_the_device_cannot_read(cuda_dev):
     with pytest.raises(tsa.TsaError, match="UNSUPPORTED"):
         G.step(Q, _pinned(L.K), _pinned(L.V), ln, mode=tsa.SELECT, scale=SCALE, k_max=4,
                flags=tsa.KV_HOST)
+
+
+def test_hylra_calibrate_then_run_the_policy(cuda_dev):
+    """HyLRA end to end (secs. 2.2-2.3): calibrate on a stack of layers whose
+    queries drift (every layer full, handing on its top-k), measure M with
+    tsa_index_overlap, derive the policy with tsa_reuse_policy, then run the stack
+    by it -- resets as full layers that hand on their top-k, the others reusing
+    their source's list -- and check every layer against the oracle."""
+    B, Hq, Hkv, N, nl = 2, 16, 4, 6000, 6
+    kreq, k_max = [240, 150], 240
+    lens = [6000, 3777]
+    L0 = layer(B, Hq, Hkv, N, lens, seed=121)
+    Q0, K, V, ln = G.to_dev(L0, cuda_dev)
+    qs = [L0.Q]
+    for l in range(1, nl):  # layers 2 and 4 drift far, the others a little
+        qs.append(inputs.drift_query(qs[-1], 1.5 if l in (2, 4) else 0.15, 300 + l))
+    ws = G.ws_for(Q0, K, k_max, 1, tsa.FULL)
+    kr = torch.tensor(kreq, dtype=torch.int32, device=cuda_dev)
+    O = torch.empty(B, Hq, 128, dtype=torch.float32, device=cuda_dev)
+    cal = torch.full((nl, B, Hkv, k_max), -7, dtype=torch.int32, device=cuda_dev)
+    for l in range(nl):
+        a = tsa.step_args(qs[l].to(cuda_dev), K, V, ln, O, ws, mode=tsa.FULL, scale=SCALE, k_max=k_max,
+                          k_per_seq=kr, idx_out=cal[l])
+        tsa.decode_step(a)
+    tsa.check_device_status(ws)
+    counts, M = _check_overlap(cal)
+    # a threshold between the small-drift and the large-drift neighbours
+    sub = np.sort(np.diagonal(M, -1))
+    theta = float(sub[1] + sub[2]) / 2
+    src, n_full, sim = tsa.reuse_policy(M, theta)
+    want = oracle.reuse_policy(M, theta)
+    assert src.tolist() == want[0].tolist() and n_full == want[1]
+    assert 1 < n_full < nl, f"the drift should make some but not all layers reset: {src}"
+    # run the stack by the policy
+    lists = torch.full((nl, B, Hkv, k_max), -7, dtype=torch.int32, device=cuda_dev)
+    for l in range(nl):
+        q = qs[l].to(cuda_dev)
+        if src[l] == l:
+            O_l, idx_l = G.step(q, K, V, ln, mode=tsa.FULL, scale=SCALE, k_max=k_max, kreq=kreq, ws=ws,
+                                emit=True)
+            lists[l].copy_(idx_l)
+            ref = oracle.attn(qs[l], L0.K, L0.V, L0.seq_lens, None, None, 0, 1, SCALE)
+            compare_idx(lists[l].cpu().numpy(), oracle.scores(qs[l], L0.K, L0.seq_lens, SCALE), lens, kreq)
+        else:
+            O_l, _ = G.step(q, K, V, ln, mode=tsa.REUSE, scale=SCALE, k_max=k_max, kreq=kreq,
+                            idx_in=lists[src[l]], ws=ws)
+            ref = oracle.attn(qs[l], L0.K, L0.V, L0.seq_lens, lists[src[l]].cpu().numpy(), kreq, k_max, 1, SCALE)
+        torch.cuda.synchronize()
+        check_output(O_l.cpu().numpy(), ref, f"layer {l} ({'full' if src[l] == l else f'reuses {src[l]}'})")
