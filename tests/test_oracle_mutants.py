@@ -82,3 +82,48 @@ def test_mutant_is_caught(name, old, new, nth, tmp_path):
 def test_unmutated_oracle_passes_every_pin():
     for _, f in PIN_TESTS:
         _call(f)
+
+
+# The numpy parts of the oracle: (name, function, text in its source, replacement)
+PY_MUTANTS = [
+    ("overlap normalised by the source set", "index_overlap",
+     "counts[i, j, u] / sets[j][u].size", "counts[i, j, u] / sets[i][u].size"),
+    ("overlap keeps empty targets", "index_overlap",
+     "for u in range(units) if sets[j][u].size > 0]", "for u in range(units) if True]"),
+    ("overlap matrix transposed", "index_overlap", "M[j, i] = float(np.mean(ratios))",
+     "M[i, j] = float(np.mean(ratios))"),
+    ("overlap counts the -1 padding", "index_overlap", "a[l, u][a[l, u] >= 0]", "a[l, u]"),
+    ("overlap of no units is 0", "index_overlap", "if ratios else 1.0", "if ratios else 0.0"),
+    ("policy threshold not strict", "reuse_policy", "not M[j, cur] > theta", "not M[j, cur] >= theta"),
+    ("policy ignores similarity", "reuse_policy", "key = (sum(full), -sim, src[::-1])",
+     "key = (sum(full), src[::-1])"),
+    ("policy minimises similarity", "reuse_policy", "key = (sum(full), -sim, src[::-1])",
+     "key = (sum(full), sim, src[::-1])"),
+    ("policy ties read forwards", "reuse_policy", "key = (sum(full), -sim, src[::-1])",
+     "key = (sum(full), -sim, src)"),
+    ("policy ignores forced layers", "reuse_policy",
+     "forced = [j == 0 or (force_full is not None and bool(force_full[j])) for j in range(L)]",
+     "forced = [j == 0 for j in range(L)]"),
+    ("policy reads M transposed", "reuse_policy", "not M[j, cur] > theta", "not M[cur, j] > theta"),
+]
+
+
+@pytest.mark.parametrize("name,fn,old,new", PY_MUTANTS, ids=[m[0] for m in PY_MUTANTS])
+def test_python_mutant_is_caught(name, fn, old, new, monkeypatch):
+    import inspect
+    import warnings
+
+    src = inspect.getsource(getattr(oracle, fn))
+    assert src.count(old) == 1, f"mutation site for {name!r} not found once"
+    ns = dict(vars(oracle))
+    exec(compile(src.replace(old, new), f"<mutant {name}>", "exec"), ns)
+    monkeypatch.setattr(oracle, fn, ns[fn])
+    caught = []
+    with warnings.catch_warnings():
+        warnings.simplefilter("ignore")
+        for tname, f in PIN_TESTS:
+            try:
+                _call(f)
+            except Exception:  # a failed pin, or a mutant that cannot even run
+                caught.append(tname)
+    assert caught, f"no pin rejects the mutant {name!r}"

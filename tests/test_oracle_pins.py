@@ -450,6 +450,10 @@ def test_policy_prefers_more_similarity_at_equal_full_count():
     M = _sim(3, {(1, 0): 0.6, (2, 1): 0.9})
     src, n, sim = oracle.reuse_policy(M, 0.5)
     assert src.tolist() == [0, 1, 1] and n == 2 and sim == 0.9
+    # and the other way round, where the tie rule alone would pick the other policy
+    M = _sim(3, {(1, 0): 0.9, (2, 1): 0.6})
+    src, n, sim = oracle.reuse_policy(M, 0.5)
+    assert src.tolist() == [0, 0, 2] and n == 2 and sim == 0.9
 
 
 def test_policy_threshold_is_strict_and_forced_layers_are_full():
