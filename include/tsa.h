@@ -206,6 +206,56 @@ typedef struct {
  * block, TSA_FULL), k_max > 0. */
 tsa_status tsa_decode_step(const tsa_step_args* args, void* stream);
 
+/* ------------------------------------------------------------------ sequence sharding */
+
+/* One sequence's cache split by rows across R ranks (R <= 64): shard r holds rows
+ * [row0_r, row0_r + Ncap_r) of every unit, with row0 increasing with r (rank
+ * order = row order), as K_shard, V_shard [B, Hkv, Ncap_r, d] and its own
+ * lengths shard_lens[b] = clamp(len_b - row0_r, 0, Ncap_r).  A SELECT layer then
+ * runs as: tsa_shard_select on every rank; an all-gather of the candidates (rank
+ * order); tsa_shard_merge (every rank, same result); tsa_shard_attend on every
+ * rank; an all-gather of the parts; tsa_shard_combine.  The result is the
+ * single-GPU SELECT step's: the same indices (every row of the global top-k is
+ * among its shard's top-k, and rank order keeps the lower-index tie rule) and
+ * the same attention up to rounding (split-K over shards, as flash decoding
+ * splits a sequence).  shard_shape is (B, Hq, Hkv, Ncap_r, d); `shape` in the
+ * merge and combine calls is the same with any Ncap.  Workspace: at least
+ * tsa_shard_workspace_size(shard_shape, k_max, n_shards), shared by the four
+ * calls of a rank, initialised with tsa_workspace_init. */
+size_t tsa_shard_workspace_size(tsa_shape shard_shape, int32_t k_max, int32_t n_shards);
+
+/* This shard's top-k (score -> select, as in a SELECT step, with
+ * k_b = min(k_per_seq[b], shard_lens[b])) as candidates: cand_scores
+ * [B, Hkv, k_max] fp32 and cand_rows [B, Hkv, k_max] int32 GLOBAL rows
+ * (row0 + local row), ascending, then (-inf, -1). */
+tsa_status tsa_shard_select(const void* Q, const void* K_shard, const int32_t* shard_lens, tsa_shape shard_shape,
+                            const int32_t* k_per_seq, int32_t k_max, float scale, int32_t row0,
+                            float* cand_scores, int32_t* cand_rows, void* ws, size_t ws_bytes, void* stream);
+
+/* The exact global top-k from the gathered candidates of all shards:
+ * cand_scores, cand_rows [n_shards, B, Hkv, k_max] (rank order) -> idx
+ * [B, Hkv, k_max] global rows, ascending, then -1.  Candidates out of row
+ * order across shards set the device bounds flag. */
+tsa_status tsa_shard_merge(const float* cand_scores, const int32_t* cand_rows, int32_t n_shards, tsa_shape shape,
+                           const int32_t* k_per_seq, int32_t k_max, int32_t* idx, void* ws, size_t ws_bytes,
+                           void* stream);
+
+/* This shard's part of the attention over the global idx: the rows of idx in
+ * [row0, row0 + Ncap_r).  O_part [B, Hq, d] fp32 is the softmax-normalised
+ * output over those rows (0 if none) and lse_part [B, Hq] fp32 the base-2
+ * log-sum-exp of their scaled logits, log2(sum_j 2^(scale*log2(e)*q.k_j)), or
+ * -inf if the shard holds none of them. */
+tsa_status tsa_shard_attend(const void* Q, const void* K_shard, const void* V_shard, const int32_t* shard_lens,
+                            tsa_shape shard_shape, const int32_t* idx, const int32_t* k_per_seq, int32_t k_max,
+                            int32_t row0, float scale, float* O_part, float* lse_part, void* ws, size_t ws_bytes,
+                            void* stream);
+
+/* O [B, Hq, d] = sum_r 2^(lse_r - M) O_r / sum_r 2^(lse_r - M), M = max_r lse_r
+ * (0 where every lse_r is -inf), from O_parts [n_shards, B, Hq, d] and
+ * lse_parts [n_shards, B, Hq].  O_parts and O 16-byte aligned. */
+tsa_status tsa_shard_combine(const float* O_parts, const float* lse_parts, int32_t n_shards, tsa_shape shape,
+                             float* O, void* stream);
+
 /* ------------------------------------------------------------------ reuse profiling */
 
 /* Overlap of the top-k index sets of n_layers layers: the similarity matrix

@@ -220,3 +220,40 @@ def test_reuse_policy_argument_errors(tsa):
     assert L.tsa_reuse_policy(M.ctypes.data, 0, 0.5, None, 0x1000, None, None) == 1
     assert L.tsa_reuse_policy(M.ctypes.data, 2, float("nan"), None, 0x1000, None, None) == 1
     assert "NaN" in tsa.last_error()
+
+
+def test_shard_entry_points_argument_errors(tsa):
+    """The sequence-sharding calls: host-side checks only (fake aligned addresses)."""
+    L = tsa.lib()
+    s = _shape(tsa, B=2, Hq=8, Hkv=2, N=1000)
+    n1 = tsa.shard_workspace_size(s, 64, 1)
+    n64 = tsa.shard_workspace_size(s, 64, 64)  # the merge's candidates: 4 units x 64 shards x 64
+    assert n1 >= 256 + 4 * 2048 * 4 and n1 % 256 == 0
+    # the merge's scratch starts after the flag, the histograms and the split counters
+    assert n64 >= (256 + 4 * 2048 * 4 + 256) + 2 * (4 * 64 * 64 * 4)
+    assert L.tsa_shard_workspace_size(s, 64, 65) == 0 and "n_shards" in tsa.last_error()
+    args = (0x1000, 0x2000, 0x3000, s, None, 64, 0.1, 0, 0x4000, 0x5000, 0x10000, 1 << 30, None)
+    # every call below fails a host-side check before anything is launched
+    bad = list(args)
+    bad[7] = -5
+    assert L.tsa_shard_select(*bad) == 1 and "row0" in tsa.last_error()
+    bad = list(args)
+    bad[5] = 0
+    assert L.tsa_shard_select(*bad) == 1 and "k_max" in tsa.last_error()
+    bad = list(args)
+    bad[1] = 0x2008
+    assert L.tsa_shard_select(*bad) == 1 and "aligned" in tsa.last_error()
+    bad = list(args)
+    bad[11] = 100
+    assert L.tsa_shard_select(*bad) == 3
+    assert L.tsa_shard_merge(0x1000, 0x2000, 0, s, None, 64, 0x3000, 0x10000, 1 << 30, None) == 1
+    assert L.tsa_shard_merge(0x1000, None, 2, s, None, 64, 0x3000, 0x10000, 1 << 30, None) == 1
+    huge = tsa.tsa_shape(2, 8, 2, 1000, 128)
+    assert L.tsa_shard_merge(0x1000, 0x2000, 64, huge, None, 1 << 16, 0x3000, 0x10000, 1 << 40, None) == 2
+    assert "capacity" in tsa.last_error()
+    assert L.tsa_shard_attend(0x1000, 0x2000, 0x3000, 0x4000, s, 0x5000, None, 64, -1, 0.1, 0x6000, 0x7000,
+                              0x10000, 1 << 30, None) == 1
+    assert L.tsa_shard_attend(0x1000, 0x2000, 0x3000, 0x4000, s, None, None, 64, 0, 0.1, 0x6000, 0x7000,
+                              0x10000, 1 << 30, None) == 1
+    assert L.tsa_shard_combine(0x1000, 0x2000, 0, s, 0x3000, None) == 1
+    assert L.tsa_shard_combine(0x1008, 0x2000, 2, s, 0x3000, None) == 1 and "aligned" in tsa.last_error()

@@ -46,3 +46,138 @@ def test_two_ranks_take_the_slowest_time_and_sum_the_work():
     got = sorted(q.get(timeout=10) for _ in range(2))
     assert [g[1] for g in got] == [1.5, 1.5]  # both ranks report the max
     assert got[0][2] == pytest.approx(2 * 10**12 / 2e-3 / 1e12)  # work of both replicas
+
+
+# ------------------------------------------------------------------ sequence-sharded SELECT step
+
+class OracleShardOps:
+    """The four libtsa sharding calls restated with the fp64 oracle on CPU tensors,
+    so that the exchange in shard.sharded_select_step can run over gloo."""
+
+    @staticmethod
+    def shape_of(Q, K):
+        return (Q.shape[0], Q.shape[1], K.shape[1], K.shape[2], Q.shape[2])
+
+    @staticmethod
+    def shard_select(Q, K_r, lens_r, kreq, k_max, scale, row0, cand_scores, cand_rows, ws, stream):
+        import numpy as np
+
+        import oracle
+
+        S = oracle.scores(Q, K_r, lens_r, scale)
+        idx = oracle.topk(S, lens_r.numpy(), kreq.numpy(), k_max)
+        B, Hkv, _ = idx.shape
+        cs = np.full(idx.shape, -np.inf, dtype=np.float32)
+        cr = np.full(idx.shape, -1, dtype=np.int32)
+        for b in range(B):
+            for h in range(Hkv):
+                for t, r in enumerate(idx[b, h]):
+                    if r >= 0:
+                        cs[b, h, t], cr[b, h, t] = S[b, h, r], row0 + r
+        cand_scores.copy_(torch.from_numpy(cs))
+        cand_rows.copy_(torch.from_numpy(cr))
+
+    @staticmethod
+    def shard_merge(all_s, all_r, shape, kreq, k_max, idx, ws, stream):
+        R, B, Hkv, _ = all_s.shape
+        idx.fill_(-1)
+        for b in range(B):
+            for h in range(Hkv):
+                pairs = [(float(all_s[r, b, h, t]), int(all_r[r, b, h, t])) for r in range(R) for t in range(k_max)
+                         if all_r[r, b, h, t] >= 0]
+                kb = min(int(kreq[b]), len(pairs))
+                rows = sorted(row for _, row in sorted(pairs, key=lambda p: (-p[0], p[1]))[:kb])
+                idx[b, h, :kb] = torch.tensor(rows, dtype=torch.int32)
+
+    @staticmethod
+    def shard_attend(Q, K_r, V_r, lens_r, idx, kreq, k_max, row0, scale, O_part, lse_part, ws, stream):
+        import numpy as np
+
+        import oracle
+
+        B, Hkv, ncap = K_r.shape[:3]
+        g = Q.shape[1] // Hkv
+        local = np.full((B, Hkv, k_max), -1, dtype=np.int32)
+        lse = np.full((B, Q.shape[1]), -np.inf)
+        q, k = Q.double().numpy(), K_r.double().numpy()
+        for b in range(B):
+            for h in range(Hkv):
+                own = [int(x) - row0 for x in idx[b, h] if row0 <= x < row0 + ncap]
+                local[b, h, :len(own)] = own
+                for hh in range(g):
+                    if own:
+                        z = scale * (k[b, h, own] @ q[b, h * g + hh])
+                        lse[b, h * g + hh] = (z.max() + np.log(np.exp(z - z.max()).sum())) / np.log(2.0)
+        O_part.copy_(torch.from_numpy(oracle.attn(Q, K_r, V_r, lens_r, local, kreq.numpy(), k_max, 1, scale)))
+        lse_part.copy_(torch.from_numpy(lse))
+
+    @staticmethod
+    def shard_combine(O_all, lse_all, shape, O, stream):
+        M = lse_all.max(dim=0).values
+        w = torch.where(torch.isinf(lse_all), torch.zeros_like(lse_all), torch.exp2(lse_all - M))
+        den = w.sum(dim=0)
+        num = (w.unsqueeze(-1) * O_all).sum(dim=0)
+        O.copy_(torch.where(den.unsqueeze(-1) > 0, num / den.clamp_min(1e-300).unsqueeze(-1), torch.zeros_like(num)))
+
+
+SHARD_CASE = dict(B=2, Hq=8, Hkv=2, N=3000, lens=[3000, 1100], kreq=[90, 90], bounds=[0, 1300, 3000])
+
+
+def _shard_rank_main(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    import datetime
+    import sys
+
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+        from top_sparse_attention_02_b200 import inputs, shard
+
+        c = SHARD_CASE
+        L = inputs.decode_layer(c["B"], c["Hq"], c["Hkv"], c["N"], c["lens"], plant_frac=0.01, seed=41)
+        lo, hi = c["bounds"][rank], c["bounds"][rank + 1]
+        K_r, V_r = L.K[:, :, lo:hi].contiguous(), L.V[:, :, lo:hi].contiguous()
+        lens_r = (L.seq_lens - lo).clamp(0, hi - lo).to(torch.int32)
+        kreq = torch.tensor(c["kreq"], dtype=torch.int32)
+        k_max = max(c["kreq"])
+        O = torch.empty(c["B"], c["Hq"], 128, dtype=torch.float64)
+        idx = torch.empty(c["B"], c["Hkv"], k_max, dtype=torch.int32)
+        shard.sharded_select_step(L.Q, K_r, V_r, lens_r, kreq, k_max, 1 / 128 ** 0.5, lo, O, idx, None,
+                                  ops=OracleShardOps)
+        q.put((rank, idx.numpy(), O.numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_sequence_sharded_step_exchange_over_two_ranks():
+    """Two ranks, each holding a contiguous part of every sequence's rows (the
+    second sequence lies wholly in rank 0's part): after the candidate and the
+    partial exchanges both ranks hold the unsharded top-k and attention."""
+    import sys
+
+    import numpy as np
+
+    sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+    import oracle
+    from parity import check_output, compare_idx
+    from top_sparse_attention_02_b200 import inputs
+
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_shard_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = sorted((q.get(timeout=300) for _ in range(2)), key=lambda x: x[0])
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    c = SHARD_CASE
+    L = inputs.decode_layer(c["B"], c["Hq"], c["Hkv"], c["N"], c["lens"], plant_frac=0.01, seed=41)
+    S = oracle.scores(L.Q, L.K, L.seq_lens, 1 / 128 ** 0.5)
+    k_max = max(c["kreq"])
+    for rank, idx, O in got:
+        compare_idx(idx, S, c["lens"], c["kreq"])
+        ref = oracle.attn(L.Q, L.K, L.V, L.seq_lens, idx, c["kreq"], k_max, 1, 1 / 128 ** 0.5)
+        check_output(O, ref, f"rank {rank}")
+    assert np.array_equal(got[0][1], got[1][1]) and np.array_equal(got[0][2], got[1][2])

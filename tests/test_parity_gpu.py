@@ -680,3 +680,62 @@ def test_hylra_calibrate_then_run_the_policy(cuda_dev):
             ref = oracle.attn(qs[l], L0.K, L0.V, L0.seq_lens, lists[src[l]].cpu().numpy(), kreq, k_max, 1, SCALE)
         torch.cuda.synchronize()
         check_output(O_l.cpu().numpy(), ref, f"layer {l} ({'full' if src[l] == l else f'reuses {src[l]}'})")
+
+
+# ------------------------------------------------------------------ sequence sharding (one GPU, shards in turn)
+
+@pytest.mark.parametrize("case", ["two_uneven", "three_with_an_empty_shard", "four_k_eq_len"])
+def test_sequence_sharded_select_on_one_gpu(cuda_dev, case):
+    """The sharded SELECT step with its R shards run one after another on one
+    GPU and the all-gathers replaced by stacking: the same indices as the one-GPU
+    SELECT step (exact top-k of the whole cache) and the same attention."""
+    if case == "two_uneven":
+        B, Hq, Hkv, N, lens, kreq, bounds = 2, 32, 8, 7000, [7000, 3500], [200, 120], [0, 2900, 7000]
+    elif case == "three_with_an_empty_shard":  # sequence 1 ends inside shard 0
+        B, Hq, Hkv, N, lens, kreq, bounds = 2, 16, 4, 9000, [9000, 100], [300, 300], [0, 4000, 4100, 9000]
+    else:  # k = len: every row, spread over four shards
+        B, Hq, Hkv, N, lens, kreq, bounds = 1, 8, 2, 4096, [4000], [4000], [0, 1024, 2048, 3072, 4096]
+    R, k_max = len(bounds) - 1, max(kreq)
+    L = layer(B, Hq, Hkv, N, lens, seed=131, tail_fill=float("nan"))
+    Q, K, V, ln = G.to_dev(L, cuda_dev)
+    kr = torch.tensor(kreq, dtype=torch.int32, device=cuda_dev)
+    _, idx_one = G.step(Q, K, V, ln, mode=tsa.SELECT, scale=SCALE, k_max=k_max, kreq=kreq)
+    shards = []
+    for r in range(R):
+        lo, hi = bounds[r], bounds[r + 1]
+        K_r, V_r = K[:, :, lo:hi].contiguous(), V[:, :, lo:hi].contiguous()
+        lens_r = (ln - lo).clamp(0, hi - lo).to(torch.int32)
+        ws = torch.empty(tsa.shard_workspace_size(tsa.shape_of(Q, K_r), k_max, R), dtype=torch.uint8,
+                         device=cuda_dev)
+        tsa.workspace_init(ws)
+        shards.append((lo, K_r, V_r, lens_r, ws))
+    cs = torch.full((R, B, Hkv, k_max), float("nan"), dtype=torch.float32, device=cuda_dev)
+    cr = torch.full((R, B, Hkv, k_max), -7, dtype=torch.int32, device=cuda_dev)
+    for r, (lo, K_r, V_r, lens_r, ws) in enumerate(shards):
+        tsa.shard_select(Q, K_r, lens_r, kr, k_max, SCALE, lo, cs[r], cr[r], ws)
+        tsa.check_device_status(ws)
+    idx = torch.full((B, Hkv, k_max), -7, dtype=torch.int32, device=cuda_dev)
+    tsa.shard_merge(cs, cr, tsa.shape_of(Q, K), kr, k_max, idx, shards[0][4])
+    tsa.check_device_status(shards[0][4])
+    S = oracle.scores(L.Q, L.K, L.seq_lens, SCALE)
+    compare_idx(idx.cpu().numpy(), S, lens, kreq)
+    assert torch.equal(idx, idx_one), "the shards must select what one GPU selects"
+    O_parts = torch.full((R, B, Hq, 128), float("nan"), dtype=torch.float32, device=cuda_dev)
+    lse = torch.full((R, B, Hq), float("nan"), dtype=torch.float32, device=cuda_dev)
+    for r, (lo, K_r, V_r, lens_r, ws) in enumerate(shards):
+        tsa.shard_attend(Q, K_r, V_r, lens_r, idx, kr, k_max, lo, SCALE, O_parts[r], lse[r], ws)
+        tsa.check_device_status(ws)
+    O = torch.full((B, Hq, 128), float("nan"), dtype=torch.float32, device=cuda_dev)
+    tsa.shard_combine(O_parts, lse, tsa.shape_of(Q, K), O)
+    torch.cuda.synchronize()
+    ref = oracle.attn(L.Q, L.K, L.V, L.seq_lens, idx.cpu().numpy(), kreq, k_max, 1, SCALE)
+    check_output(O.cpu().numpy(), ref, f"sharded {case}")
+    # each part alone is the attention over the rows its shard holds
+    for r, (lo, K_r, V_r, lens_r, ws) in enumerate(shards):
+        own = np.where((idx.cpu().numpy() >= lo) & (idx.cpu().numpy() < lo + K_r.shape[2]),
+                       idx.cpu().numpy() - lo, -1).astype(np.int32)
+        own = np.sort(np.where(own < 0, np.iinfo(np.int32).max, own), axis=-1)
+        own = np.where(own == np.iinfo(np.int32).max, -1, own).astype(np.int32)
+        ref_r = oracle.attn(L.Q, L.K[:, :, lo:lo + K_r.shape[2]].contiguous(), L.V[:, :, lo:lo + K_r.shape[2]].contiguous(),
+                            lens_r.cpu(), own, kreq, k_max, 1, SCALE)
+        check_output(O_parts[r].cpu().numpy(), ref_r, f"{case} shard {r} part")

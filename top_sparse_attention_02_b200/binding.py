@@ -57,6 +57,12 @@ _SIGS = {
     "tsa_decode_step": (ctypes.c_int, [ctypes.POINTER(tsa_step_args), _vp]),
     "tsa_index_overlap": (ctypes.c_int, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _sz, _vp]),
     "tsa_reuse_policy": (ctypes.c_int, [_vp, _i32, ctypes.c_double, _vp, _vp, _vp, _vp]),
+    "tsa_shard_workspace_size": (_sz, [tsa_shape, _i32, _i32]),
+    "tsa_shard_select": (ctypes.c_int, [_vp, _vp, _vp, tsa_shape, _vp, _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp]),
+    "tsa_shard_merge": (ctypes.c_int, [_vp, _vp, _i32, tsa_shape, _vp, _i32, _vp, _vp, _sz, _vp]),
+    "tsa_shard_attend": (ctypes.c_int, [_vp, _vp, _vp, _vp, tsa_shape, _vp, _vp, _i32, _i32, _f32, _vp, _vp, _vp,
+                                        _sz, _vp]),
+    "tsa_shard_combine": (ctypes.c_int, [_vp, _vp, _i32, tsa_shape, _vp, _vp]),
     "tsa_check_device_status": (ctypes.c_int, [_vp, _vp]),
     "tsa_last_error_string": (ctypes.c_char_p, []),
     "tsa_launch_count": (ctypes.c_uint64, []),
@@ -209,6 +215,35 @@ def reuse_policy(M, theta: float, force_full=None):
     _ok(_lib.tsa_reuse_policy(Mh.ctypes.data, L, float(theta), None if ff is None else ff.ctypes.data,
                               src.ctypes.data, ctypes.byref(nf), ctypes.byref(sim)))
     return src, nf.value, sim.value
+
+
+def shard_workspace_size(shard_shape: tsa_shape, k_max: int, n_shards: int) -> int:
+    n = _lib.tsa_shard_workspace_size(shard_shape, k_max, n_shards)
+    if n == 0:
+        raise TsaError(TSA_ERR_INVALID_ARG, last_error())
+    return int(n)
+
+
+def shard_select(Q, K_shard, shard_lens, k_per_seq, k_max: int, scale: float, row0: int, cand_scores, cand_rows,
+                 ws, stream=None):
+    _ok(_lib.tsa_shard_select(_ptr(Q), _ptr(K_shard), _ptr(shard_lens), shape_of(Q, K_shard), _ptr(k_per_seq),
+                              k_max, scale, row0, _ptr(cand_scores), _ptr(cand_rows), *_wsargs(ws), _stream(stream)))
+
+
+def shard_merge(cand_scores, cand_rows, shape: tsa_shape, k_per_seq, k_max: int, idx, ws, stream=None):
+    _ok(_lib.tsa_shard_merge(_ptr(cand_scores), _ptr(cand_rows), cand_scores.shape[0], shape, _ptr(k_per_seq),
+                             k_max, _ptr(idx), *_wsargs(ws), _stream(stream)))
+
+
+def shard_attend(Q, K_shard, V_shard, shard_lens, idx, k_per_seq, k_max: int, row0: int, scale: float, O_part,
+                 lse_part, ws, stream=None):
+    _ok(_lib.tsa_shard_attend(_ptr(Q), _ptr(K_shard), _ptr(V_shard), _ptr(shard_lens), shape_of(Q, K_shard),
+                              _ptr(idx), _ptr(k_per_seq), k_max, row0, scale, _ptr(O_part), _ptr(lse_part),
+                              *_wsargs(ws), _stream(stream)))
+
+
+def shard_combine(O_parts, lse_parts, shape: tsa_shape, O, stream=None):
+    _ok(_lib.tsa_shard_combine(_ptr(O_parts), _ptr(lse_parts), O_parts.shape[0], shape, _ptr(O), _stream(stream)))
 
 
 def check_device_status(ws, stream=None):

@@ -2,6 +2,8 @@
 // workspace layout and stream-ordered launches.  No allocation, no
 // synchronisation (except tsa_check_device_status), no exceptions.
 #include <atomic>
+#include <algorithm>
+#include <climits>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -177,6 +179,168 @@ tsa_status tsa_index_overlap(const int32_t* idx, int32_t n_layers, int32_t units
     cudaError_t e = tsa::launch_index_overlap(idx, n_layers, units, k_max, counts, M, flag_of(ws),
                                               static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "tsa_index_overlap");
+    return TSA_OK;
+}
+
+// ---------------------------------------------------------------- sequence sharding
+
+namespace {
+
+tsa_status check_shards(int n_shards) {
+    if (n_shards < 1 || n_shards > tsa::kMaxShards)
+        return fail(TSA_ERR_INVALID_ARG, "n_shards must be in [1, %d] (got %d)", tsa::kMaxShards, n_shards);
+    return TSA_OK;
+}
+
+// The four calls of a rank share one workspace, and none of them may write over
+// the regions that must be zero when a call starts (the top-digit histograms and
+// the split counters, right after the flag).  select and attend use
+// [flag][histograms][counters][partials][scores][local rows]; the merge writes
+// its scratch (candidate scores, candidate rows, counts, positions) from the end
+// of the counters on, over space that select and attend use only inside a call,
+// at offsets that do not depend on the shard's capacity.
+struct ShardLayout {
+    Layout front;  // select / attend
+    size_t local, front_total;
+    size_t pk_scores, pk_rows, n_cand, pos, merge_total;
+    size_t total() const { return std::max(front_total, merge_total); }
+};
+
+ShardLayout shard_layout(const tsa::Dims& d, int k_max, int R) {
+    ShardLayout S;
+    S.front = layout(d, k_max, 1, true, false, true);
+    S.local = S.front.total;
+    S.front_total = S.local + a256((size_t)d.units() * k_max * 4);
+    size_t off = S.front.partials;  // flag, histograms and counters come first in every layout
+    const size_t wide = a256((size_t)d.units() * R * k_max * 4);
+    S.pk_scores = off;
+    off += wide;
+    S.pk_rows = off;
+    off += wide;
+    S.n_cand = off;
+    off += a256((size_t)d.B * 4);
+    S.pos = off;
+    off += a256((size_t)d.units() * k_max * 4);
+    S.merge_total = off;
+    return S;
+}
+
+}  // namespace
+
+size_t tsa_shard_workspace_size(tsa_shape shard_shape, int32_t k_max, int32_t n_shards) {
+    tsa::Dims d;
+    if (check_shape(shard_shape, &d) != TSA_OK || check_kmax(k_max) != TSA_OK || check_shards(n_shards) != TSA_OK)
+        return 0;
+    return shard_layout(d, k_max, n_shards).total();
+}
+
+tsa_status tsa_shard_select(const void* Q, const void* K_shard, const int32_t* shard_lens, tsa_shape shard_shape,
+                            const int32_t* k_per_seq, int32_t k_max, float scale, int32_t row0,
+                            float* cand_scores, int32_t* cand_rows, void* ws, size_t ws_bytes, void* stream) {
+    tsa::Dims d;
+    TSA_TRY(check_shape(shard_shape, &d));
+    TSA_TRY(check_scale(scale));
+    TSA_TRY(check_kmax(k_max));
+    if (k_max == 0) return fail(TSA_ERR_INVALID_ARG, "tsa_shard_select: k_max must be > 0");
+    if (row0 < 0 || (long long)row0 + d.Ncap > INT32_MAX)
+        return fail(TSA_ERR_INVALID_ARG, "tsa_shard_select: row0 must be >= 0 and row0 + Ncap fit in int32");
+    if (!Q || !K_shard || !shard_lens || !cand_scores || !cand_rows)
+        return fail(TSA_ERR_INVALID_ARG, "tsa_shard_select: NULL pointer");
+    if (!aligned16(Q) || !aligned16(K_shard)) return fail(TSA_ERR_INVALID_ARG, "tsa_shard_select: Q and K must be 16-byte aligned");
+    int C, chunk;
+    if (!tsa::topk_plan(d.Ncap, &C, &chunk))
+        return fail(TSA_ERR_UNSUPPORTED, "tsa_shard_select: %d rows per unit exceed the top-k cluster capacity", d.Ncap);
+    const Layout L = shard_layout(d, k_max, 1).front;
+    TSA_TRY(check_ws(ws, ws_bytes, L.total));
+    char* w = static_cast<char*>(ws);
+    float* scores = reinterpret_cast<float*>(w + L.scores);
+    uint32_t* hist = reinterpret_cast<uint32_t*>(w + L.hist);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = tsa::launch_score(Q, K_shard, shard_lens, d, 1, scale, scores, hist, flag_of(ws), st);
+    if (e != cudaSuccess) return cuda_fail(e, "tsa_shard_select (score)");
+    e = tsa::launch_topk(scores, shard_lens, k_per_seq, k_max, d, 1, cand_rows, hist, flag_of(ws), st);
+    if (e != cudaSuccess) {
+        cudaMemsetAsync(hist, 0, (size_t)d.units() * tsa::kHistBins * sizeof(uint32_t), st);
+        return cuda_fail(e, "tsa_shard_select (top-k)");
+    }
+    e = tsa::launch_shard_pack(scores, d.Ncap, d.units(), k_max, row0, cand_rows, cand_scores, flag_of(ws), st);
+    if (e != cudaSuccess) return cuda_fail(e, "tsa_shard_select (candidates)");
+    return TSA_OK;
+}
+
+tsa_status tsa_shard_merge(const float* cand_scores, const int32_t* cand_rows, int32_t n_shards, tsa_shape shape,
+                           const int32_t* k_per_seq, int32_t k_max, int32_t* idx, void* ws, size_t ws_bytes,
+                           void* stream) {
+    tsa::Dims d;
+    TSA_TRY(check_shape(shape, &d));
+    TSA_TRY(check_shards(n_shards));
+    TSA_TRY(check_kmax(k_max));
+    if (k_max == 0) return fail(TSA_ERR_INVALID_ARG, "tsa_shard_merge: k_max must be > 0");
+    if (!cand_scores || !cand_rows || !idx) return fail(TSA_ERR_INVALID_ARG, "tsa_shard_merge: NULL pointer");
+    const long long width = (long long)n_shards * k_max;
+    int C, chunk;
+    if (width > INT32_MAX || !tsa::topk_plan((int)width, &C, &chunk))
+        return fail(TSA_ERR_UNSUPPORTED, "tsa_shard_merge: %lld candidates per unit exceed the top-k capacity", width);
+    const ShardLayout S = shard_layout(d, k_max, n_shards);  // merge offsets do not depend on Ncap
+    TSA_TRY(check_ws(ws, ws_bytes, S.merge_total));
+    char* w = static_cast<char*>(ws);
+    float* pk_scores = reinterpret_cast<float*>(w + S.pk_scores);
+    int32_t* pk_rows = reinterpret_cast<int32_t*>(w + S.pk_rows);
+    int32_t* n_cand = reinterpret_cast<int32_t*>(w + S.n_cand);
+    int32_t* pos = reinterpret_cast<int32_t*>(w + S.pos);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = tsa::launch_merge_pack(cand_scores, cand_rows, n_shards, d.units(), d.Hkv, k_max, pk_scores,
+                                           pk_rows, n_cand, flag_of(ws), st);
+    if (e != cudaSuccess) return cuda_fail(e, "tsa_shard_merge (pack)");
+    tsa::Dims dc = d;
+    dc.Ncap = (int)width;  // the candidates are the rows of this top-k
+    e = tsa::launch_topk(pk_scores, n_cand, k_per_seq, k_max, dc, 1, pos, nullptr, flag_of(ws), st);
+    if (e != cudaSuccess) return cuda_fail(e, "tsa_shard_merge (top-k)");
+    e = tsa::launch_merge_map(pos, pk_rows, d.units(), (int)width, k_max, idx, st);
+    if (e != cudaSuccess) return cuda_fail(e, "tsa_shard_merge (rows)");
+    return TSA_OK;
+}
+
+tsa_status tsa_shard_attend(const void* Q, const void* K_shard, const void* V_shard, const int32_t* shard_lens,
+                            tsa_shape shard_shape, const int32_t* idx, const int32_t* k_per_seq, int32_t k_max,
+                            int32_t row0, float scale, float* O_part, float* lse_part, void* ws, size_t ws_bytes,
+                            void* stream) {
+    tsa::Dims d;
+    TSA_TRY(check_shape(shard_shape, &d));
+    TSA_TRY(check_scale(scale));
+    TSA_TRY(check_kmax(k_max));
+    if (k_max == 0) return fail(TSA_ERR_INVALID_ARG, "tsa_shard_attend: k_max must be > 0");
+    if (row0 < 0) return fail(TSA_ERR_INVALID_ARG, "tsa_shard_attend: row0 must be >= 0");
+    if (!Q || !K_shard || !V_shard || !shard_lens || !idx || !O_part || !lse_part)
+        return fail(TSA_ERR_INVALID_ARG, "tsa_shard_attend: NULL pointer");
+    if (!aligned16(Q) || !aligned16(K_shard) || !aligned16(V_shard) || !aligned16(O_part))
+        return fail(TSA_ERR_INVALID_ARG, "tsa_shard_attend: Q, K, V and O_part must be 16-byte aligned");
+    const ShardLayout S = shard_layout(d, k_max, 1);
+    const Layout& L = S.front;
+    TSA_TRY(check_ws(ws, ws_bytes, S.front_total));
+    char* w = static_cast<char*>(ws);
+    int32_t* local = reinterpret_cast<int32_t*>(w + S.local);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = tsa::launch_localize(idx, d.units(), k_max, row0, d.Ncap, local, st);
+    if (e != cudaSuccess) return cuda_fail(e, "tsa_shard_attend (local rows)");
+    e = tsa::launch_attn(Q, K_shard, V_shard, shard_lens, local, k_per_seq, k_max, 1, d, scale, L.splits,
+                         reinterpret_cast<float*>(w + L.partials), reinterpret_cast<unsigned*>(w + L.counters), O_part,
+                         flag_of(ws), st, false, nullptr, false, lse_part);
+    if (e != cudaSuccess) return cuda_fail(e, "tsa_shard_attend (attention)");
+    return TSA_OK;
+}
+
+tsa_status tsa_shard_combine(const float* O_parts, const float* lse_parts, int32_t n_shards, tsa_shape shape,
+                             float* O, void* stream) {
+    tsa::Dims d;
+    TSA_TRY(check_shape(shape, &d));
+    TSA_TRY(check_shards(n_shards));
+    if (!O_parts || !lse_parts || !O) return fail(TSA_ERR_INVALID_ARG, "tsa_shard_combine: NULL pointer");
+    if (!aligned16(O_parts) || !aligned16(O))
+        return fail(TSA_ERR_INVALID_ARG, "tsa_shard_combine: O_parts and O must be 16-byte aligned");
+    cudaError_t e = tsa::launch_shard_combine(O_parts, lse_parts, n_shards, d.B * d.Hq, O,
+                                              static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "tsa_shard_combine");
     return TSA_OK;
 }
 

@@ -146,7 +146,7 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
             const int32_t* __restrict__ idx, const int32_t* __restrict__ kreq, int k_max,
             int block, int Hkv, int Ncap, float scale_log2, int S, float* __restrict__ part,
             unsigned* __restrict__ counters, float* __restrict__ O, unsigned* __restrict__ flag, int early,
-            float* __restrict__ sout, float scale) {
+            float* __restrict__ sout, float scale, float* __restrict__ lse) {
     using Cfg = AttnCfg<G>;
     extern __shared__ __align__(128) unsigned char smem_raw[];
     // 1024-byte aligned work area (the swizzled layout needs it)
@@ -557,6 +557,7 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
                 float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (L > 0.f) r = make_float4(A.x / L, A.y / L, A.z / L, A.w / L);
                 *reinterpret_cast<float4*>(O + ((size_t)unit * G + h_me) * kD + 4 * qd_me) = r;
+                if (lse && qd_me == 0) lse[(size_t)unit * G + h_me] = L > 0.f ? s_M[h_me] + log2f(L) : -INFINITY;
             }
             return;
         }
@@ -596,6 +597,7 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
             float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
             if (den > 0.f) r = make_float4(num.x / den, num.y / den, num.z / den, num.w / den);
             *reinterpret_cast<float4*>(O + ((size_t)unit * G + h) * kD + 4 * qd) = r;
+            if (lse && qd == 0) lse[(size_t)unit * G + h] = den > 0.f ? M + log2f(den) : -INFINITY;
         }
         return;  // no remote access after the barrier: CTAs may leave in any order
     } else {
@@ -642,6 +644,7 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
             float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
             if (den > 0.f) r = make_float4(num.x / den, num.y / den, num.z / den, num.w / den);
             *reinterpret_cast<float4*>(O + ((size_t)unit * G + h) * kD + 4 * qd) = r;
+            if (lse && qd == 0) lse[(size_t)unit * G + h] = den > 0.f ? M + log2f(den) : -INFINITY;
         }
         if (tid == 0) counters[unit] = 0u;  // ready for the next launch on this workspace
     }
@@ -766,6 +769,7 @@ struct AttnArgs {
     int early;
     float* sout;
     float scale;
+    float* lse;
 };
 
 template <int G, int STAGES, bool CLUSTER, bool CONTIG, bool ONE = false>
@@ -785,7 +789,7 @@ static cudaError_t attn_launch_g(dim3 grid, cudaStream_t st, const AttnArgs& a) 
     cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, attn_kernel<G, STAGES, CLUSTER, CONTIG, ONE>, a.kmap, a.vmap, a.q, a.k, a.v, a.lens,
                               a.idx, a.kreq, a.k_max, a.block, a.Hkv, a.Ncap, a.sl2, a.splits, a.partials, a.counters,
-                              a.O, a.flag, a.early, a.sout, a.scale);
+                              a.O, a.flag, a.early, a.sout, a.scale, a.lse);
 }
 
 template <int G, int STAGES, bool CLUSTER, bool CONTIG, bool ONE = false>
@@ -858,7 +862,7 @@ cudaError_t launch_attn(const void* Q, const void* K, const void* V, const int32
                         const int32_t* idx, const int32_t* kreq, int k_max, int block,
                         const Dims& d, float scale, int splits, float* partials,
                         unsigned* counters, float* O, unsigned* flag, cudaStream_t st, bool early,
-                        float* scores_out, bool host_kv) {
+                        float* scores_out, bool host_kv, float* lse_out) {
     if (d.units() == 0) return cudaSuccess;
     // scores come with full attention on the tensor-map path only
     if (scores_out && (idx != nullptr || host_kv)) return cudaErrorInvalidValue;
@@ -917,6 +921,7 @@ cudaError_t launch_attn(const void* Q, const void* K, const void* V, const int32
     a.early = early ? 1 : 0;
     a.sout = scores_out;
     a.scale = scale;
+    a.lse = lse_out;
     dim3 grid(splits, d.units());
     switch (d.G) {
         case 1: e = attn_dispatch<1>(contig, one_tile, cluster, grid, st, a); break;

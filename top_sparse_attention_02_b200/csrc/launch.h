@@ -38,6 +38,20 @@ void set_error_message(const char* msg);
 cudaError_t launch_index_overlap(const int32_t* idx, int L, int units, int k_max, int32_t* counts, double* M,
                                  unsigned* flag, cudaStream_t st);
 
+// sequence-sharded decode (shard.cu)
+constexpr int kMaxShards = 64;
+cudaError_t launch_shard_pack(const float* scores, int rows_cap, int units, int k_max, int row0, int32_t* cand_rows,
+                              float* cand_scores, unsigned* flag, cudaStream_t st);
+cudaError_t launch_merge_pack(const float* cand_scores, const int32_t* cand_rows, int R, int units, int Hkv,
+                              int k_max, float* pk_scores, int32_t* pk_rows, int32_t* n_cand, unsigned* flag,
+                              cudaStream_t st);
+cudaError_t launch_merge_map(const int32_t* pos, const int32_t* pk_rows, int units, int width, int k_max,
+                             int32_t* idx, cudaStream_t st);
+cudaError_t launch_localize(const int32_t* idx, int units, int k_max, int row0, int rows_cap, int32_t* local,
+                            cudaStream_t st);
+cudaError_t launch_shard_combine(const float* O_parts, const float* lse_parts, int R, int heads, float* O,
+                                 cudaStream_t st);
+
 cudaError_t launch_block_summarize(const void* K, const int32_t* lens, const Dims& d, int block,
                                    float* Kmean, unsigned* flag, cudaStream_t st);
 
@@ -84,7 +98,8 @@ cudaError_t launch_attn(const void* Q, const void* K, const void* V, const int32
                         unsigned* counters, float* O, unsigned* flag, cudaStream_t st,
                         bool early = false,  // early: lens, k's and Q not written by the previous kernel
                         float* scores_out = nullptr,  // full attention: each row's group-max scaled score
-                        bool host_kv = false);        // K, V in mapped page-locked host memory: gather only  // full attention only: [units][Ncap] scores of the valid rows
+                        bool host_kv = false,         // K, V in mapped page-locked host memory: gather only
+                        float* lse_out = nullptr);    // [units*G]: base-2 log-sum-exp of each head's scaled logits  // full attention only: [units][Ncap] scores of the valid rows
 
 cudaError_t launch_copy(const void* src, void* dst, size_t bytes, cudaStream_t st);
 cudaError_t launch_gather(const void* base, size_t base_bytes, const int32_t* rows, int nrows, unsigned* flag,
