@@ -83,8 +83,11 @@ typedef struct {
 /* ------------------------------------------------------------------ sizing */
 
 /* Bytes of workspace that tsa_decode_step needs for (shape, k_max, block, mode);
- * enough for every other entry point called with the same arguments.  Returns 0
- * on invalid arguments (see tsa_last_error_string). */
+ * enough for every other entry point called with the same arguments.  Layers of
+ * different modes may share one workspace sized with the largest of their
+ * sizes: every layout keeps the regions that must stay zero between calls (the
+ * top-digit histograms, the split counters) at the same offsets.  Returns 0 on
+ * invalid arguments (see tsa_last_error_string). */
 size_t tsa_workspace_size(tsa_shape shape, int32_t k_max, int32_t block, int32_t mode);
 
 /* Zero a workspace (enqueued memset).  Call once after allocating it. */
