@@ -120,10 +120,15 @@ class OracleShardOps:
         O.copy_(torch.where(den.unsqueeze(-1) > 0, num / den.clamp_min(1e-300).unsqueeze(-1), torch.zeros_like(num)))
 
 
-SHARD_CASE = dict(B=2, Hq=8, Hkv=2, N=3000, lens=[3000, 1100], kreq=[90, 90], bounds=[0, 1300, 3000])
+SHARD_CASES = {
+    # the second sequence lies wholly in rank 0's part
+    "two": dict(B=2, Hq=8, Hkv=2, N=3000, lens=[3000, 1100], kreq=[90, 90], bounds=[0, 1300, 3000]),
+    # three ranks, the middle one narrow; k above a sequence's length; g = 4
+    "three": dict(B=2, Hq=16, Hkv=4, N=2000, lens=[2000, 700], kreq=[60, 900], bounds=[0, 650, 720, 2000]),
+}
 
 
-def _shard_rank_main(rank, world, port, q):
+def _shard_rank_main(rank, world, port, q, name):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
     import datetime
     import sys
@@ -133,7 +138,7 @@ def _shard_rank_main(rank, world, port, q):
         sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
         from top_sparse_attention_02_b200 import inputs, shard
 
-        c = SHARD_CASE
+        c = SHARD_CASES[name]
         L = inputs.decode_layer(c["B"], c["Hq"], c["Hkv"], c["N"], c["lens"], plant_frac=0.01, seed=41)
         lo, hi = c["bounds"][rank], c["bounds"][rank + 1]
         K_r, V_r = L.K[:, :, lo:hi].contiguous(), L.V[:, :, lo:hi].contiguous()
@@ -149,10 +154,11 @@ def _shard_rank_main(rank, world, port, q):
         dist.destroy_process_group()
 
 
-def test_sequence_sharded_step_exchange_over_two_ranks():
-    """Two ranks, each holding a contiguous part of every sequence's rows (the
-    second sequence lies wholly in rank 0's part): after the candidate and the
-    partial exchanges both ranks hold the unsharded top-k and attention."""
+@pytest.mark.parametrize("name", sorted(SHARD_CASES))
+def test_sequence_sharded_step_exchange(name):
+    """Ranks each holding a contiguous part of every sequence's rows: after the
+    candidate and the partial exchanges every rank holds the unsharded top-k and
+    attention."""
     import sys
 
     import numpy as np
@@ -165,14 +171,15 @@ def test_sequence_sharded_step_exchange_over_two_ranks():
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_shard_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    c = SHARD_CASES[name]
+    world = len(c["bounds"]) - 1
+    procs = [ctx.Process(target=_shard_rank_main, args=(r, world, port, q, name)) for r in range(world)]
     for p in procs:
         p.start()
-    got = sorted((q.get(timeout=300) for _ in range(2)), key=lambda x: x[0])
+    got = sorted((q.get(timeout=300) for _ in range(world)), key=lambda x: x[0])
     for p in procs:
         p.join(timeout=120)
         assert p.exitcode == 0
-    c = SHARD_CASE
     L = inputs.decode_layer(c["B"], c["Hq"], c["Hkv"], c["N"], c["lens"], plant_frac=0.01, seed=41)
     S = oracle.scores(L.Q, L.K, L.seq_lens, 1 / 128 ** 0.5)
     k_max = max(c["kreq"])
@@ -180,4 +187,5 @@ def test_sequence_sharded_step_exchange_over_two_ranks():
         compare_idx(idx, S, c["lens"], c["kreq"])
         ref = oracle.attn(L.Q, L.K, L.V, L.seq_lens, idx, c["kreq"], k_max, 1, 1 / 128 ** 0.5)
         check_output(O, ref, f"rank {rank}")
-    assert np.array_equal(got[0][1], got[1][1]) and np.array_equal(got[0][2], got[1][2])
+    for _, idx, O in got[1:]:
+        assert np.array_equal(got[0][1], idx) and np.array_equal(got[0][2], O)
