@@ -24,6 +24,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -142,7 +143,9 @@ class Clocks:
         except Exception:
             self.idx = str(gpu_index)
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_dev{gpu_index}.csv")
+        # the raw samples; TSA_CLOCKS_CSV keeps them where the caller wants them
+        self.path = os.environ.get("TSA_CLOCKS_CSV") or os.path.join(tempfile.gettempdir(),
+                                                                     f"tsa_clocks_dev{gpu_index}_{os.getpid()}.csv")
 
     def __enter__(self):
         try:
