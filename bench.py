@@ -697,9 +697,10 @@ def run_reference(args, w_name, rank, world):
     }
 
 
-def cpu_baseline(w_name, budget_s=20.0):
+def cpu_baseline(w_name, budget_s=20.0, single_core_s=8.0):
     """The oracle, as it stands, on a bounded sample of the workload: whole layers of
-    the step until about budget_s of host time; scaled to the metric's unit."""
+    the step until about budget_s of host time on all host cores, then again until
+    about single_core_s on one core; scaled to the metric's unit."""
     import oracle
     from top_sparse_attention_02_b200 import workloads
 
@@ -707,27 +708,40 @@ def cpu_baseline(w_name, budget_s=20.0):
     lens = workload_lens(w)
     plan = Plan(w, lens)
     layers = make_layers(w, "cpu", lens)
-    t0 = time.perf_counter()
-    done_bytes, nlayers, idx = 0, 0, {}
-    while True:
-        for li, L in enumerate(layers):
-            m = w.route[li]
-            if m == 2:
-                oracle.decode_step(L.Q, L.K, L.V, L.seq_lens, plan.kreq, plan.k_max, w.scale, mode=2,
-                                   block=w.block, idx_in=idx[w.reuse_from[li]])
-            else:
-                _, ix, _ = oracle.decode_step(L.Q, L.K, L.V, L.seq_lens, plan.kreq, plan.k_max,
-                                              w.scale, mode=m, block=w.block)
-                idx[li] = ix
-            done_bytes += plan.layer_bytes[li]
-            nlayers += 1
-        if time.perf_counter() - t0 > budget_s:
-            break
-    s = time.perf_counter() - t0
-    return {"value": done_bytes / s / 1e12, "unit": "TB/s", "cores": oracle.num_threads(),
-            "kind": "oracle", "seconds": s,
-            "sample": f"{nlayers} layers = {nlayers // w.layers} whole step(s) of the workload "
-                      "(every unit), fp64 C oracle, OpenMP over (seq, kv-head) units"}
+
+    def run(budget):
+        t0 = time.perf_counter()
+        done_bytes, nlayers, idx = 0, 0, {}
+        while True:
+            for li, L in enumerate(layers):
+                m = w.route[li]
+                if m == 2:
+                    oracle.decode_step(L.Q, L.K, L.V, L.seq_lens, plan.kreq, plan.k_max, w.scale, mode=2,
+                                       block=w.block, idx_in=idx[w.reuse_from[li]])
+                else:
+                    _, ix, _ = oracle.decode_step(L.Q, L.K, L.V, L.seq_lens, plan.kreq, plan.k_max,
+                                                  w.scale, mode=m, block=w.block)
+                    idx[li] = ix
+                done_bytes += plan.layer_bytes[li]
+                nlayers += 1
+            if time.perf_counter() - t0 > budget:
+                break
+        return done_bytes, nlayers, time.perf_counter() - t0
+
+    cores = oracle.num_threads()
+    done_bytes, nlayers, s = run(budget_s)
+    res = {"value": done_bytes / s / 1e12, "unit": "TB/s", "cores": cores, "kind": "oracle", "seconds": s,
+           "sample": f"{nlayers} layers = {nlayers // w.layers} whole step(s) of the workload "
+                     "(every unit), fp64 C oracle, OpenMP over (seq, kv-head) units"}
+    if single_core_s > 0:
+        oracle.set_threads(1)
+        try:
+            b1, n1, s1 = run(single_core_s)
+        finally:
+            oracle.set_threads(cores)
+        res["single_core"] = {"value": b1 / s1 / 1e12, "unit": "TB/s", "cores": 1, "seconds": s1,
+                              "sample": f"{n1} layers = {n1 // w.layers} whole step(s), one thread"}
+    return res
 
 
 # ---------------------------------------------------------------- distributed plumbing
