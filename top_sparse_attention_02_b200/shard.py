@@ -44,7 +44,7 @@ def sharded_select_step(Q, K_shard, V_shard, shard_lens, k_per_seq, k_max: int, 
     with shard_lens[b] = clamp(len_b - row0, 0, Ncap_r).  Writes the global
     top-k into idx [B, Hkv, k_max] and the attention output into O [B, Hq, d]
     (the same on every rank).  ws: ``ops.shard_workspace_size`` bytes.  stream: a
-    torch.cuda.Stream (the all-gathers run on it too) or None (the default stream)."""
+    torch.cuda.Stream (the all-gathers run on it too) or None (torch's current stream)."""
     B, Hq, d = Q.shape
     Hkv = K_shard.shape[1]
     dev = Q.device
