@@ -94,6 +94,16 @@ class Plan:
                                    for n, kb in zip(self.lens, self.kb))
 
 
+def config_of(w, plan, world):
+    """The workload as both arms report it (the same dict, so that the two lines
+    can be compared key by key)."""
+    kv_bytes = w.layers * w.B * w.Hkv * w.Ncap * w.d * 2 * 2
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.Ncap, "k": plan.k_max,
+            "layers": w.layers, "route": "".join("FSR"[m] for m in w.route), "block": w.block,
+            "parallelism": f"replicas x{world}",
+            "l2": "inputs larger than L2 (%.2f GB of K/V per step)" % (kv_bytes / 1e9)}
+
+
 def make_layers(w, dev, lens):
     from top_sparse_attention_02_b200 import inputs
 
@@ -217,15 +227,23 @@ def run_ours(args, rank, world, dev):
             Kmean.append(km)
         else:
             Kmean.append(None)
-    step_args = []
-    for li, L in enumerate(layers):
-        mode = w.route[li]
-        src = w.reuse_from[li]
-        step_args.append(tsa.step_args(
-            L.Q, L.K, L.V, L.seq_lens, O[li], ws, mode=mode, scale=w.scale, k_max=plan.k_max,
-            block=w.block, k_per_seq=kreq_t, Kmean=Kmean[li],
-            idx_in=idx[src] if mode == tsa.REUSE else None,
-            idx_out=idx[li] if mode == tsa.SELECT else None))
+    # Every layer's lengths, k's, K, V and reused indices were written before the
+    # step (or by a layer at least two launches back), so each layer may read them
+    # before the kernel just before it has finished (TSA_EARLY_INPUTS); Q, the
+    # workspace and O are still touched only after it.
+    def make_step_args(flags):
+        out = []
+        for li, L in enumerate(layers):
+            mode = w.route[li]
+            src = w.reuse_from[li]
+            out.append(tsa.step_args(
+                L.Q, L.K, L.V, L.seq_lens, O[li], ws, mode=mode, scale=w.scale, k_max=plan.k_max,
+                block=w.block, k_per_seq=kreq_t, Kmean=Kmean[li],
+                idx_in=idx[src] if mode == tsa.REUSE else None,
+                idx_out=idx[li] if mode == tsa.SELECT else None, flags=flags))
+        return out
+
+    step_args = make_step_args(tsa.EARLY_INPUTS)
     # The step is captured once into a CUDA graph (the library never allocates or
     # synchronises, so its calls capture cleanly) and replayed: the timing is
     # device time, not Python/ctypes launch overhead.
@@ -269,6 +287,25 @@ def run_ours(args, rank, world, dev):
     tsa.check_device_status(ws, stream)
     del graph
 
+    # the same step with every kernel waiting for its predecessor before its
+    # first read (no TSA_EARLY_INPUTS), for comparison
+    plain_args = make_step_args(0)
+    g2 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g2, stream=stream):
+        for a in plain_args:
+            tsa.decode_step(a, stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            g2.replay()
+        e0.record(stream)
+        for _ in range(args.steps):
+            g2.replay()
+        e1.record(stream)
+    stream.synchronize()
+    ms_plain = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+    tsa.check_device_status(ws, stream)
+    del g2
+
     # per-stage device times: each stage alone, repeated in its own graph
     stages = stage_times(tsa, w, plan, layers, Kmean, ws, kreq_t, idx, O, stream)
     copy_gbs = copy_probe(tsa, dev, stream)
@@ -283,13 +320,10 @@ def run_ours(args, rank, world, dev):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "us_per_step": ms * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16 Q/K/V, resident in HBM)",
-        "config": {"workload": w.name, "B": B, "Hq": Hq, "Hkv": Hkv, "N": w.Ncap,
-                   "k": plan.k_max, "layers": w.layers,
-                   "route": "".join("FSR"[m] for m in w.route), "block": w.block,
-                   "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2 (%.2f GB of K/V per step)" %
-                         (sum(L.K.numel() + L.V.numel() for L in layers) * 2 / 1e9)},
+        "config": config_of(w, plan, world),
         "algorithmic_bytes_per_step": plan.step_bytes,
+        "step_flags": "TSA_EARLY_INPUTS on every layer (its inputs are not written by the kernel before it)",
+        "ms_per_step_without_early_inputs": ms_plain,
         "tokens_attended_per_s": world * plan.tokens_attended * w.layers / (ms * 1e-3),
         "stages_us": stages,
         "roofline": {"kernel": "score_tc_kernel (layer-0 K scan)", "bound": "hbm",
@@ -304,7 +338,7 @@ def run_ours(args, rank, world, dev):
         "timing": "CUDA graph of one whole step, replayed K times between CUDA events",
     }
     if not args.no_e2e:
-        res["e2e"] = e2e_measure(tsa, w, plan, layers, step_args, O, idx, stream, args)
+        res["e2e"] = e2e_measure(tsa, w, plan, layers, step_args, O, idx, ws, kreq_t, stream, args)
     if args.offload:
         res["offload"] = offload_probe(tsa, w, plan, layers, Kmean, ws, kreq_t, idx, O, stream)
     if args.probes:
@@ -611,39 +645,75 @@ def attn_roofline(w, plan, stages, gather):
             "algorithmic_bytes_per_launch": plan.bytes["gather"]}
 
 
-def e2e_measure(tsa, w, plan, layers, step_args, O, idx, stream, args):
-    """The same step through the C ABI, with every input copied from pinned host memory
-    and the outputs (O of every layer, the selected indices) copied back, all inside the
-    timed region."""
-    host_in = [[t.cpu().pin_memory() for t in (L.Q, L.K, L.V, L.seq_lens)] for L in layers]
-    dev_in = [(L.Q, L.K, L.V, L.seq_lens) for L in layers]
+def e2e_measure(tsa, w, plan, layers, step_args, O, idx, ws, kreq_t, stream, args):
+    """The same step through the C ABI from host buffers, inside the timed region:
+    - every layer's Q and lengths are copied host -> device from pinned memory;
+    - a layer that scans its cache (SELECT in token mode, FULL) gets its K and V
+      copied host -> device (the scorer reads every K row);
+    - a REUSE layer leaves its K and V in pinned host memory and reads only the
+      selected rows across the host link (TSA_KV_HOST, index-guided offload);
+    - every layer's O and the selected indices are copied back.
+    h2d_bytes_per_step counts the copies plus the rows the reuse layers read
+    through the mapping."""
+    from top_sparse_attention_02_b200 import binding as _b
+
+    offload = [m == tsa.REUSE for m in w.route]
+    host_in, dev_in, hkv = [], [], []
+    for li, L in enumerate(layers):
+        if offload[li]:
+            host_in.append([L.Q.cpu().pin_memory(), L.seq_lens.cpu().pin_memory()])
+            dev_in.append((L.Q, L.seq_lens))
+            hkv.append((L.K.cpu().pin_memory(), L.V.cpu().pin_memory()))
+        else:
+            host_in.append([t.cpu().pin_memory() for t in (L.Q, L.K, L.V, L.seq_lens)])
+            dev_in.append((L.Q, L.K, L.V, L.seq_lens))
+            hkv.append(None)
+    e2e_args = []
+    for li, (a, L) in enumerate(zip(step_args, layers)):
+        if not offload[li]:
+            e2e_args.append(a)
+            continue
+        Kh, Vh = hkv[li]
+        e2e_args.append(_b.step_args(L.Q, Kh, Vh, L.seq_lens, O[li], ws, mode=tsa.REUSE, scale=w.scale,
+                                     k_max=plan.k_max, block=w.block, k_per_seq=kreq_t,
+                                     idx_in=idx[w.reuse_from[li]], flags=tsa.KV_HOST))
     O_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in O]
     sel = [li for li, m in enumerate(w.route) if m == tsa.SELECT]
     idx_host = [torch.empty(idx[li].shape, dtype=torch.int32).pin_memory() for li in sel]
-    h2d = sum(t.numel() * t.element_size() for hs in host_in for t in hs)
+    copied = sum(t.numel() * t.element_size() for hs in host_in for t in hs)
+    mapped = sum(1 for m in offload if m) * plan.bytes["gather"]
     d2h = sum(t.numel() * t.element_size() for t in O_host + idx_host)
     reps = max(1, min(args.steps, 5))
+
+    def one():
+        for hs, ds in zip(host_in, dev_in):
+            for h, d in zip(hs, ds):
+                d.copy_(h, non_blocking=True)
+        for a in e2e_args:
+            tsa.decode_step(a, stream)
+        for oh, od in zip(O_host, O):
+            oh.copy_(od, non_blocking=True)
+        for ih, li in zip(idx_host, sel):
+            ih.copy_(idx[li], non_blocking=True)
+
+    with torch.cuda.stream(stream):  # one untimed pass: the host pointer checks, first touches
+        one()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):  # copies and kernels in one stream order
         e0.record(stream)
         for _ in range(reps):
-            for hs, ds in zip(host_in, dev_in):
-                for h, d in zip(hs, ds):
-                    d.copy_(h, non_blocking=True)
-            for a in step_args:
-                tsa.decode_step(a, stream)
-            for oh, od in zip(O_host, O):
-                oh.copy_(od, non_blocking=True)
-            for ih, li in zip(idx_host, sel):
-                ih.copy_(idx[li], non_blocking=True)
+            one()
         e1.record(stream)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / reps
+    del hkv
     return {"value": plan.step_bytes / (ms * 1e-3) / 1e12, "unit": "TB/s", "ms_per_step": ms,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": reps,
-            "note": "Q, K, V and lengths of every layer copied host->device from pinned memory, "
-                    "O and indices copied back, inside the timed region"}
+            "h2d_bytes_per_step": copied + mapped, "d2h_bytes_per_step": d2h, "steps": reps,
+            "h2d_copied_bytes_per_step": copied, "h2d_mapped_read_bytes_per_step": mapped,
+            "note": "from pinned host buffers each step: Q and lengths of every layer and K, V of the scanning "
+                    "layers copied host->device; reuse layers read only their selected K/V rows from pinned "
+                    "host memory (TSA_KV_HOST); O and indices copied back; all inside the timed region"}
 
 
 # ---------------------------------------------------------------- reference arm (oracle on CPU)
@@ -689,8 +759,7 @@ def run_reference(args, w_name, rank, world):
         "steps": n, "warmup": args.warmup, "ms_per_step": s * 1e3, "us_per_step": s * 1e6,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1) bf16 Q/K/V)",
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.Ncap,
-                   "k": plan.k_max, "layers": w.layers, "parallelism": "host cores (OpenMP)"},
+        "config": config_of(w, plan, world),
         "cpu_baseline": {"value": val, "unit": "TB/s", "cores": cores, "kind": "oracle",
                          "sample": f"{n} whole step(s) of the workload (all layers, all units)"},
         "e2e": {"value": val, "unit": "TB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -759,7 +828,7 @@ def max_over_ranks(x, world, dev):
         return x
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    t = torch.tensor([x], dtype=torch.float64, device=dev)  # dev: the rank's GPU (NCCL) or "cpu" (gloo)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -767,6 +836,43 @@ def max_over_ranks(x, world, dev):
 def whole_job_value(step_bytes: int, ms: float, world: int) -> float:
     """TB/s of the whole job: every rank runs its own replica of the workload."""
     return world * step_bytes / (ms * 1e-3) / 1e12
+
+
+def launch_ranks(n, argv):
+    """Start this script as n ranks on this node (torch.distributed.run, one
+    process per GPU, rendezvous on 127.0.0.1), bounded by an outer timeout."""
+    import socket
+
+    with socket.socket() as so:
+        so.bind(("127.0.0.1", 0))
+        port = so.getsockname()[1]
+    cmd = ["timeout", "-k", "60", "3600", sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={n}", "--master-addr=127.0.0.1", f"--master-port={port}",
+           os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
+
+
+def dry_run(args, rank, world):
+    """The multi-rank plumbing alone, on the CPU (gloo, no CUDA): every rank takes
+    a stand-in time, the max goes over the ranks, rank 0 prints the line."""
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    try:
+        barrier(world)
+        ms = max_over_ranks(1.0 + 0.25 * rank, world, "cpu")
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "value": whole_job_value(10 ** 9, ms, world), "unit": "TB/s",
+                              "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                              "dry_run": True}), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
 
 
 def main():
@@ -785,11 +891,22 @@ def main():
                     help="block-mode workloads: also time a layer whose K/V sit in pinned host memory")
     ap.add_argument("--ncap", type=int, default=0,
                     help="shrink the workload's context to this many tokens (profiler captures only)")
+    ap.add_argument("--dry-run", action="store_true",
+                    help="only the rank plumbing (start, barrier, max over ranks) on the CPU over gloo")
     args = ap.parse_args()
 
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        # not started as a rank: start --gpus ranks of this same command
+        sys.exit(launch_ranks(args.gpus, sys.argv[1:]))
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+        sys.exit(2)
+    if args.dry_run:
+        dry_run(args, rank, world)
+        return
 
     if args.impl == "reference":
         if rank != 0:

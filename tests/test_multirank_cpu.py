@@ -189,3 +189,35 @@ def test_sequence_sharded_step_exchange(name):
         check_output(O, ref, f"rank {rank}")
     for _, idx, O in got[1:]:
         assert np.array_equal(got[0][1], idx) and np.array_equal(got[0][2], O)
+
+
+def test_bench_gpus_n_starts_n_ranks():
+    """`bench.py --gpus 2` started by hand (no WORLD_SIZE) starts two ranks of
+    itself; they rendezvous, take the slower rank's time and rank 0 alone prints
+    one line with n_gpus = 2 (the rank plumbing only, on the CPU over gloo)."""
+    import json
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2", "--dry-run",
+                          "--steps", "1", "--warmup", "0"], capture_output=True, text=True, timeout=300,
+                         env=env, cwd=root)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, out.stdout
+    res = json.loads(lines[0])
+    assert res["n_gpus"] == 2 and res["dry_run"]
+    assert res["ms_per_step"] == 1.25  # rank 1's stand-in time, the slower one
+
+
+def test_bench_refuses_a_world_size_that_disagrees_with_gpus():
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, WORLD_SIZE="3", RANK="0", LOCAL_RANK="0")
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2", "--dry-run"],
+                         capture_output=True, text=True, timeout=120, env=env, cwd=root)
+    assert out.returncode != 0 and "WORLD_SIZE=3" in out.stderr
