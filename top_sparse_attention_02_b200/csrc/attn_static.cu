@@ -11,7 +11,6 @@
 // `ws`.  It calls no cudaMalloc, cudaFree or allocating library routine.
 #include <cmath>
 #include <cstdio>
-#include <mutex>
 
 #include "common.cuh"
 #include "launch.h"
@@ -24,11 +23,8 @@ constexpr size_t kFlagBytes = 256;
 
 // File-scope device scratch.  In host code this name is only a stand-in for the
 // device array, never a device address: the address comes from
-// cudaGetSymbolAddress, once per device, below.
+// cudaGetSymbolAddress, on every call, with the calling device current.
 static __device__ __align__(256) unsigned char g_attn_scratch[kScratchBytes];
-
-std::mutex g_mu;
-void* g_scratch_ptr[64] = {};  // per device ordinal, set on the first call on that device
 
 tsa_status bad(tsa_status st, const char* msg) {
     tsa::set_error_message(msg);  // read back with tsa_last_error_string()
@@ -77,25 +73,16 @@ tsa_status sparse_decode_attn_noalloc(const void* Q, const void* K, const void* 
         return bad(TSA_ERR_WORKSPACE, msg);
     }
 
-    // ---- set-up, once per device, with that device current
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return bad(TSA_ERR_CUDA, "sparse_decode_attn_noalloc: cudaGetDevice failed");
-    if (dev < 0 || dev >= 64) return bad(TSA_ERR_UNSUPPORTED, "sparse_decode_attn_noalloc: device ordinal above 63");
+    // ---- the array's device address on the current device.  Looked up on
+    // every call (it allocates nothing and is cheap), so that it is never stale:
+    // after cudaDeviceReset, or with another primary context, the library's
+    // module is loaded again and the array may sit elsewhere.  The first call
+    // on a device loads the module (with lazy loading) and so commits the array.
     void* base = nullptr;
-    {
-        std::lock_guard<std::mutex> lock(g_mu);
-        if (g_scratch_ptr[dev] == nullptr) {
-            void* p = nullptr;
-            e = cudaGetSymbolAddress(&p, g_attn_scratch);
-            if (e != cudaSuccess || p == nullptr) {
-                snprintf(msg, sizeof msg, "sparse_decode_attn_noalloc: cudaGetSymbolAddress: %s",
-                         cudaGetErrorString(e));
-                return bad(TSA_ERR_CUDA, msg);
-            }
-            g_scratch_ptr[dev] = p;
-        }
-        base = g_scratch_ptr[dev];
+    cudaError_t e = cudaGetSymbolAddress(&base, g_attn_scratch);
+    if (e != cudaSuccess || base == nullptr) {
+        snprintf(msg, sizeof msg, "sparse_decode_attn_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+        return bad(TSA_ERR_CUDA, msg);
     }
     char* s = static_cast<char*>(base);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
