@@ -45,6 +45,14 @@ def test_library_exports_every_declared_symbol(tsa):
     for name in declared_functions():
         assert name in exported, f"{name} declared in tsa.h but not exported"
         assert getattr(tsa.lib(), name) is not None
+    # the test-only knobs exist in libtsa_debug.so alone
+    assert not any("debug" in n for n in exported), "the product library exports a debug knob"
+    dbg = os.path.join(ROOT, "top_sparse_attention_02_b200", "libtsa_debug.so")
+    if os.path.exists(dbg):
+        out = subprocess.run(["nm", "-D", "--defined-only", dbg], capture_output=True, text=True,
+                             check=True).stdout
+        names = {line.split()[-1] for line in out.splitlines() if line.strip()}
+        assert "tsa_debug_skip_tile" in names and set(declared_functions()) <= names
 
 
 def _shape(tsa, B=1, Hq=8, Hkv=2, N=4096, d=128):

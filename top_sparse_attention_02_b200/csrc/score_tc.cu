@@ -27,7 +27,16 @@
 //           digit, counted here where the ALUs idle behind HBM).
 // Q is written once per CTA into shared memory in the same swizzled K-major
 // layout (the B operand).  Every mbarrier wait is bounded: on expiry the kernel
-// raises the device timeout flag and moves on; TMEM is always freed.
+// raises the device timeout flag and each role stops; before the CTA leaves,
+// the producer waits (bounded) for the tile loads it issued and the MMA issuer
+// for the MMAs it issued, so that nothing lands in shared memory or TMEM after
+// TMEM is freed and the CTA is gone.  The scores are then unspecified.
+//
+// With `early` (the caller's promise that the kernel before this one on the
+// stream writes neither the lengths nor K), the first two K tiles are requested
+// before waiting on that kernel (programmatic dependent launch), so the scan's
+// first loads overlap its end; Q, the scores and the histogram are touched only
+// after the wait.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -46,7 +55,17 @@ constexpr int kTcQHalfBytes = kTcN * 128;             // 16 rows x 128 B = 2 KB
 constexpr int kTcTilesPerCta = 32;                    // 4096 rows per CTA (the 128K scan: 256 CTAs, one wave)
 constexpr int kTcSms = 148;
 constexpr int kTcSmem = 1024 /*align slack*/ + kTcStages * kTcStageBytes + 2 * kTcQHalfBytes;
+#ifndef TSA_WAIT_SPINS
 constexpr long kTcSpins = 1L << 22;
+#else
+constexpr long kTcSpins = TSA_WAIT_SPINS;  // a debug build's short limit
+#endif
+
+#ifdef TSA_DEBUG_KNOBS
+// Debug build only (never in the product library): the tile (of CTA (0, 0))
+// whose load the producer leaves out, so that the waits on it run out; -1: none.
+__device__ int g_debug_skip_tile = -1;
+#endif
 // instruction descriptor: D f32 (bits 4-5 = 1), A bf16 (7-9 = 1), B bf16 (10-12 = 1),
 // both K-major (bits 15, 16 = 0), N >> 3 at bits 17-22, M >> 4 at bits 24-28
 constexpr uint32_t kTcIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kTcN >> 3) << 17) |
@@ -72,7 +91,8 @@ __device__ __forceinline__ void tc_arrive_tx(unsigned bar, unsigned bytes) {
                  "r"(bytes)
                  : "memory");
 }
-// bounded wait for the phase of the given parity; false = gave up (flag raised)
+// bounded wait for the phase of the given parity; false = gave up (flag raised,
+// unless flag is NULL: a drain wait at the end)
 __device__ __forceinline__ bool tc_wait(unsigned bar, unsigned parity, unsigned* flag) {
     for (long i = 0; i < kTcSpins; ++i) {
         unsigned done;
@@ -83,7 +103,7 @@ __device__ __forceinline__ bool tc_wait(unsigned bar, unsigned parity, unsigned*
             : "memory");
         if (done) return true;
     }
-    atomicOr(flag, kFlagTimeout);
+    if (flag) atomicOr(flag, kFlagTimeout);
     return false;
 }
 
@@ -92,7 +112,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
 score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16* __restrict__ Q,
                 const int32_t* __restrict__ lens, int Hkv, int Ncap, float scale,
                 float* __restrict__ scores, uint32_t* __restrict__ hist, int tiles_per_cta,
-                unsigned* __restrict__ flag) {
+                unsigned* __restrict__ flag, int early) {
     extern __shared__ unsigned char tc_smem_raw[];
     __shared__ __align__(8) uint64_t s_full[kTcStages], s_empty[kTcStages], s_tfull[2], s_tempty[2];
     __shared__ uint32_t s_tmem;
@@ -101,8 +121,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16* _
     const int unit = blockIdx.y;
     const int b = unit / Hkv;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    griddep_wait();
-    int len = lens[b];
+    if (!early) griddep_wait();
+    int len = early ? __ldcg(lens + b) : lens[b];
     if (len < 0 || len > Ncap) {
         if (tid == 0 && blockIdx.x == 0) atomicOr(flag, kFlagBounds);
         len = len < 0 ? 0 : Ncap;
@@ -139,6 +159,38 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16* _
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
     }
+    // ---- the producer's tile loads (warp 0, lane 0)
+    const int row_base = unit * Ncap;
+    // K is read once: evict it from L2 first, so the scores (kept with
+    // evict_last below) are still there when the top-k reads them
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(pol));
+    auto issue = [&](int i) {
+        const int s = i % kTcStages;
+        const unsigned full = su32(&s_full[s]);
+#ifdef TSA_DEBUG_KNOBS
+        if (i == g_debug_skip_tile && blockIdx.x == 0 && unit == 0) return;  // neither armed nor loaded
+#endif
+        tc_arrive_tx(full, kTcStageBytes);
+        const int y = row_base + (t0 + i) * kTcTileRows;
+        const unsigned dst = base + s * kTcStageBytes;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            asm volatile(
+                "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;\n" ::"r"(
+                    dst + half * kTcHalfBytes),
+                "l"(&kmap), "r"(half * 64), "r"(y), "r"(full), "l"(pol)
+                : "memory");
+        }
+    };
+    int issued = 0;  // warp 0, lane 0: tiles requested so far
+    if (early) {
+        // the first stages' loads before waiting on the previous kernel
+        __syncthreads();  // the barriers are initialised
+        if (warp == 0 && lane == 0)
+            for (; issued < nt && issued < kTcStages; ++issued) issue(issued);
+        griddep_wait();
+    }
     if (warp >= 2) {  // Q rows n < G (bf16 as stored), rows G..15 zero; 16-byte chunks swizzled
         const int t = tid - 64;  // 0..127: (row n, 16-byte chunk c of the 256-byte row)
         const int n = t >> 3, c16 = t & 7;
@@ -159,32 +211,21 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16* _
     if (warp == 0) {
         // ---- TMA producer
         if (lane == 0) {
-            const int row_base = unit * Ncap;
-            // K is read once: evict it from L2 first, so the scores (kept with
-            // evict_last below) are still there when the top-k reads them
-            uint64_t pol;
-            asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(pol));
-            for (int i = 0; i < nt; ++i) {
-                const int s = i % kTcStages;
+            for (; issued < nt; ++issued) {
+                const int i = issued, s = i % kTcStages;
                 if (i >= kTcStages && !tc_wait(su32(&s_empty[s]), (unsigned)((i / kTcStages) - 1) & 1u, flag)) break;
-                const unsigned full = su32(&s_full[s]);
-                tc_arrive_tx(full, kTcStageBytes);
-                const int y = row_base + (t0 + i) * kTcTileRows;
-                const unsigned dst = base + s * kTcStageBytes;
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    asm volatile(
-                        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;\n" ::"r"(
-                            dst + half * kTcHalfBytes),
-                        "l"(&kmap), "r"(half * 64), "r"(y), "r"(full), "l"(pol)
-                        : "memory");
-                }
+                issue(i);
             }
+            // the last load of each stage has landed (at once, unless a wait
+            // gave up): none may land after the CTA has gone
+            for (int j = max(0, issued - kTcStages); j < issued; ++j)
+                tc_wait(su32(&s_full[j % kTcStages]), (unsigned)(j / kTcStages) & 1u, nullptr);
         }
         __syncwarp();
     } else if (warp == 1) {
         // ---- MMA issuer
         if (lane == 0) {
+            int done = 0;  // tiles whose MMAs were issued
             for (int i = 0; i < nt; ++i) {
                 const int s = i % kTcStages, bsel = i & 1;
                 if (!tc_wait(su32(&s_full[s]), (unsigned)(i / kTcStages) & 1u, flag)) break;
@@ -210,6 +251,13 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16* _
                 asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
                                  su32(&s_tfull[bsel]))
                              : "memory");
+                done = i + 1;
+            }
+            // the last MMAs issued have completed (their commit freed the ring
+            // stage) before TMEM is freed below
+            if (done > 0) {
+                const int j = done - 1;
+                tc_wait(su32(&s_empty[j % kTcStages]), (unsigned)(j / kTcStages) & 1u, nullptr);
             }
         }
         __syncwarp();
@@ -221,7 +269,10 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16* _
         asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;\n" : "=l"(keep));
         for (int i = 0; i < nt; ++i) {
             const int bsel = i & 1;
-            const bool ok = tc_wait(su32(&s_tfull[bsel]), (unsigned)(i >> 1) & 1u, flag);
+            // every lane waits itself; the warp goes on only if all saw the
+            // accumulator (tcgen05.ld below is warp-collective), else it stops
+            const bool ok = __all_sync(0xffffffffu, tc_wait(su32(&s_tfull[bsel]), (unsigned)(i >> 1) & 1u, flag));
+            if (!ok) break;
             asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
             uint32_t r[16];
             const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(bsel * kTcN);
@@ -239,7 +290,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16* _
             for (int h = 1; h < G; ++h) m = fmaxf(m, __uint_as_float(r[h]));
             const int row = (t0 + i) * kTcTileRows + q * 32 + lane;
             // scale > 0, so scale * max_h(z_h) = max_h(scale * z_h) exactly (rounding is monotone)
-            if (ok && row < len) {
+            if (row < len) {
                 const float v = m * scale;
                 asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;\n" ::"l"(out + row), "f"(v), "l"(keep)
                              : "memory");
@@ -282,7 +333,7 @@ static cudaError_t get_encode() {
 static int g_tc_configured[64];
 
 cudaError_t launch_score_tc(const void* Q, const void* K, const int32_t* lens, const Dims& d, float scale,
-                            float* scores, uint32_t* hist, unsigned* flag, cudaStream_t st) {
+                            float* scores, uint32_t* hist, unsigned* flag, cudaStream_t st, bool early) {
     if (d.units() == 0 || d.Ncap == 0) return cudaSuccess;
     cudaError_t e = get_encode();
     if (e != cudaSuccess) return e;
@@ -324,10 +375,10 @@ cudaError_t launch_score_tc(const void* Q, const void* K, const int32_t* lens, c
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     switch (d.G) {
-        case 1: e = cudaLaunchKernelEx(&cfg, score_tc_kernel<1>, map, q, lens, d.Hkv, d.Ncap, scale, scores, hist, per, flag); break;
-        case 2: e = cudaLaunchKernelEx(&cfg, score_tc_kernel<2>, map, q, lens, d.Hkv, d.Ncap, scale, scores, hist, per, flag); break;
-        case 4: e = cudaLaunchKernelEx(&cfg, score_tc_kernel<4>, map, q, lens, d.Hkv, d.Ncap, scale, scores, hist, per, flag); break;
-        case 8: e = cudaLaunchKernelEx(&cfg, score_tc_kernel<8>, map, q, lens, d.Hkv, d.Ncap, scale, scores, hist, per, flag); break;
+        case 1: e = cudaLaunchKernelEx(&cfg, score_tc_kernel<1>, map, q, lens, d.Hkv, d.Ncap, scale, scores, hist, per, flag, early ? 1 : 0); break;
+        case 2: e = cudaLaunchKernelEx(&cfg, score_tc_kernel<2>, map, q, lens, d.Hkv, d.Ncap, scale, scores, hist, per, flag, early ? 1 : 0); break;
+        case 4: e = cudaLaunchKernelEx(&cfg, score_tc_kernel<4>, map, q, lens, d.Hkv, d.Ncap, scale, scores, hist, per, flag, early ? 1 : 0); break;
+        case 8: e = cudaLaunchKernelEx(&cfg, score_tc_kernel<8>, map, q, lens, d.Hkv, d.Ncap, scale, scores, hist, per, flag, early ? 1 : 0); break;
         default: return cudaErrorInvalidValue;
     }
     note_launch();
@@ -336,3 +387,14 @@ cudaError_t launch_score_tc(const void* Q, const void* K, const int32_t* lens, c
 }
 
 }  // namespace tsa
+
+#ifdef TSA_DEBUG_KNOBS
+// Debug build only: which tile's load the scorer (0) or the attention's
+// contiguous-tile path (1) leaves out in CTA (0, 0); -1 for none.  Returns a
+// cudaError_t.
+extern "C" int tsa_debug_attn_skip_tile(int tile);
+extern "C" int tsa_debug_skip_tile(int which, int tile) {
+    if (which == 1) return tsa_debug_attn_skip_tile(tile);
+    return (int)cudaMemcpyToSymbol(tsa::g_debug_skip_tile, &tile, sizeof tile);
+}
+#endif
