@@ -143,19 +143,24 @@ tsa_status sparse_decode_attn(const void* Q, const void* K, const void* V,
  * 8 MiB device array inside the library, which every GPU that loads the library
  * holds until the process exits.  It allocates nothing (no cudaMalloc, cudaFree
  * or allocating library routine).
- *  - The first call on a device looks up that array's device address (with that
- *    device current) and caches it; later calls reuse it.
+ *  - Every call looks up that array's device address on the current device.
+ *    The first call on a device loads the library's device code there (with
+ *    CUDA's lazy module loading), which commits the array and may block: make
+ *    it during warm-up, before any stream capture.
  *  - Every call clears the counters it needs, then launches: all calls share the
  *    one array, so calls that overlap on the GPU (different streams, or other
  *    host threads, on the same device) race and must be ordered by the caller.
  *  - A shape whose scratch exceeds 8 MiB returns TSA_ERR_WORKSPACE with the
  *    bytes it needs (use sparse_decode_attn with a workspace instead).  The
- *    array holds about 16000 split partials of 520 bytes (one per unit, split
- *    and query head); the 128K-token shape (8 units, 74 splits, 4 heads) uses
- *    1.2 MB of it.
- *  - Device-detected range errors skip the offending rows as in
- *    sparse_decode_attn, but are not reported: the flag lives in the shared
- *    array and is cleared by the next call. */
+ *    array holds about 15,880 split partials of (d + 4) * 4 = 528 bytes (one
+ *    per unit, split and query head); the 128K-token shape (8 units, 8 splits,
+ *    4 heads) uses 135 KB of it.
+ *  - Nothing the device detects is reported: the device flag lives in the
+ *    shared array and the next call clears it.  Range errors skip the offending
+ *    rows, as in sparse_decode_attn; a bounded wait that gives up (contiguous
+ *    128-row tiles: idx == NULL, or block == 128) leaves O unspecified, and that
+ *    goes unreported too.  A caller that must know uses sparse_decode_attn and
+ *    tsa_check_device_status. */
 tsa_status sparse_decode_attn_noalloc(const void* Q, const void* K, const void* V,
                                       const int32_t* seq_lens, const int32_t* idx,
                                       const int32_t* k_per_seq, int32_t k_max, int32_t block,
@@ -181,7 +186,7 @@ typedef struct {
     float* O;                 /* [B, Hq, d] fp32 */
     void* ws;                 /* workspace */
     size_t ws_bytes;
-    uint32_t flags;           /* 0, or TSA_KV_HOST */
+    uint32_t flags;           /* 0, or TSA_KV_HOST and/or TSA_EARLY_INPUTS */
 } tsa_step_args;
 
 /* tsa_step_args.flags: K and V live in page-locked host memory that the device
@@ -196,6 +201,20 @@ typedef struct {
  * TSA_FULL layer reads all of K and V across the link.  A K or V pointer that is
  * not such memory returns TSA_ERR_INVALID_ARG (pageable memory would fault). */
 #define TSA_KV_HOST 1u
+
+/* tsa_step_args.flags: the caller's promise that the kernel enqueued on
+ * `stream` just before this step (the end of the previous layer, say) writes
+ * none of seq_lens, k_per_seq, K, V and (TSA_REUSE) idx_in: they were written
+ * two or more launches earlier, or are constant for the step.  The step's first
+ * kernel may then read them before that kernel has finished (programmatic
+ * dependent launch): a TSA_REUSE or TSA_FULL layer reads its index list and
+ * issues the loads of its first K/V tiles, and a TSA_SELECT layer's scorer
+ * requests its first K tiles, while the previous kernel runs.  Q, the
+ * workspace, idx_out and O are still touched only after it has finished, so Q
+ * may come from the kernel just before.  Breaking the promise gives results
+ * computed from stale inputs (no fault).  Without the flag every kernel waits
+ * for its predecessor before its first read. */
+#define TSA_EARLY_INPUTS 2u
 
 /* One decode step of one layer: TSA_SELECT = score -> top-k -> attention;
  * TSA_REUSE = attention over idx_in; TSA_FULL = attention over every valid row.

@@ -41,6 +41,7 @@ class tsa_step_args(ctypes.Structure):
 
 
 KV_HOST = 1  # tsa_step_args.flags: K and V in mapped page-locked host memory
+EARLY_INPUTS = 2  # tsa_step_args.flags: the kernel before the step writes none of lens, k's, K, V, idx_in
 
 
 _vp, _sz, _i32, _f32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_float

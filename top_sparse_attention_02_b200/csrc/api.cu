@@ -325,7 +325,7 @@ tsa_status tsa_shard_attend(const void* Q, const void* K_shard, const void* V_sh
     if (e != cudaSuccess) return cuda_fail(e, "tsa_shard_attend (local rows)");
     e = tsa::launch_attn(Q, K_shard, V_shard, shard_lens, local, k_per_seq, k_max, 1, d, scale, L.splits,
                          reinterpret_cast<float*>(w + L.partials), reinterpret_cast<unsigned*>(w + L.counters), O_part,
-                         flag_of(ws), st, false, nullptr, false, lse_part);
+                         flag_of(ws), st, 0, nullptr, false, lse_part);
     if (e != cudaSuccess) return cuda_fail(e, "tsa_shard_attend (attention)");
     return TSA_OK;
 }
@@ -402,7 +402,7 @@ tsa_status check_host_kv(const void* K, const void* V) {
 
 tsa_status attn_stage(const void* Q, const void* K, const void* V, const int32_t* seq_lens, const int32_t* idx,
                       const int32_t* k_per_seq, int32_t k_max, int32_t block, tsa_shape shape, float scale, float* O,
-                      void* ws, size_t ws_bytes, void* stream, bool host_kv);
+                      void* ws, size_t ws_bytes, void* stream, bool host_kv, int early);
 
 }  // namespace
 
@@ -412,14 +412,14 @@ tsa_status sparse_decode_attn(const void* Q, const void* K, const void* V,
                               tsa_shape shape, float scale, float* O, void* ws, size_t ws_bytes,
                               void* stream) {
     return attn_stage(Q, K, V, seq_lens, idx, k_per_seq, k_max, block, shape, scale, O, ws, ws_bytes, stream,
-                      false);
+                      false, 0);
 }
 
 namespace {
 
 tsa_status attn_stage(const void* Q, const void* K, const void* V, const int32_t* seq_lens, const int32_t* idx,
                       const int32_t* k_per_seq, int32_t k_max, int32_t block, tsa_shape shape, float scale, float* O,
-                      void* ws, size_t ws_bytes, void* stream, bool host_kv) {
+                      void* ws, size_t ws_bytes, void* stream, bool host_kv, int early) {
     tsa::Dims d;
     TSA_TRY(check_shape(shape, &d));
     TSA_TRY(check_block(block));
@@ -437,7 +437,7 @@ tsa_status attn_stage(const void* Q, const void* K, const void* V, const int32_t
     cudaError_t e = tsa::launch_attn(Q, K, V, seq_lens, idx, k_per_seq, k_max, dense ? 1 : block, d,
                                      scale, L.splits, reinterpret_cast<float*>(w + L.partials),
                                      reinterpret_cast<unsigned*>(w + L.counters), O, flag_of(ws),
-                                     static_cast<cudaStream_t>(stream), false, nullptr, host_kv);
+                                     static_cast<cudaStream_t>(stream), early, nullptr, host_kv);
     if (e != cudaSuccess) return cuda_fail(e, "sparse_decode_attn");
     return TSA_OK;
 }
@@ -448,9 +448,12 @@ tsa_status tsa_decode_step(const tsa_step_args* a, void* stream) {
     if (!a) return fail(TSA_ERR_INVALID_ARG, "tsa_decode_step: NULL args");
     tsa::Dims d;
     TSA_TRY(check_shape(a->shape, &d));
-    if (a->flags & ~(uint32_t)TSA_KV_HOST)
+    if (a->flags & ~(uint32_t)(TSA_KV_HOST | TSA_EARLY_INPUTS))
         return fail(TSA_ERR_INVALID_ARG, "tsa_decode_step: unknown flags 0x%x", a->flags);
     const bool host_kv = (a->flags & TSA_KV_HOST) != 0;
+    // the caller's promise (TSA_EARLY_INPUTS): the first kernel of the step may
+    // read lens, k's, K, V and idx_in before the kernel before it has finished
+    const bool early_in = (a->flags & TSA_EARLY_INPUTS) != 0;
     if (host_kv && a->block == 1 && (a->mode == TSA_SELECT || (a->mode == TSA_FULL && a->idx_out)))
         return fail(TSA_ERR_UNSUPPORTED,
                     "tsa_decode_step: with TSA_KV_HOST a layer that selects must score block means (block > 1); "
@@ -459,7 +462,7 @@ tsa_status tsa_decode_step(const tsa_step_args* a, void* stream) {
         case TSA_FULL: {
             if (!a->idx_out)
                 return attn_stage(a->Q, a->K, a->V, a->seq_lens, nullptr, nullptr, 0, 1, a->shape, a->scale, a->O,
-                                  a->ws, a->ws_bytes, stream, host_kv);
+                                  a->ws, a->ws_bytes, stream, host_kv, early_in ? 2 : 0);
             // A full layer that also hands its top-k on (HyLRA: a sensitive layer's
             // extracted indices pass to the tolerant layers after it).  Token mode:
             // the full attention writes each row's score as it forms S (no second
@@ -490,7 +493,7 @@ tsa_status tsa_decode_step(const tsa_step_args* a, void* stream) {
             cudaError_t e;
             if (a->block == 1) {
                 e = tsa::launch_attn(a->Q, a->K, a->V, a->seq_lens, nullptr, nullptr, 0, 1, d, a->scale, L.splits,
-                                     partials, counters, a->O, flag_of(a->ws), st, false, scores);
+                                     partials, counters, a->O, flag_of(a->ws), st, early_in ? 2 : 0, scores);
                 if (e != cudaSuccess) return cuda_fail(e, "tsa_decode_step (full attention)");
                 e = tsa::launch_topk(scores, a->seq_lens, a->k_per_seq, a->k_max, d, 1, a->idx_out, nullptr,
                                      flag_of(a->ws), st);
@@ -506,14 +509,14 @@ tsa_status tsa_decode_step(const tsa_step_args* a, void* stream) {
                 return cuda_fail(e, "tsa_decode_step (top-k)");
             }
             e = tsa::launch_attn(a->Q, a->K, a->V, a->seq_lens, nullptr, nullptr, 0, 1, d, a->scale, L.splits,
-                                 partials, counters, a->O, flag_of(a->ws), st, false, nullptr, host_kv);
+                                 partials, counters, a->O, flag_of(a->ws), st, 0, nullptr, host_kv);
             if (e != cudaSuccess) return cuda_fail(e, "tsa_decode_step (full attention)");
             return TSA_OK;
         }
         case TSA_REUSE:
             if (!a->idx_in) return fail(TSA_ERR_INVALID_ARG, "tsa_decode_step: TSA_REUSE needs idx_in");
             return attn_stage(a->Q, a->K, a->V, a->seq_lens, a->idx_in, a->k_per_seq, a->k_max, a->block, a->shape,
-                              a->scale, a->O, a->ws, a->ws_bytes, stream, host_kv);
+                              a->scale, a->O, a->ws, a->ws_bytes, stream, host_kv, early_in ? 2 : 0);
         case TSA_SELECT: {
             TSA_TRY(check_block(a->block));
             TSA_TRY(check_scale(a->scale));
@@ -540,7 +543,7 @@ tsa_status tsa_decode_step(const tsa_step_args* a, void* stream) {
             const void* keys = a->block == 1 ? a->K : static_cast<const void*>(a->Kmean);
             cudaStream_t st = static_cast<cudaStream_t>(stream);
             cudaError_t e = tsa::launch_score(a->Q, keys, a->seq_lens, d, a->block, a->scale, scores, hist,
-                                              flag_of(a->ws), st);
+                                              flag_of(a->ws), st, early_in);
             if (e != cudaSuccess) return cuda_fail(e, "tsa_decode_step (score)");
             e = tsa::launch_topk(scores, a->seq_lens, a->k_per_seq, a->k_max, d, a->block, a->idx_out, hist,
                                  flag_of(a->ws), st);
@@ -553,7 +556,7 @@ tsa_status tsa_decode_step(const tsa_step_args* a, void* stream) {
             // indices: it may read the lengths, k's and Q before waiting on it
             e = tsa::launch_attn(a->Q, a->K, a->V, a->seq_lens, a->idx_out, a->k_per_seq, a->k_max, a->block, d,
                                  a->scale, L.splits, reinterpret_cast<float*>(w + L.partials),
-                                 reinterpret_cast<unsigned*>(w + L.counters), a->O, flag_of(a->ws), st, true,
+                                 reinterpret_cast<unsigned*>(w + L.counters), a->O, flag_of(a->ws), st, 1,
                                  nullptr, host_kv);
             if (e != cudaSuccess) return cuda_fail(e, "tsa_decode_step (attention)");
             return TSA_OK;

@@ -12,26 +12,34 @@
 // Design: grid = (split, unit); a CTA is 8 warps and owns a contiguous range of
 // the unit's index list, walked in tiles of 128 rows (16 per warp).  Two ways
 // of bringing a tile's K and V (256 B a row) into shared memory:
-//   - gather (an index list of tokens): each warp fetches its own 16 rows with
-//     16-byte vector loads (a half-warp per row) one tile ahead in registers,
-//     or, when the CTA's range is a single tile, with cp.async straight into
-//     shared memory (no registers held, so two CTAs fit an SM); rows are padded
-//     to 272 B so the fragment loads below are free of bank conflicts, and no
-//     barrier wider than a warp is needed per tile.  (One TMA bulk copy per
-//     256-byte row was the first design: issuing them cost ~13 ns a copy.)
+//   - gather (an index list of tokens): each warp fetches its own 16 rows of
+//     every tile with cp.async straight into shared memory, into a per-warp
+//     ring of up to 3 tiles, so that all of a CTA's tiles (3 at the 128K
+//     shape) are in flight at once; with one tile a CTA the ring is one stage
+//     and two CTAs fit an SM.  (K and V in mapped host memory are fetched with
+//     16-byte vector loads one tile ahead in registers instead.)  Rows are
+//     padded to 272 B so the fragment loads below are free of bank conflicts,
+//     and no barrier wider than a warp is needed per tile: a warp only ever
+//     reads the rows it copied.  (One TMA bulk copy per 256-byte row was the
+//     first design: issuing them cost ~13 ns a copy.)
 //   - contiguous tiles (full attention, or a 128-token block): four 2-D TMA
 //     tensor loads a tile in the 128-byte swizzle into a 3-stage ring, each
 //     stage completing on an mbarrier, refilled as soon as it is consumed.
 // Each warp then runs, on its
 // 16 rows, the two contractions of flash decoding on the tensor cores
-// (mma.sync m16n8k16, bf16 in, fp32 accumulate), with the g <= 8 query heads as
-// the M dimension padded to 16:
-//   S = Q K^T   (8 k-steps, K fragments by ldmatrix),
-//   online softmax per head on the S fragments (fp32, log2 units),
-//   O += P V    (P split as bf16 hi + bf16 lo so that the weights keep ~16
-//               bits; V fragments by ldmatrix.trans).
-// tcgen05's smallest M is 64, so there 87-94% of every MMA would be padding;
-// the m16 warp MMA fits a GQA group.  The 8 warps are merged at the end into
+// (mma.sync m16n8k16, bf16 in, fp32 accumulate), transposed so that the 16
+// rows are the M dimension and the g <= 8 query heads of the group the N
+// dimension (one n-tile of 8):
+//   S^T = K Q^T    (8 k-steps of 16 dims: 8 MMAs; K fragments by ldmatrix,
+//                  Q^T fragments held in registers for the whole kernel),
+//   online softmax per head on the S^T fragments (fp32, log2 units),
+//   O^T += V^T P^T (8 m-tiles of 16 dims: 16 MMAs with P split as bf16 hi +
+//                  bf16 lo so that the weights keep ~16 bits; V^T fragments by
+//                  ldmatrix.trans, P^T fragments from the S^T accumulator by
+//                  movmatrix.trans).
+// With the heads as M instead (padded to 16), each 16 rows took twice the
+// MMAs and twice the accumulator registers.  tcgen05's smallest M is 64, so
+// a GQA group would leave most of every tcgen05 MMA idle.  The 8 warps are merged at the end into
 // the CTA's partial (M, L, acc[128]) per head.  When a unit has at most 8
 // splits and every unit's cluster can be resident at once, the splits of a unit
 // form one thread-block cluster: each CTA pushes the slices of its partial to
@@ -41,6 +49,16 @@
 // only 15 clusters of 8 CTAs of ~226 KB) each CTA writes its partial to the
 // workspace and the last CTA of the unit to arrive (an atomic counter in the
 // workspace, reset by that CTA) combines the partials into O.
+//
+// Programmatic dependent launch: the kernel may start while the kernel before
+// it on the stream is still running.  It waits for it (griddepcontrol.wait)
+// before the first read of anything that kernel may have written.  How much it
+// does before that wait is the `early` level: 0 nothing; 1 the lengths and k's
+// (the decode step's own top-k writes only the indices); 2 also the index list
+// and the first tiles' K and V rows (the caller has promised that the kernel
+// just before does not write them), so that a reuse layer's gather overlaps the
+// end of the layer before it.  Q, the workspace and O are touched only after
+// the wait.
 #include <cooperative_groups.h>
 #include <cstring>
 #include <cuda.h>
@@ -54,27 +72,47 @@ namespace cg = cooperative_groups;
 namespace tsa {
 
 constexpr int kMaxSplits = 256;
-constexpr int kClusterMax = 8;  // splits per unit that combine inside one (portable) cluster
+constexpr int kClusterMax = 16;     // splits per unit that combine inside one cluster (16: non-portable)
+constexpr int kPortableCluster = 8; // the largest cluster size every GPU supports
 constexpr int kSms = 148;
 constexpr int kPartStride = kD + 4;  // M, L, 2 pad, acc[128]: 528 B, 16-byte aligned
 constexpr int kAttnThreads = 256;
+constexpr int kAccStride = kD + 4;  // floats per (warp, head) row of the merge buffer: 16-byte rows, no bank conflicts
 constexpr int kAttnWarps = 8;
 constexpr int kTileRows = 128;                         // 16 rows per warp
 constexpr int kRowStride = kD * 2 + 16;                // 272 B: padded so 8 rows hit 8 bank groups
 constexpr int kStageBytes = kTileRows * kRowStride * 2;  // K and V of one tile: 68 KB
+// cp.async gather: one warp's 16 rows of one tile (K rows, then V rows) form a
+// slot; slot (t % STAGES) * 8 + warp holds warp `warp`'s rows of tile t, so a
+// CTA whose range is n warp-tiles (16 rows each) uses only slots 0 .. n - 1
+// (no ring wrap) and its shared memory is sized by n at launch
+constexpr int kSlotBytes = 16 * kRowStride * 2;  // 8.5 KB
 constexpr int kRing = 3;                               // tiles in flight (the multi-tile kernel)
-constexpr long kWaitSpins = 1L << 22;                  // bounded mbarrier wait (then flag + go on)
+#ifndef TSA_WAIT_SPINS
+constexpr long kWaitSpins = 1L << 22;  // bounded mbarrier wait (then flag, drain and stop)
+#else
+constexpr long kWaitSpins = TSA_WAIT_SPINS;  // a debug build's short limit
+#endif
+#ifdef TSA_DEBUG_KNOBS
+// Debug build only (never in the product library): the contiguous tile (of CTA
+// (0, 0)) whose loads are left out, so that the wait on it runs out; -1: none.
+__device__ int g_debug_attn_skip_tile = -1;
+#endif
 
 template <int G>
 struct AttnCfg {
-    static constexpr int kPer = G * 16;  // output float4 slots per CTA when S >= 2
-    static constexpr int kRecvBytes = kClusterMax * kPer * 16;
-    static constexpr int kAccBytes = kAttnWarps * G * kD * 4;
+    // cluster combine: S sources x ceil(G*32/S) float4 output slots per owner
+    static constexpr int kRecvBytes = (G * 32 + kClusterMax) * 16;
+    static constexpr int kAccBytes = kAttnWarps * G * kAccStride * 4;
     static constexpr int work_bytes(int stages) {
         return stages * kStageBytes > kAccBytes ? stages * kStageBytes : kAccBytes;
     }
     static constexpr int smem_bytes(int stages, bool cluster) {
         return 1024 /* alignment slack */ + work_bytes(stages) + (cluster ? kRecvBytes : 0);
+    }
+    // the cp.async gather with `slots` warp-tile slots in use
+    static constexpr int slot_work_bytes(int slots) {
+        return slots * kSlotBytes > kAccBytes ? slots * kSlotBytes : kAccBytes;
     }
 };
 
@@ -90,16 +128,18 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, unsigned by
                  ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
 // Wait for the phase with the given parity; gives up after kWaitSpins polls,
-// raising the timeout flag (the copies are still bounded: they read valid rows).
-__device__ __forceinline__ void mbar_wait(uint64_t* bar, unsigned parity, unsigned* flag) {
+// raising the timeout flag, and returns false (the CTA then stops its tile loop;
+// see the contiguous-tile loop).  flag == nullptr: no flag (a drain wait).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity, unsigned* flag) {
     const unsigned a = smem_u32(bar);
     for (long i = 0; i < kWaitSpins; ++i) {
         unsigned done;
         asm volatile("{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
                      : "=r"(done) : "r"(a), "r"(parity) : "memory");
-        if (done) return;
+        if (done) return true;
     }
-    atomicOr(flag, kFlagTimeout);
+    if (flag) atomicOr(flag, kFlagTimeout);
+    return false;
 }
 // 1-D bulk copy (TMA engine) global -> this CTA's shared memory, completing on `bar`
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned bytes, uint64_t* bar) {
@@ -115,15 +155,22 @@ __device__ __forceinline__ void ldsm_x4_t(unsigned addr, uint32_t& r0, uint32_t&
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];\n"
                  : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
 }
-// D += A * B, m16n8k16, bf16 inputs, fp32 accumulate.  Only the rows of A that
-// carry query heads (a0/a1 and a4/a5: row lane/4) are non-zero here, so the
-// rows lane/4 + 8 of A are passed as zero.
-__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
+// D += A * B, m16n8k16, bf16 inputs, fp32 accumulate (A row-major 16x16 in
+// a0..a3, B column-major 16x8 in b0, b1; the PTX ISA's fragment layouts).
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
     asm volatile(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
         "{%0, %1, %2, %3};\n"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// transpose of an 8x8 b16 matrix held one row pair per lane (lane/4 = row,
+// lane%4 = column pair) into the same layout
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t a) {
+    uint32_t d;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(d) : "r"(a));
+    return d;
 }
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -136,25 +183,27 @@ __device__ __forceinline__ int roff(int row, int chunk) { return row * kRowStrid
 // one 128-token block in block mode) and arrives by 2-D TMA tensor loads in the
 // 128-byte-swizzled layout (4 loads per tile); otherwise each row is its own
 // 256-byte bulk copy into rows padded to 272 bytes.
-// ONE (gather only): every CTA's range is one tile; rows are copied straight into
-// shared memory (cp.async) instead of through registers, so two CTAs fit an SM.
-template <int G, int STAGES, bool CLUSTER, bool CONTIG, bool ONE>
-__global__ void __launch_bounds__(kAttnThreads, ONE ? 2 : 1)
+// ASYNC (gather only): rows are copied straight into shared memory (cp.async)
+// into a per-warp ring of STAGES tiles; with STAGES == 1 (every CTA's range is
+// one tile) two CTAs fit an SM.  Otherwise (K and V in mapped host memory) each
+// warp loads its rows into registers one tile ahead and stores them.
+template <int G, int STAGES, bool CLUSTER, bool CONTIG, bool ASYNC>
+__global__ void __launch_bounds__(kAttnThreads, ASYNC ? 2 : 1)
 attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
             const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
             const __nv_bfloat16* __restrict__ V, const int32_t* __restrict__ lens,
             const int32_t* __restrict__ idx, const int32_t* __restrict__ kreq, int k_max,
             int block, int Hkv, int Ncap, float scale_log2, int S, float* __restrict__ part,
             unsigned* __restrict__ counters, float* __restrict__ O, unsigned* __restrict__ flag, int early,
-            float* __restrict__ sout, float scale, float* __restrict__ lse) {
+            float* __restrict__ sout, float scale, float* __restrict__ lse, int work) {
     using Cfg = AttnCfg<G>;
     extern __shared__ __align__(128) unsigned char smem_raw[];
     // 1024-byte aligned work area (the swizzled layout needs it)
     unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     __shared__ float s_wm[kAttnWarps][G], s_wl[kAttnWarps][G];
-    __shared__ float s_M[G], s_L[G];
     __shared__ float s_Mr[kClusterMax][G], s_Lr[kClusterMax][G];  // cluster path: received (M, L)
     __shared__ int s_last;
+    __shared__ int s_fail;  // CONTIG: a bounded wait gave up; the CTA stops its tile loop
     __shared__ __align__(8) uint64_t s_bar[STAGES];
     __shared__ int s_first[STAGES];  // CONTIG: first cache row of the tile in each stage, or -1
 
@@ -162,15 +211,42 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
     const int b = unit / Hkv;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t4 = lane & 3;  // mma fragment coordinates
-    // early: the kernel before this one did not write the lengths, the k's or Q
-    // (the decode step's own top-k), so they are read before waiting on it
+    // early >= 1: the kernel before this one did not write the lengths or the
+    // k's (the decode step's own top-k), so they are read before waiting on it;
+    // early == 2: neither the index list nor K and V (the caller's promise), so
+    // the first tiles are fetched before the wait too (below)
     int len = 0, kreq_b = k_max;
     if (early) {
-        len = lens[b];
-        if (kreq) kreq_b = kreq[b];
+        len = __ldcg(lens + b);
+        if (kreq) kreq_b = __ldcg(kreq + b);
     }
-    griddep_wait();
-    griddep_launch();
+    if (early < 2) {
+        griddep_wait();
+        griddep_launch();
+    }
+    // Gather: the index entries of this lane's rows (lanes 0-15: rows r0 +
+    // lane) in the first ring stages, loaded at once for the range this split
+    // has when every unit attends to k_max entries -- before the lengths and
+    // k's have arrived.  Checked against the real range below (the same range
+    // unless k_b < k_max), and loaded again where it differs.
+    constexpr int NEV = CONTIG ? 1 : (ASYNC ? STAGES : 1);
+    const int32_t* iu = idx ? idx + (size_t)unit * k_max : nullptr;
+    const int r0 = warp * 16;  // this warp's rows in a tile
+    int ev[NEV];
+    int spec_p0 = -1;
+    if constexpr (!CONTIG) {
+        if (iu != nullptr) {
+            const int npos_s = k_max * block;
+            const int chunk_s = ceil_div(npos_s, S);
+            spec_p0 = min(s * chunk_s, npos_s);
+            const int spec_p1 = min(spec_p0 + chunk_s, npos_s);
+#pragma unroll
+            for (int i = 0; i < NEV; ++i) {
+                const int pos = spec_p0 + i * kTileRows + r0 + lane;
+                ev[i] = (lane < 16 && pos < spec_p1) ? __ldcg(iu + (block == 1 ? pos : pos / block)) : -1;
+            }
+        }
+    }
     if (!early) {
         len = lens[b];
         if (kreq) kreq_b = kreq[b];
@@ -194,23 +270,20 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
     const int chunk = CONTIG ? ceil_div(ceil_div(npos, S), kTileRows) * kTileRows : ceil_div(npos, S);
     const int p0 = min(s * chunk, npos), p1 = min(p0 + chunk, npos);
     const int ntiles = ceil_div(p1 - p0, kTileRows);
-    const int32_t* iu = idx ? idx + (size_t)unit * k_max : nullptr;
     const __nv_bfloat16* Ku = K + (size_t)unit * Ncap * kD;
     const __nv_bfloat16* Vu = V + (size_t)unit * Ncap * kD;
 
-    // cache row of position pos, or -1 (skipped entry, tail of a partial block)
-    auto row_of = [&](int pos) -> int {
-        if (iu == nullptr) return pos;
+    // cache row of position pos given its index entry e (token mode: the row;
+    // block mode: the block), or -1 (skipped entry, tail of a partial block)
+    auto row_check = [&](int pos, int e) -> int {
         if (block == 1) {
-            const int r = iu[pos];
-            if (r >= len) {
+            if (e >= len) {
                 atomicOr(flag, kFlagBounds);
                 return -1;
             }
-            return r < 0 ? -1 : r;
+            return e < 0 ? -1 : e;
         }
         const int slot = pos / block;
-        const int e = iu[slot];
         if (e >= nb) {
             atomicOr(flag, kFlagBounds);
             return -1;
@@ -219,13 +292,17 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
         const int r = e * block + (pos - slot * block);
         return r < len ? r : -1;
     };
+    auto row_of = [&](int pos) -> int {
+        if (iu == nullptr) return pos;
+        return row_check(pos, __ldcg(iu + (block == 1 ? pos : pos / block)));
+    };
     // CONTIG: the tile's first cache row (dense: its position; block mode: the
     // chosen block's first row), or -1 when the block entry is absent
     auto tile_first = [&](int t) -> int {
         const int pos0 = p0 + t * kTileRows;
         if (t >= ntiles) return -1;
         if (iu == nullptr) return pos0;
-        const int e = iu[pos0 / kTileRows];
+        const int e = __ldcg(iu + pos0 / kTileRows);
         if (e >= nb) {
             atomicOr(flag, kFlagBounds);
             return -1;
@@ -238,6 +315,9 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
         if (t >= ntiles) return;
         const int st = t % STAGES;
         s_first[st] = first;
+#ifdef TSA_DEBUG_KNOBS
+        if (t == g_debug_attn_skip_tile && blockIdx.x == 0 && blockIdx.y == 0) return;  // neither armed nor loaded
+#endif
         if (first >= 0) {
             fence_proxy_async();
             mbar_arrive_expect_tx(&s_bar[st], 4 * 64 * kTileRows * 2);
@@ -262,6 +342,7 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
         }
     };
     if (tid == 0) {
+        s_fail = 0;
 #pragma unroll
         for (int i = 0; i < STAGES; ++i) mbar_init(&s_bar[i], CONTIG ? 1 : kTileRows);
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
@@ -269,8 +350,10 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
     __syncthreads();
     // CONTIG: the first STAGES tiles' block indices in one round, then their loads
     int next_first = -1;  // CONTIG, thread 0: first row of the tile that refills the stage next
+    int issued = 0;       // CONTIG, thread 0: tiles whose loads have been issued
     if constexpr (CONTIG) {
         if (tid == 0) {
+            issued = min(ntiles, STAGES);
             int f[STAGES];
 #pragma unroll
             for (int t = 0; t < STAGES; ++t) f[t] = tile_first(t);
@@ -279,42 +362,64 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
         }
     }
 
-    const int r0 = warp * 16;  // this warp's rows in a tile
-    // Gather: each warp fetches its own 16 rows of a tile with 16-byte vector
-    // loads (a half-warp per 256-byte row; lane l takes chunk l & 15 of rows
-    // (l >> 4), +2, ..., +14), one tile ahead in registers, and stores them
-    // into its rows of the padded tile: no TMA queue (one 256-byte bulk copy
-    // per row issued at ~13 ns a copy per SM, which bounded short gathers) and
-    // no CTA barrier per tile.  Rows not in the set are zeros (0 x NaN = NaN).
-    unsigned char* kw = smem + r0 * kRowStride;
-    unsigned char* vw = smem + (kTileRows + r0) * kRowStride;
+    // Gather: each warp copies its own 16 rows of a tile (a half-warp per
+    // 256-byte row; lane l takes 16-byte chunk l & 15 of rows (l >> 4), +2,
+    // ..., +14) into its rows of the padded tile, and only that warp reads
+    // them: no TMA queue (one 256-byte bulk copy per row issued at ~13 ns a
+    // copy per SM, which bounded short gathers) and no CTA barrier per tile.
+    // Rows not in the set are zeros (their weight is 0, and 0 x NaN = NaN).
     const int hl = lane >> 4, c16 = lane & 15;
-    uint4 pk[8], pv[8];
-    uint32_t vm_next = 0;
-    auto fetch = [&](int t) {
-        if constexpr (CONTIG) return;
+    // this lane's cache row of tile t (lanes 0-15: rows r0 + lane), or -1
+    auto my_row = [&](int t) -> int {
         int myrow = -1;
         if (lane < 16) {
             const int pos = p0 + t * kTileRows + r0 + lane;
             if (pos < p1) myrow = row_of(pos);
         }
-        vm_next = __ballot_sync(0xffffffffu, myrow >= 0) & 0xffffu;
+        return myrow;
+    };
+    // the rows of the first NEV tiles: their index entries all in flight at
+    // once (the speculative loads above where the range agrees)
+    int rows0[NEV];
+    if constexpr (!CONTIG) {
+        const bool spec = iu != nullptr && p0 == spec_p0;
+        int e[NEV];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int rr = __shfl_sync(0xffffffffu, myrow, hl + 2 * j);
-            pk[j] = rr >= 0 ? ld_stream(Ku + (size_t)rr * kD + 8 * c16) : make_uint4(0, 0, 0, 0);
-            pv[j] = rr >= 0 ? ld_stream(Vu + (size_t)rr * kD + 8 * c16) : make_uint4(0, 0, 0, 0);
+        for (int i = 0; i < NEV; ++i) {
+            const int pos = p0 + i * kTileRows + r0 + lane;
+            e[i] = -1;
+            if (iu != nullptr && lane < 16 && pos < p1) e[i] = spec ? ev[i] : __ldcg(iu + (block == 1 ? pos : pos / block));
+        }
+#pragma unroll
+        for (int i = 0; i < NEV; ++i) {
+            const int pos = p0 + i * kTileRows + r0 + lane;
+            rows0[i] = -1;
+            if (lane < 16 && pos < p1) rows0[i] = iu != nullptr ? row_check(pos, e[i]) : pos;
+        }
+    }
+    // register path (K and V in host memory): tile t's rows into registers
+    uint4 pk[ASYNC ? 1 : 8], pv[ASYNC ? 1 : 8];
+    uint32_t vm_next = 0;
+    auto fetch = [&](int t, int myrow) {
+        if constexpr (!CONTIG && !ASYNC) {
+            vm_next = __ballot_sync(0xffffffffu, myrow >= 0) & 0xffffu;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int rr = __shfl_sync(0xffffffffu, myrow, hl + 2 * j);
+                pk[j] = rr >= 0 ? ld_stream(Ku + (size_t)rr * kD + 8 * c16) : make_uint4(0, 0, 0, 0);
+                pv[j] = rr >= 0 ? ld_stream(Vu + (size_t)rr * kD + 8 * c16) : make_uint4(0, 0, 0, 0);
+            }
         }
     };
-    // ONE: cp.async copies of tile t's rows of this warp (zeros for rows not in the set)
-    uint32_t vm_one = 0;
-    auto issue_one = [&](int t) {
-        int myrow = -1;
-        if (lane < 16) {
-            const int pos = p0 + t * kTileRows + r0 + lane;
-            if (pos < p1) myrow = row_of(pos);
-        }
-        vm_one = __ballot_sync(0xffffffffu, myrow >= 0) & 0xffffu;
+    // cp.async path: tile t's rows of this warp (this lane's: myrow) into its
+    // slot of ring stage st (not committed here); returns the tile's row mask.
+    // A warp with no position of the CTA's range in tile t writes nothing (its
+    // slot may lie past the shared memory a short range is given).
+    auto issue_async = [&](int t, int st, int myrow) -> uint32_t {
+        if (p0 + t * kTileRows + r0 >= p1) return 0u;  // warp-uniform
+        const uint32_t vm = __ballot_sync(0xffffffffu, myrow >= 0) & 0xffffu;
+        unsigned char* kw = smem + (st * kAttnWarps + warp) * kSlotBytes;
+        unsigned char* vw = kw + 16 * kRowStride;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int rr = __shfl_sync(0xffffffffu, myrow, hl + 2 * j);
@@ -330,17 +435,31 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
                 *reinterpret_cast<uint4*>(vd) = make_uint4(0, 0, 0, 0);
             }
         }
-        asm volatile("cp.async.commit_group;\n" ::: "memory");
+        return vm;
     };
+    // masks of the tiles in the ring, oldest first (a shift register, so it
+    // stays in registers)
+    uint32_t vmr[ASYNC ? STAGES : 1];
+#pragma unroll
+    for (int i = 0; i < (ASYNC ? STAGES : 1); ++i) vmr[i] = 0u;
     if constexpr (!CONTIG) {
-        if (ntiles > 0) {  // in flight while Q is read
-            if constexpr (ONE) issue_one(0);
-            else fetch(0);
+        if constexpr (ASYNC) {  // the whole ring in flight (empty groups past the last tile)
+#pragma unroll
+            for (int i = 0; i < STAGES; ++i) {
+                if (i < ntiles) vmr[i] = issue_async(i, i, rows0[i < NEV ? i : 0]);
+                asm volatile("cp.async.commit_group;\n" ::: "memory");
+            }
+        } else if (ntiles > 0) {
+            fetch(0, rows0[0]);
         }
     }
+    if (early >= 2) {  // everything above read only what the caller promised is not being written
+        griddep_wait();
+        griddep_launch();
+    }
 
-    // A fragments of Q (bf16, unscaled: the scale is applied to S in fp32).
-    // Row g of A = query head g of the group (zero for g >= G); rows g+8 are zero.
+    // B fragments of Q^T (bf16, unscaled: the scale is applied to S in fp32):
+    // column g = query head g of the group (zero for g >= G), rows = dims.
     uint32_t qa[8][2];
     {
         const uint32_t* qrow = reinterpret_cast<const uint32_t*>(Q + ((size_t)unit * G + (g < G ? g : 0)) * kD);
@@ -350,12 +469,14 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
             qa[ks][1] = g < G ? qrow[ks * 8 + 4 + t4] : 0u;   // dims 16ks + 8 + 2t4, +1
         }
     }
-    float o[16][4];  // O fragments: head g, dims 8n + 2t4 (+1); [2],[3] are padding rows
+    // O^T fragments: o[mt][0], [1] = dim 16mt + g, heads 2t4, 2t4 + 1; [2], [3] = dim 16mt + g + 8
+    float o[8][4];
 #pragma unroll
-    for (int n = 0; n < 16; ++n)
+    for (int n = 0; n < 8; ++n)
 #pragma unroll
         for (int e = 0; e < 4; ++e) o[n][e] = 0.f;
-    float m_run = -INFINITY, l_run = 0.f;  // this warp's running max / sum for head g
+    // this warp's running max / sum for heads 2t4 and 2t4 + 1 (equal across the lanes of a t4)
+    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
 
     const unsigned sbase = smem_u32(smem);
     // The two contractions of flash decoding on this warp's 16 rows of a tile
@@ -373,89 +494,104 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
             else
                 return (unsigned)roff(r, c);
         };
-        // ---- S = Q K^T over this warp's 16 rows (two n-tiles of 8 rows)
-        float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        // ---- S^T = K Q^T over this warp's 16 rows (M = rows, N = heads)
+        float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};  // even / odd k-steps: two chains
         {
             const int m = lane >> 3, i = lane & 7;  // ldmatrix: matrix m, row i
-            const int row = r0 + (m >> 1) * 8 + i;   // n-tile (m>>1), k-half (m&1)
+            const int row = r0 + (m & 1) * 8 + i;    // rows +8 (m&1), dims +8 (m>>1)
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
-                uint32_t b0, b1, b2, b3;
-                ldsm_x4(kt + off(row, 2 * ks + (m & 1)), b0, b1, b2, b3);
-                mma_bf16(sc[0], qa[ks][0], qa[ks][1], b0, b1);
-                mma_bf16(sc[1], qa[ks][0], qa[ks][1], b2, b3);
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4(kt + off(row, 2 * ks + (m >> 1)), a0, a1, a2, a3);
+                mma_bf16(sc[ks & 1], a0, a1, a2, a3, qa[ks][0], qa[ks][1]);
             }
         }
+        // c[0], c[1]: row g, heads 2t4, 2t4 + 1; c[2], c[3]: row g + 8
+        float c[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) c[e] = sc[0][e] + sc[1][e];
+        const int h0 = 2 * t4, h1 = 2 * t4 + 1;  // this lane's two heads
+        const bool va = (vm >> g) & 1u, vb = (vm >> (g + 8)) & 1u;  // rows g, g + 8 in the set
         if constexpr (CONTIG) {
-            if (su_out) {  // uniform: the max over heads g < G of each row's dot, by lanes of equal t4
-                float e[4] = {g < G ? sc[0][0] : -INFINITY, g < G ? sc[0][1] : -INFINITY,
-                              g < G ? sc[1][0] : -INFINITY, g < G ? sc[1][1] : -INFINITY};
+            if (su_out) {  // uniform: each row's max over the heads < G, across the 4 lanes of the row
+                float ea = fmaxf(h0 < G ? c[0] : -INFINITY, h1 < G ? c[1] : -INFINITY);
+                float eb = fmaxf(h0 < G ? c[2] : -INFINITY, h1 < G ? c[3] : -INFINITY);
 #pragma unroll
-                for (int o = 4; o < 32; o <<= 1)
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) e[q] = fmaxf(e[q], __shfl_xor_sync(0xffffffffu, e[q], o));
-                if (g == 0) {
-                    const int ia = 2 * t4;
-                    const int lrow[4] = {ia, ia + 1, ia + 8, ia + 9};
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)  // scale > 0: scale x max = max of the scaled logits
-                        if ((vm >> lrow[q]) & 1u) su_out[first + r0 + lrow[q]] = e[q] * scale;
+                for (int o2 = 1; o2 < 4; o2 <<= 1) {
+                    ea = fmaxf(ea, __shfl_xor_sync(0xffffffffu, ea, o2));
+                    eb = fmaxf(eb, __shfl_xor_sync(0xffffffffu, eb, o2));
+                }
+                if (t4 == 0) {  // scale > 0: scale x max = max of the scaled logits
+                    if (va) su_out[first + r0 + g] = ea * scale;
+                    if (vb) su_out[first + r0 + g + 8] = eb * scale;
                 }
             }
         }
-        // ---- online softmax for head g (columns = rows of the tile)
+        // ---- online softmax per head (columns of S^T): rows not in the set are -inf
         float z[4];
-        {
-            const int ia = 2 * t4;  // local rows of sc[0][0..1]; sc[1] adds 8
-            z[0] = (vm >> ia) & 1u ? sc[0][0] * scale_log2 : -INFINITY;
-            z[1] = (vm >> (ia + 1)) & 1u ? sc[0][1] * scale_log2 : -INFINITY;
-            z[2] = (vm >> (ia + 8)) & 1u ? sc[1][0] * scale_log2 : -INFINITY;
-            z[3] = (vm >> (ia + 9)) & 1u ? sc[1][1] * scale_log2 : -INFINITY;
+        z[0] = va ? c[0] * scale_log2 : -INFINITY;
+        z[1] = va ? c[1] * scale_log2 : -INFINITY;
+        z[2] = vb ? c[2] * scale_log2 : -INFINITY;
+        z[3] = vb ? c[3] * scale_log2 : -INFINITY;
+        float mt[2] = {fmaxf(z[0], z[2]), fmaxf(z[1], z[3])};
+#pragma unroll
+        for (int o2 = 4; o2 < 32; o2 <<= 1) {  // over the 8 lanes of a t4 (the rows)
+            mt[0] = fmaxf(mt[0], __shfl_xor_sync(0xffffffffu, mt[0], o2));
+            mt[1] = fmaxf(mt[1], __shfl_xor_sync(0xffffffffu, mt[1], o2));
         }
-        float mt = fmaxf(fmaxf(z[0], z[1]), fmaxf(z[2], z[3]));
-        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
-        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
-        const float mnew = fmaxf(m_run, mt);
-        if (mnew != -INFINITY) {  // uniform across the 4 lanes of head g
-            const float alpha = m_run == -INFINITY ? 0.f : exp2f(m_run - mnew);
-            float p[4];
+        float alpha[2], p[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) p[e] = z[e] == -INFINITY ? 0.f : exp2f(z[e] - mnew);
-            float ps = (p[0] + p[1]) + (p[2] + p[3]);
-            ps += __shfl_xor_sync(0xffffffffu, ps, 1);
-            ps += __shfl_xor_sync(0xffffffffu, ps, 2);
-            l_run = l_run * alpha + ps;
-            m_run = mnew;
+        for (int j = 0; j < 2; ++j) {
+            const float mnew = fmaxf(m_run[j], mt[j]);
+            // a head with no finite logit yet keeps m = -inf, alpha = 0 and p = 0
+            alpha[j] = m_run[j] == -INFINITY ? 0.f : exp2f(m_run[j] - mnew);
+            m_run[j] = mnew;
+        }
 #pragma unroll
-            for (int n = 0; n < 16; ++n) {
-                o[n][0] *= alpha;
-                o[n][1] *= alpha;
-            }
-            // P as the A operand (row g, k = tile rows), split hi + lo
-            const uint32_t ph0 = pack_bf16(p[0], p[1]), ph1 = pack_bf16(p[2], p[3]);
-            const __nv_bfloat162 h0 = *reinterpret_cast<const __nv_bfloat162*>(&ph0);
-            const __nv_bfloat162 h1 = *reinterpret_cast<const __nv_bfloat162*>(&ph1);
-            const uint32_t pl0 = pack_bf16(p[0] - __low2float(h0), p[1] - __high2float(h0));
-            const uint32_t pl1 = pack_bf16(p[2] - __low2float(h1), p[3] - __high2float(h1));
-            // ---- O += P V over 16 dim n-tiles
-            const int m = lane >> 3, i = lane & 7;  // ldmatrix.trans: matrix m, row i
-            const int row = r0 + (m & 1) * 8 + i;    // k-half (m&1), dim n-tile (m>>1)
+        for (int e = 0; e < 4; ++e) p[e] = z[e] == -INFINITY ? 0.f : exp2f(z[e] - m_run[e & 1]);
+        float ps[2] = {p[0] + p[2], p[1] + p[3]};
 #pragma unroll
-            for (int np = 0; np < 8; ++np) {
-                uint32_t b0, b1, b2, b3;
-                ldsm_x4_t(vt + off(row, 2 * np + (m >> 1)), b0, b1, b2, b3);
-                mma_bf16(o[2 * np], ph0, ph1, b0, b1);
-                mma_bf16(o[2 * np], pl0, pl1, b0, b1);
-                mma_bf16(o[2 * np + 1], ph0, ph1, b2, b3);
-                mma_bf16(o[2 * np + 1], pl0, pl1, b2, b3);
-            }
+        for (int o2 = 4; o2 < 32; o2 <<= 1) {
+            ps[0] += __shfl_xor_sync(0xffffffffu, ps[0], o2);
+            ps[1] += __shfl_xor_sync(0xffffffffu, ps[1], o2);
+        }
+        l_run[0] = l_run[0] * alpha[0] + ps[0];
+        l_run[1] = l_run[1] * alpha[1] + ps[1];
+#pragma unroll
+        for (int n = 0; n < 8; ++n) {
+            o[n][0] *= alpha[0];
+            o[n][1] *= alpha[1];
+            o[n][2] *= alpha[0];
+            o[n][3] *= alpha[1];
+        }
+        // P^T as the B operand (k = tile rows, n = heads), split hi + lo: the
+        // accumulator holds row g / heads 2t4.. of each 8x8 block, the operand
+        // rows 2t4.. / head g, so each block is transposed in registers
+        const uint32_t pa = pack_bf16(p[0], p[1]), pb = pack_bf16(p[2], p[3]);
+        const __nv_bfloat162 ha = *reinterpret_cast<const __nv_bfloat162*>(&pa);
+        const __nv_bfloat162 hb = *reinterpret_cast<const __nv_bfloat162*>(&pb);
+        const uint32_t la = pack_bf16(p[0] - __low2float(ha), p[1] - __high2float(ha));
+        const uint32_t lb = pack_bf16(p[2] - __low2float(hb), p[3] - __high2float(hb));
+        const uint32_t bh0 = movmatrix_t(pa), bh1 = movmatrix_t(pb);
+        const uint32_t bl0 = movmatrix_t(la), bl1 = movmatrix_t(lb);
+        // ---- O^T += V^T P^T over 8 m-tiles of 16 dims
+        const int m = lane >> 3, i = lane & 7;  // ldmatrix.trans: matrix m, row i
+        const int row = r0 + (m >> 1) * 8 + i;   // rows +8 (m>>1), dims +8 (m&1)
+#pragma unroll
+        for (int mt2 = 0; mt2 < 8; ++mt2) {
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4_t(vt + off(row, 2 * mt2 + (m & 1)), a0, a1, a2, a3);
+            mma_bf16(o[mt2], a0, a1, a2, a3, bh0, bh1);
+            mma_bf16(o[mt2], a0, a1, a2, a3, bl0, bl1);
         }
     };
 
     if constexpr (CONTIG) {
-        for (int t = 0; t < ntiles; ++t) {
+        int t = 0;
+        for (; t < ntiles; ++t) {
             if (tid == 0) next_first = tile_first(t + STAGES);  // in flight during this tile
-            mbar_wait(&s_bar[t % STAGES], (unsigned)(t / STAGES) & 1u, flag);  // tile t has landed
+            // tile t has landed (on a timeout: flag, and the whole CTA stops below)
+            if (!mbar_wait(&s_bar[t % STAGES], (unsigned)(t / STAGES) & 1u, flag)) s_fail = 1;
             const int st = t % STAGES;
             // the valid rows are a prefix: the range's and the sequence's ends cut it;
             // an absent block (first < 0) has none and nothing landed
@@ -475,6 +611,9 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
                 fence_proxy_async();  // before the stage's next tensor load overwrites them
             }
             __syncthreads();  // every thread, every tile (never a divergent barrier)
+            // s_fail is written only before the barrier above and read only
+            // between it and the one below, so every thread sees the same value
+            if (s_fail) break;
             const int nv = tile_rows - r0;
             const uint32_t vm = nv >= 16 ? 0xffffu : (nv > 0 ? (1u << nv) - 1u : 0u);
             if (vm) {  // warp-uniform
@@ -482,17 +621,36 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
                 warp_tile(kt, kt + 2 * 64 * kTileRows * 2, vm, first);
             }
             __syncthreads();  // every warp is done with this stage
-            if (tid == 0) stage_contig(t + STAGES, next_first);  // refill it (nothing past the end)
+            if (tid == 0 && t + STAGES < ntiles) {  // refill it (nothing past the end)
+                stage_contig(t + STAGES, next_first);
+                ++issued;
+            }
         }
-    } else if constexpr (ONE) {
-        for (int t = 0; t < ntiles; ++t) {  // one tile (any count stays correct, unpipelined)
-            if (t > 0) issue_one(t);
-            asm volatile("cp.async.wait_all;\n" ::: "memory");
+        // after a timeout: wait (bounded, no second flag) for the loads still in
+        // flight, so that none lands in this SM's shared memory after the CTA
+        // has gone; the output is then unspecified, and the flag says so
+        if (t < ntiles && tid == 0)
+            for (int j = t; j < issued; ++j) mbar_wait(&s_bar[j % STAGES], (unsigned)(j / STAGES) & 1u, nullptr);
+    } else if constexpr (ASYNC) {
+        for (int t = 0; t < ntiles; ++t) {
+            // this lane's copies of tile t have landed (at most STAGES - 1 newer
+            // groups still pending), then the warp's
+            asm volatile("cp.async.wait_group %0;\n" ::"n"(STAGES - 1) : "memory");
             __syncwarp();
-            if (vm_one) warp_tile(sbase, sbase + kTileRows * kRowStride, vm_one, 0);
-            __syncwarp();  // the math has read these rows before the next copies land
+            const int st = t % STAGES;
+            // the slot's rows seen as rows r0 .. r0 + 15 of a tile (the math's row offsets)
+            const unsigned ks = sbase + (unsigned)((st * kAttnWarps + warp) * kSlotBytes) - (unsigned)(r0 * kRowStride);
+            if (vmr[0]) warp_tile(ks, ks + 16 * kRowStride, vmr[0], 0);
+            __syncwarp();  // the math has read these rows before the stage is refilled
+#pragma unroll
+            for (int i = 0; i + 1 < STAGES; ++i) vmr[i] = vmr[i + 1];
+            vmr[STAGES - 1] = t + STAGES < ntiles ? issue_async(t + STAGES, st, my_row(t + STAGES)) : 0u;
+            asm volatile("cp.async.commit_group;\n" ::: "memory");
         }
+        asm volatile("cp.async.wait_all;\n" ::: "memory");  // nothing in flight over the merge below
     } else {
+        unsigned char* kw = smem + r0 * kRowStride;
+        unsigned char* vw = smem + (kTileRows + r0) * kRowStride;
         for (int t = 0; t < ntiles; ++t) {
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
@@ -501,48 +659,51 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
             }
             const uint32_t vm = vm_next;
             __syncwarp();
-            if (t + 1 < ntiles) fetch(t + 1);  // the next tile's loads fly during this tile's math
+            if (t + 1 < ntiles) fetch(t + 1, my_row(t + 1));  // the next tile's loads fly during this tile's math
             if (vm) warp_tile(sbase, sbase + kTileRows * kRowStride, vm, 0);
             __syncwarp();  // the math has read these rows before the next store
         }
     }
     __syncthreads();
 
-    // ---- merge the 4 warps: each warp's (m, l, o) for heads g < G
-    float* s_acc = reinterpret_cast<float*>(smem);  // [kAttnWarps][G][128], over the staging ring
-    if (g < G) {
+    // ---- merge the 8 warps: each warp's (m, l, o) for heads < G
+    float* s_acc = reinterpret_cast<float*>(smem);  // [kAttnWarps][G][kAccStride], over the staging ring
 #pragma unroll
-        for (int n = 0; n < 16; ++n)
-            *reinterpret_cast<float2*>(s_acc + (warp * G + g) * kD + 8 * n + 2 * t4) = make_float2(o[n][0], o[n][1]);
-        if (t4 == 0) {
-            s_wm[warp][g] = m_run;
-            s_wl[warp][g] = l_run;
+    for (int j = 0; j < 2; ++j) {
+        const int h = 2 * t4 + j;
+        if (h < G) {
+            float* row = s_acc + (warp * G + h) * kAccStride;
+#pragma unroll
+            for (int n = 0; n < 8; ++n) {
+                row[16 * n + g] = o[n][j];
+                row[16 * n + g + 8] = o[n][j + 2];
+            }
+            if (g == 0) {
+                s_wm[warp][h] = m_run[j];
+                s_wl[warp][h] = l_run[j];
+            }
         }
-    }
-    __syncthreads();
-    if (tid < G) {
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, s_wm[w][tid]);
-        float L = 0.f;
-#pragma unroll
-        for (int w = 0; w < kAttnWarps; ++w)
-            L += s_wm[w][tid] == -INFINITY ? 0.f : s_wl[w][tid] * exp2f(s_wm[w][tid] - M);
-        s_M[tid] = M;
-        s_L[tid] = L;
     }
     __syncthreads();
     const int nslots = G * 32;  // (head, quad of dims) output slots: thread tid owns slot tid
     const bool has_slot = tid < nslots;
     const int h_me = tid >> 5, qd_me = tid & 31;
+    // the CTA's (M, L, acc) for head h_me: every slot thread of the head forms
+    // M and L itself from the 8 warps' (m, l) (no extra barrier)
     float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
+    float M_me = -INFINITY, L_me = 0.f;
     if (has_slot) {
-        const float M = s_M[h_me];
+        float wm[kAttnWarps];
 #pragma unroll
         for (int w = 0; w < kAttnWarps; ++w) {
-            const float wm = s_wm[w][h_me];
-            const float sc = (wm == -INFINITY || M == -INFINITY) ? 0.f : exp2f(wm - M);
-            const float4 a = *reinterpret_cast<const float4*>(s_acc + (w * G + h_me) * kD + 4 * qd_me);
+            wm[w] = s_wm[w][h_me];
+            M_me = fmaxf(M_me, wm[w]);
+        }
+#pragma unroll
+        for (int w = 0; w < kAttnWarps; ++w) {
+            const float sc = (wm[w] == -INFINITY || M_me == -INFINITY) ? 0.f : exp2f(wm[w] - M_me);
+            L_me += s_wl[w][h_me] * sc;
+            const float4 a = *reinterpret_cast<const float4*>(s_acc + (w * G + h_me) * kAccStride + 4 * qd_me);
             A.x += a.x * sc;
             A.y += a.y * sc;
             A.z += a.z * sc;
@@ -553,26 +714,25 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
     if constexpr (CLUSTER) {
         if (S == 1) {  // nothing to combine
             if (has_slot) {
-                const float L = s_L[h_me];
+                const float L = L_me;
                 float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (L > 0.f) r = make_float4(A.x / L, A.y / L, A.z / L, A.w / L);
                 *reinterpret_cast<float4*>(O + ((size_t)unit * G + h_me) * kD + 4 * qd_me) = r;
-                if (lse && qd_me == 0) lse[(size_t)unit * G + h_me] = L > 0.f ? s_M[h_me] + log2f(L) : -INFINITY;
+                if (lse && qd_me == 0) lse[(size_t)unit * G + h_me] = L > 0.f ? M_me + log2f(L) : -INFINITY;
             }
             return;
         }
         // the S splits of this unit are the S CTAs of this cluster (rank = split)
         cg::cluster_group cluster = cg::this_cluster();
         const int per = ceil_div(nslots, S);  // output slots owned by each CTA
-        float4* recv = reinterpret_cast<float4*>(smem + Cfg::work_bytes(STAGES));  // [src][Cfg::kPer]
+        float4* recv = reinterpret_cast<float4*>(smem + work);  // [src][per], past the work area
         if (has_slot) {
             const int owner = tid / per, lslot = tid - owner * per;
-            *cluster.map_shared_rank(recv + s * Cfg::kPer + lslot, owner) = A;
+            *cluster.map_shared_rank(recv + s * per + lslot, owner) = A;
         }
-        if (tid < G * S) {
-            const int r = tid / G, h = tid - (tid / G) * G;
-            *cluster.map_shared_rank(&s_Mr[s][h], r) = s_M[h];
-            *cluster.map_shared_rank(&s_Lr[s][h], r) = s_L[h];
+        if (has_slot && qd_me < S) {  // head h_me's (M, L) to rank qd_me
+            *cluster.map_shared_rank(&s_Mr[s][h_me], qd_me) = M_me;
+            *cluster.map_shared_rank(&s_Lr[s][h_me], qd_me) = L_me;
         }
         cluster.sync();  // every slice has arrived at its owner
         for (int ls = tid; ls < per; ls += kAttnThreads) {
@@ -586,7 +746,7 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
             if (M != -INFINITY) {
                 for (int j = 0; j < S; ++j) {
                     const float w = s_Mr[j][h] == -INFINITY ? 0.f : exp2f(s_Mr[j][h] - M);
-                    const float4 oj = recv[j * Cfg::kPer + ls];
+                    const float4 oj = recv[j * per + ls];
                     den += w * s_Lr[j][h];
                     num.x += w * oj.x;
                     num.y += w * oj.y;
@@ -604,7 +764,7 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
         if (has_slot) {
             float* pu = part + (((size_t)unit * S + s) * G + h_me) * kPartStride;
             *reinterpret_cast<float4*>(pu + 4 + 4 * qd_me) = A;
-            if (qd_me == 0) *reinterpret_cast<float2*>(pu) = make_float2(s_M[h_me], s_L[h_me]);
+            if (qd_me == 0) *reinterpret_cast<float2*>(pu) = make_float2(M_me, L_me);
         }
         // the last CTA of this unit to arrive combines all splits
         __threadfence();
@@ -679,12 +839,24 @@ int attn_splits(const Dims& d, int k_max, int block, bool dense) {
         rows = (long long)(k_max < nbmax ? k_max : nbmax) * block;
         s = (int)((rows + kTileRows - 1) / kTileRows);
         const int room = kSms / units > 1 ? kSms / units : 1;
-        if (s > room) s = room;
+        if (s > room) {
+            // token gathers: two CTAs an SM when a CTA's range fits 12 warp-tiles
+            // (192 rows, ~102 KB of staging); more, shorter CTAs shorten the
+            // chain of tiles each warp works through
+            const int room2 = 2 * kSms / units > 1 ? 2 * kSms / units : 1;
+            const int s2 = s < room2 ? s : room2;
+            s = (block == 1 && (rows + s2 - 1) / s2 <= 12 * 16) ? s2 : room;
+        }
         // past 8 splits the partials combine through the workspace (the last CTA
         // of a unit reads them all), which costs more than the extra splits save
         // unless there are too few units to fill the GPU (16-CTA clusters measured
         // no faster than 8: the per-launch chain of dependent loads dominates)
-        if (s > kClusterMax && units >= 4) s = kClusterMax;
+        // token gathers spread over up to 16 CTAs a unit (a non-portable
+        // cluster): a CTA's gather rate is bound by its loads in flight (about
+        // 50-60 GB/s an SM), so a 128K layer's 8 units want all the SMs, not 64
+        // of them; contiguous 128-token blocks stay at 8
+        const int cap = block == 1 ? kClusterMax : kPortableCluster;
+        if (s > cap && units >= 4) s = cap;
     }
     const long long smax = (rows + 31) / 32;  // at least 32 positions per split
     if (s > smax) s = (int)smax;
@@ -705,14 +877,29 @@ static int g_attn_configured[64];
 // device and kernel configuration, and the cluster combine is used only when
 // every unit's cluster is co-resident; otherwise the splits combine through the
 // workspace (sized for them in either case).
-static int g_max_clusters[64][4][2][2][kClusterMax + 1];  // dev, log2 G, one-tile, contig, S; 0 = unknown
+// Instance of the kernel a launch takes (besides G and the cluster choice):
+// contiguous tiles in a 1-stage or kRing-stage TMA ring; or the gather, through
+// registers (host memory), or by cp.async in a 1-stage or kRing-stage ring.
+enum AttnVariant { kContig1 = 0, kContigRing = 1, kGatherReg = 2, kGatherAsync1 = 3, kGatherAsyncRing = 4, kVariants = 5 };
 
-template <int G, int STAGES, bool CONTIG, bool ONE>
-static int max_active_clusters(int S) {
+// co-resident clusters by (device, log2 G, variant, S, warp-tile slots of the
+// cp.async gather or 0); 0 = not queried yet
+constexpr int kCacheDevs = 16;
+static int g_max_clusters[kCacheDevs][4][kVariants][kClusterMax + 1][3 * kAttnWarps + 1];
+
+// the work area (staging, merge buffer) of an instance: the cp.async gather by
+// the slots its CTAs use, every other instance its whole ring
+template <int G, int STAGES, bool CONTIG, bool ASYNC>
+static int work_bytes_of(int slots) {
+    return (ASYNC && !CONTIG) ? AttnCfg<G>::slot_work_bytes(slots) : AttnCfg<G>::work_bytes(STAGES);
+}
+
+template <int G, int STAGES, bool CONTIG, bool ASYNC>
+static int max_active_clusters(int S, int slots) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)S, 1);
     cfg.blockDim = dim3(kAttnThreads);
-    cfg.dynamicSmemBytes = AttnCfg<G>::smem_bytes(STAGES, true);
+    cfg.dynamicSmemBytes = 1024 + work_bytes_of<G, STAGES, CONTIG, ASYNC>(slots) + AttnCfg<G>::kRecvBytes;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)S;
@@ -721,7 +908,7 @@ static int max_active_clusters(int S) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, attn_kernel<G, STAGES, true, CONTIG, ONE>, &cfg) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveClusters(&n, attn_kernel<G, STAGES, true, CONTIG, ASYNC>, &cfg) != cudaSuccess) {
         cudaGetLastError();  // clear it: the workspace combine is always available
         return -1;
     }
@@ -729,30 +916,41 @@ static int max_active_clusters(int S) {
 }
 
 template <int G>
-static bool attn_cluster_fits_g(int dev, bool one_tile, bool contig, int S, int units) {
-    const int lg = G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : 3;
-    int& slot = g_max_clusters[dev][lg][one_tile][contig][S];
-    if (slot == 0) {
-        int n;
-        if (!contig) n = one_tile ? max_active_clusters<G, 1, false, true>(S) : max_active_clusters<G, 1, false, false>(S);
-        else n = one_tile ? max_active_clusters<G, 1, true, false>(S) : max_active_clusters<G, kRing, true, false>(S);
-        slot = n;
+static int max_clusters_g(int var, int S, int slots) {
+    switch (var) {
+        case kContig1: return max_active_clusters<G, 1, true, false>(S, 0);
+        case kContigRing: return max_active_clusters<G, kRing, true, false>(S, 0);
+        case kGatherReg: return max_active_clusters<G, 1, false, false>(S, 0);
+        case kGatherAsync1: return max_active_clusters<G, 1, false, true>(S, slots);
+        default: return max_active_clusters<G, kRing, false, true>(S, slots);
     }
-    return slot > 0 && units <= slot;
 }
 
-static bool attn_cluster_fits(int G, bool one_tile, bool contig, int S, int units) {
+static bool attn_cluster_fits(int G, int var, int S, int units, int slots) {
     if (S > kClusterMax) return false;
     if (S == 1) return true;  // a cluster of one: no co-scheduling constraint
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
-    switch (G) {
-        case 1: return attn_cluster_fits_g<1>(dev, one_tile, contig, S, units);
-        case 2: return attn_cluster_fits_g<2>(dev, one_tile, contig, S, units);
-        case 4: return attn_cluster_fits_g<4>(dev, one_tile, contig, S, units);
-        case 8: return attn_cluster_fits_g<8>(dev, one_tile, contig, S, units);
-        default: return false;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return false;
+    if (var != kGatherAsync1 && var != kGatherAsyncRing) slots = 0;
+    auto query = [&]() {
+        switch (G) {
+            case 1: return max_clusters_g<1>(var, S, slots);
+            case 2: return max_clusters_g<2>(var, S, slots);
+            case 4: return max_clusters_g<4>(var, S, slots);
+            case 8: return max_clusters_g<8>(var, S, slots);
+            default: return -1;
+        }
+    };
+    int n;
+    if (dev < kCacheDevs) {
+        const int lg = G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : 3;
+        int& c = g_max_clusters[dev][lg][var][S][slots];
+        if (c == 0) c = query();
+        n = c;
+    } else {
+        n = query();
     }
+    return n > 0 && units <= n;
 }
 
 struct AttnArgs {
@@ -770,14 +968,16 @@ struct AttnArgs {
     float* sout;
     float scale;
     float* lse;
+    int slots;  // the cp.async gather: warp-tile slots its CTAs use
 };
 
-template <int G, int STAGES, bool CLUSTER, bool CONTIG, bool ONE = false>
+template <int G, int STAGES, bool CLUSTER, bool CONTIG, bool ASYNC = false>
 static cudaError_t attn_launch_g(dim3 grid, cudaStream_t st, const AttnArgs& a) {
+    const int work = work_bytes_of<G, STAGES, CONTIG, ASYNC>(a.slots);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = dim3(kAttnThreads);
-    cfg.dynamicSmemBytes = AttnCfg<G>::smem_bytes(STAGES, CLUSTER);
+    cfg.dynamicSmemBytes = 1024 + work + (CLUSTER ? AttnCfg<G>::kRecvBytes : 0);
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -787,14 +987,14 @@ static cudaError_t attn_launch_g(dim3 grid, cudaStream_t st, const AttnArgs& a) 
     attr[1] = pdl_attr();
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, attn_kernel<G, STAGES, CLUSTER, CONTIG, ONE>, a.kmap, a.vmap, a.q, a.k, a.v, a.lens,
+    return cudaLaunchKernelEx(&cfg, attn_kernel<G, STAGES, CLUSTER, CONTIG, ASYNC>, a.kmap, a.vmap, a.q, a.k, a.v, a.lens,
                               a.idx, a.kreq, a.k_max, a.block, a.Hkv, a.Ncap, a.sl2, a.splits, a.partials, a.counters,
-                              a.O, a.flag, a.early, a.sout, a.scale, a.lse);
+                              a.O, a.flag, a.early, a.sout, a.scale, a.lse, work);
 }
 
-template <int G, int STAGES, bool CLUSTER, bool CONTIG, bool ONE = false>
+template <int G, int STAGES, bool CLUSTER, bool CONTIG, bool ASYNC = false>
 static cudaError_t attn_configure_one() {
-    const void* f = (const void*)attn_kernel<G, STAGES, CLUSTER, CONTIG, ONE>;
+    const void* f = (const void*)attn_kernel<G, STAGES, CLUSTER, CONTIG, ASYNC>;
     cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          AttnCfg<G>::smem_bytes(STAGES, CLUSTER));
     if (e == cudaSuccess && CLUSTER) e = cudaFuncSetAttribute(f, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
@@ -804,37 +1004,35 @@ static cudaError_t attn_configure_one() {
 template <int G>
 static cudaError_t attn_configure() {
     cudaError_t e = cudaSuccess;
-    // the gather runs one stage; contiguous tiles one or kRing
-    if (e == cudaSuccess) e = attn_configure_one<G, 1, true, false>();
-    if (e == cudaSuccess) e = attn_configure_one<G, 1, false, false>();
-    if (e == cudaSuccess) e = attn_configure_one<G, 1, true, false, true>();
-    if (e == cudaSuccess) e = attn_configure_one<G, 1, false, false, true>();
-    if (e == cudaSuccess) e = attn_configure_one<G, 1, true, true>();
-    if (e == cudaSuccess) e = attn_configure_one<G, kRing, true, true>();
-    if (e == cudaSuccess) e = attn_configure_one<G, 1, false, true>();
-    if (e == cudaSuccess) e = attn_configure_one<G, kRing, false, true>();
+    // contiguous tiles: one stage or kRing; the gather: registers, or cp.async
+    // with one stage or kRing
+#define TSA_CONF(ST, CONTIG, ASYNC)                                                      \
+    if (e == cudaSuccess) e = attn_configure_one<G, ST, true, CONTIG, ASYNC>();   \
+    if (e == cudaSuccess) e = attn_configure_one<G, ST, false, CONTIG, ASYNC>();
+    TSA_CONF(1, true, false)
+    TSA_CONF(kRing, true, false)
+    TSA_CONF(1, false, false)
+    TSA_CONF(1, false, true)
+    TSA_CONF(kRing, false, true)
+#undef TSA_CONF
     return e;
 }
 
-template <int G, bool CONTIG>
-static cudaError_t attn_dispatch2(bool one_tile, bool cluster, dim3 grid, cudaStream_t st, const AttnArgs& a) {
-    if constexpr (!CONTIG) {  // the gather: one stage; one tile a CTA -> the cp.async instance
-        if (one_tile)
-            return cluster ? attn_launch_g<G, 1, true, false, true>(grid, st, a)
-                           : attn_launch_g<G, 1, false, false, true>(grid, st, a);
-        return cluster ? attn_launch_g<G, 1, true, false>(grid, st, a) : attn_launch_g<G, 1, false, false>(grid, st, a);
-    } else {
-        if (cluster)
-            return one_tile ? attn_launch_g<G, 1, true, true>(grid, st, a) : attn_launch_g<G, kRing, true, true>(grid, st, a);
-        return one_tile ? attn_launch_g<G, 1, false, true>(grid, st, a) : attn_launch_g<G, kRing, false, true>(grid, st, a);
-    }
+template <int G, int STAGES, bool CONTIG, bool ASYNC>
+static cudaError_t attn_launch_c(bool cluster, dim3 grid, cudaStream_t st, const AttnArgs& a) {
+    return cluster ? attn_launch_g<G, STAGES, true, CONTIG, ASYNC>(grid, st, a)
+                   : attn_launch_g<G, STAGES, false, CONTIG, ASYNC>(grid, st, a);
 }
 
 template <int G>
-static cudaError_t attn_dispatch(bool contig, bool one_tile, bool cluster, dim3 grid, cudaStream_t st,
-                                 const AttnArgs& a) {
-    return contig ? attn_dispatch2<G, true>(one_tile, cluster, grid, st, a)
-                  : attn_dispatch2<G, false>(one_tile, cluster, grid, st, a);
+static cudaError_t attn_dispatch(int var, bool cluster, dim3 grid, cudaStream_t st, const AttnArgs& a) {
+    switch (var) {
+        case kContig1: return attn_launch_c<G, 1, true, false>(cluster, grid, st, a);
+        case kContigRing: return attn_launch_c<G, kRing, true, false>(cluster, grid, st, a);
+        case kGatherReg: return attn_launch_c<G, 1, false, false>(cluster, grid, st, a);
+        case kGatherAsync1: return attn_launch_c<G, 1, false, true>(cluster, grid, st, a);
+        default: return attn_launch_c<G, kRing, false, true>(cluster, grid, st, a);
+    }
 }
 
 // tensor map over a [units * Ncap rows] x [128 dims] bf16 cache, box 64 dims x 128 rows, 128-byte swizzle
@@ -861,7 +1059,7 @@ static cudaError_t make_row_map(CUtensorMap* map, const void* base, const Dims& 
 cudaError_t launch_attn(const void* Q, const void* K, const void* V, const int32_t* lens,
                         const int32_t* idx, const int32_t* kreq, int k_max, int block,
                         const Dims& d, float scale, int splits, float* partials,
-                        unsigned* counters, float* O, unsigned* flag, cudaStream_t st, bool early,
+                        unsigned* counters, float* O, unsigned* flag, cudaStream_t st, int early,
                         float* scores_out, bool host_kv, float* lse_out) {
     if (d.units() == 0) return cudaSuccess;
     // scores come with full attention on the tensor-map path only
@@ -889,12 +1087,40 @@ cudaError_t launch_attn(const void* Q, const void* K, const void* V, const int32
     // gather, which fetches only the rows in the set, with plain vector loads
     // through the device's mapping of the host pages (no tensor map over them).
     const bool contig = !host_kv && (idx == nullptr || block == kTileRows);
-    const long long per_split = contig ? ((rows + splits - 1) / splits + kTileRows - 1) / kTileRows * kTileRows
-                                       : (rows + splits - 1) / splits;
     // one tile a CTA: the single-stage kernel (contiguous tiles), or the gather's
-    // two-CTAs-an-SM instance (its cp.async copies are kept to device memory)
-    const bool one_tile = per_split <= kTileRows && !host_kv;
-    const bool cluster = attn_cluster_fits(d.G, one_tile, contig, splits, d.units());
+    // two-CTAs-an-SM instance; several: the 3-stage rings.  K and V in host
+    // memory: the register gather (cp.async is kept to device memory)
+    auto per_split_of = [&](int S) {
+        return contig ? ((rows + S - 1) / S + kTileRows - 1) / kTileRows * kTileRows : (rows + S - 1) / S;
+    };
+    auto variant_of = [&](int S) {
+        const bool one_tile = per_split_of(S) <= kTileRows;
+        return contig ? (one_tile ? kContig1 : kContigRing)
+                      : host_kv ? kGatherReg : one_tile ? kGatherAsync1 : kGatherAsyncRing;
+    };
+    // warp-tile slots of the cp.async gather: its range's 16-row groups, at
+    // most the ring's
+    auto slots_of = [&](int S, int var) {
+        const long long wt = (per_split_of(S) + 15) / 16;
+        const int cap = var == kGatherAsync1 ? kAttnWarps : kRing * kAttnWarps;
+        return (int)(wt < cap ? (wt < 1 ? 1 : wt) : cap);
+    };
+    int var = variant_of(splits);
+    int slots = slots_of(splits, var);
+    bool cluster = attn_cluster_fits(d.G, var, splits, d.units(), slots);
+    if (!cluster && splits > kPortableCluster) {
+        // a non-portable cluster that cannot be co-resident for every unit: the
+        // portable size, if that can (fewer splits than the workspace is sized
+        // for, which is always enough)
+        const int v8 = variant_of(kPortableCluster);
+        const int s8 = slots_of(kPortableCluster, v8);
+        if (attn_cluster_fits(d.G, v8, kPortableCluster, d.units(), s8)) {
+            splits = kPortableCluster;
+            var = v8;
+            slots = s8;
+            cluster = true;
+        }
+    }
     AttnArgs a;
     memset(&a.kmap, 0, sizeof a.kmap);
     memset(&a.vmap, 0, sizeof a.vmap);
@@ -918,16 +1144,17 @@ cudaError_t launch_attn(const void* Q, const void* K, const void* V, const int32
     a.counters = counters;
     a.O = O;
     a.flag = flag;
-    a.early = early ? 1 : 0;
+    a.early = early;
     a.sout = scores_out;
     a.scale = scale;
     a.lse = lse_out;
+    a.slots = slots;
     dim3 grid(splits, d.units());
     switch (d.G) {
-        case 1: e = attn_dispatch<1>(contig, one_tile, cluster, grid, st, a); break;
-        case 2: e = attn_dispatch<2>(contig, one_tile, cluster, grid, st, a); break;
-        case 4: e = attn_dispatch<4>(contig, one_tile, cluster, grid, st, a); break;
-        case 8: e = attn_dispatch<8>(contig, one_tile, cluster, grid, st, a); break;
+        case 1: e = attn_dispatch<1>(var, cluster, grid, st, a); break;
+        case 2: e = attn_dispatch<2>(var, cluster, grid, st, a); break;
+        case 4: e = attn_dispatch<4>(var, cluster, grid, st, a); break;
+        case 8: e = attn_dispatch<8>(var, cluster, grid, st, a); break;
         default: return cudaErrorInvalidValue;
     }
     note_launch();
@@ -936,3 +1163,9 @@ cudaError_t launch_attn(const void* Q, const void* K, const void* V, const int32
 }
 
 }  // namespace tsa
+
+#ifdef TSA_DEBUG_KNOBS
+extern "C" int tsa_debug_attn_skip_tile(int tile) {
+    return (int)cudaMemcpyToSymbol(tsa::g_debug_attn_skip_tile, &tile, sizeof tile);
+}
+#endif

@@ -60,12 +60,14 @@ cudaError_t launch_block_summarize(const void* K, const int32_t* lens, const Dim
 // read and then zeroed by the top-k that follows it (the decode step pairs them).
 constexpr int kHistBins = 2048;
 
+// early (token mode): the kernel before this one writes neither lens nor K, so
+// the first K tiles are requested before waiting on it
 cudaError_t launch_score(const void* Q, const void* keys, const int32_t* lens, const Dims& d,
                          int block, float scale, float* scores, uint32_t* hist, unsigned* flag,
-                         cudaStream_t st);
+                         cudaStream_t st, bool early = false);
 // token mode on the tensor cores (TMA + tcgen05); used by launch_score for bf16 keys
 cudaError_t launch_score_tc(const void* Q, const void* K, const int32_t* lens, const Dims& d, float scale,
-                            float* scores, uint32_t* hist, unsigned* flag, cudaStream_t st);
+                            float* scores, uint32_t* hist, unsigned* flag, cudaStream_t st, bool early);
 
 // top-k plan: cluster size and keys per CTA for a row count; false if too large
 bool topk_plan(int rows_cap, int* cluster, int* chunk);
@@ -96,10 +98,10 @@ cudaError_t launch_attn(const void* Q, const void* K, const void* V, const int32
                         const int32_t* idx, const int32_t* kreq, int k_max, int block,
                         const Dims& d, float scale, int splits, float* partials,
                         unsigned* counters, float* O, unsigned* flag, cudaStream_t st,
-                        bool early = false,  // early: lens, k's and Q not written by the previous kernel
+                        int early = 0,  // 1: lens and k's not written by the previous kernel; 2: nor idx, K, V
                         float* scores_out = nullptr,  // full attention: each row's group-max scaled score
                         bool host_kv = false,         // K, V in mapped page-locked host memory: gather only
-                        float* lse_out = nullptr);    // [units*G]: base-2 log-sum-exp of each head's scaled logits  // full attention only: [units][Ncap] scores of the valid rows
+                        float* lse_out = nullptr);    // [units*G]: base-2 log-sum-exp of each head's scaled logits
 
 cudaError_t launch_copy(const void* src, void* dst, size_t bytes, cudaStream_t st);
 cudaError_t launch_gather(const void* base, size_t base_bytes, const int32_t* rows, int nrows, unsigned* flag,

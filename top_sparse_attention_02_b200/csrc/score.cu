@@ -113,9 +113,9 @@ block_mean_kernel(const __nv_bfloat16* __restrict__ K, const int32_t* __restrict
 
 cudaError_t launch_score(const void* Q, const void* keys, const int32_t* lens, const Dims& d,
                          int block, float scale, float* scores, uint32_t* hist, unsigned* flag,
-                         cudaStream_t st) {
+                         cudaStream_t st, bool early) {
     if (d.units() == 0 || d.Ncap == 0) return cudaSuccess;
-    if (block == 1) return launch_score_tc(Q, keys, lens, d, scale, scores, hist, flag, st);
+    if (block == 1) return launch_score_tc(Q, keys, lens, d, scale, scores, hist, flag, st, early);
     const int rows_cap = rows_cap_of(d, block);
     const int rows_cta = 2 * (16 / d.G) * kScoreWarps;
     cudaLaunchConfig_t cfg = {};
