@@ -72,8 +72,7 @@ namespace cg = cooperative_groups;
 namespace tsa {
 
 constexpr int kMaxSplits = 256;
-constexpr int kClusterMax = 16;     // splits per unit that combine inside one cluster (16: non-portable)
-constexpr int kPortableCluster = 8; // the largest cluster size every GPU supports
+constexpr int kClusterMax = 8;  // splits per unit that combine inside one (portable) cluster
 constexpr int kSms = 148;
 constexpr int kPartStride = kD + 4;  // M, L, 2 pad, acc[128]: 528 B, 16-byte aligned
 constexpr int kAttnThreads = 256;
@@ -735,29 +734,42 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
             *cluster.map_shared_rank(&s_Lr[s][h_me], qd_me) = L_me;
         }
         cluster.sync();  // every slice has arrived at its owner
-        for (int ls = tid; ls < per; ls += kAttnThreads) {
+        // this CTA's `per` output slots, each from the S sources: one thread a
+        // (slot, source) pair, the S2 (S rounded up to a power of two) threads
+        // of a slot adjacent in a warp and reduced by shuffles
+        const int S2 = S <= 2 ? 2 : S <= 4 ? 4 : 8;
+        const int lg2 = S2 == 2 ? 1 : S2 == 4 ? 2 : 3;
+        const int total = (per * S2 + 31) & ~31;  // whole warps: every lane of a warp takes part
+        for (int q = tid; q < total; q += kAttnThreads) {
+            const int ls = q >> lg2, j = q & (S2 - 1);
             const int slot = s * per + ls;
-            if (slot >= nslots) break;
-            const int h = slot >> 5, qd = slot & 31;
-            float M = -INFINITY;
-            for (int j = 0; j < S; ++j) M = fmaxf(M, s_Mr[j][h]);
+            const bool live = ls < per && slot < nslots;
+            const bool src = live && j < S;
+            const int h = live ? slot >> 5 : 0, qd = slot & 31;
+            const float mj = src ? s_Mr[j][h] : -INFINITY;
+            float M = mj;
+            for (int o2 = 1; o2 < S2; o2 <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o2));
+            const float w = mj == -INFINITY ? 0.f : exp2f(mj - M);
             float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
             float den = 0.f;
-            if (M != -INFINITY) {
-                for (int j = 0; j < S; ++j) {
-                    const float w = s_Mr[j][h] == -INFINITY ? 0.f : exp2f(s_Mr[j][h] - M);
-                    const float4 oj = recv[j * per + ls];
-                    den += w * s_Lr[j][h];
-                    num.x += w * oj.x;
-                    num.y += w * oj.y;
-                    num.z += w * oj.z;
-                    num.w += w * oj.w;
-                }
+            if (src) {
+                const float4 oj = recv[j * per + ls];
+                den = w * s_Lr[j][h];
+                num = make_float4(w * oj.x, w * oj.y, w * oj.z, w * oj.w);
             }
-            float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (den > 0.f) r = make_float4(num.x / den, num.y / den, num.z / den, num.w / den);
-            *reinterpret_cast<float4*>(O + ((size_t)unit * G + h) * kD + 4 * qd) = r;
-            if (lse && qd == 0) lse[(size_t)unit * G + h] = den > 0.f ? M + log2f(den) : -INFINITY;
+            for (int o2 = 1; o2 < S2; o2 <<= 1) {
+                den += __shfl_xor_sync(0xffffffffu, den, o2);
+                num.x += __shfl_xor_sync(0xffffffffu, num.x, o2);
+                num.y += __shfl_xor_sync(0xffffffffu, num.y, o2);
+                num.z += __shfl_xor_sync(0xffffffffu, num.z, o2);
+                num.w += __shfl_xor_sync(0xffffffffu, num.w, o2);
+            }
+            if (live && j == 0) {
+                float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (den > 0.f) r = make_float4(num.x / den, num.y / den, num.z / den, num.w / den);
+                *reinterpret_cast<float4*>(O + ((size_t)unit * G + h) * kD + 4 * qd) = r;
+                if (lse && qd == 0) lse[(size_t)unit * G + h] = den > 0.f ? M + log2f(den) : -INFINITY;
+            }
         }
         return;  // no remote access after the barrier: CTAs may leave in any order
     } else {
@@ -851,12 +863,10 @@ int attn_splits(const Dims& d, int k_max, int block, bool dense) {
         // of a unit reads them all), which costs more than the extra splits save
         // unless there are too few units to fill the GPU (16-CTA clusters measured
         // no faster than 8: the per-launch chain of dependent loads dominates)
-        // token gathers spread over up to 16 CTAs a unit (a non-portable
-        // cluster): a CTA's gather rate is bound by its loads in flight (about
-        // 50-60 GB/s an SM), so a 128K layer's 8 units want all the SMs, not 64
-        // of them; contiguous 128-token blocks stay at 8
-        const int cap = block == 1 ? kClusterMax : kPortableCluster;
-        if (s > cap && units >= 4) s = cap;
+        // (16-CTA clusters of short ranges, measured at the 128K shape: the
+        // CTAs pack two to an SM and the 16-way combine costs more than the
+        // shorter ranges save)
+        if (s > kClusterMax && units >= 4) s = kClusterMax;
     }
     const long long smax = (rows + 31) / 32;  // at least 32 positions per split
     if (s > smax) s = (int)smax;
@@ -1105,22 +1115,9 @@ cudaError_t launch_attn(const void* Q, const void* K, const void* V, const int32
         const int cap = var == kGatherAsync1 ? kAttnWarps : kRing * kAttnWarps;
         return (int)(wt < cap ? (wt < 1 ? 1 : wt) : cap);
     };
-    int var = variant_of(splits);
-    int slots = slots_of(splits, var);
-    bool cluster = attn_cluster_fits(d.G, var, splits, d.units(), slots);
-    if (!cluster && splits > kPortableCluster) {
-        // a non-portable cluster that cannot be co-resident for every unit: the
-        // portable size, if that can (fewer splits than the workspace is sized
-        // for, which is always enough)
-        const int v8 = variant_of(kPortableCluster);
-        const int s8 = slots_of(kPortableCluster, v8);
-        if (attn_cluster_fits(d.G, v8, kPortableCluster, d.units(), s8)) {
-            splits = kPortableCluster;
-            var = v8;
-            slots = s8;
-            cluster = true;
-        }
-    }
+    const int var = variant_of(splits);
+    const int slots = slots_of(splits, var);
+    const bool cluster = attn_cluster_fits(d.G, var, splits, d.units(), slots);
     AttnArgs a;
     memset(&a.kmap, 0, sizeof a.kmap);
     memset(&a.vmap, 0, sizeof a.vmap);
