@@ -123,3 +123,44 @@ def test_hybrid_block_stack_sampled(cuda_dev):
     O, _ = G.step(L.Q, L.K, L.V, L.seq_lens, mode=tsa.REUSE, scale=w.scale, k_max=w.k, block=w.block,
                   kreq=kreq, idx_in=idx)
     _check_attn_units(L, idx, O, kreq, w.k, units, w.scale, block=w.block)
+
+
+def test_hybrid_block_stack_all_layers_one_workspace(cuda_dev):
+    """The whole 8-layer hybrid route (F F S R S R S R, 262144 tokens, top 32 of
+    128-token blocks) enqueued back to back on one stream and ONE shared
+    workspace, with no host synchronisation between layers; then every layer's
+    O, and every SELECT layer's block indices, are checked against the oracle
+    on sampled units (Flux Attention's hard per-layer routing; HyLRA's reuse of
+    an earlier layer's blocks)."""
+    w = workloads.HYBRID
+    units = [0, 6, 9, 15]
+    layers = [_gen(w, cuda_dev, seed_offset=li) for li in range(w.layers)]
+    shape = tsa.shape_of(layers[0].Q, layers[0].K)
+    kreq = [w.k] * w.B
+    kr = torch.tensor(kreq, dtype=torch.int32, device=cuda_dev)
+    ws_bytes = max(tsa.workspace_size(shape, w.k, w.block, m) for m in set(w.route))
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=cuda_dev)
+    tsa.workspace_init(ws)
+    Os = [torch.full((w.B, w.Hq, 128), float("nan"), dtype=torch.float32, device=cuda_dev)
+          for _ in range(w.layers)]
+    idx = {li: torch.full((w.B, w.Hkv, w.k), -7, dtype=torch.int32, device=cuda_dev)
+           for li, m in enumerate(w.route) if m == tsa.SELECT}
+    Kmean = {li: G.block_means(layers[li].K, layers[li].seq_lens, w.block) for li in idx}
+    args = []
+    for li, (L, m) in enumerate(zip(layers, w.route)):
+        args.append(tsa.step_args(L.Q, L.K, L.V, L.seq_lens, Os[li], ws, mode=m, scale=w.scale, k_max=w.k,
+                                  block=w.block, k_per_seq=kr, Kmean=Kmean.get(li),
+                                  idx_in=idx[w.reuse_from[li]] if m == tsa.REUSE else None,
+                                  idx_out=idx.get(li)))
+    for a in args:
+        tsa.decode_step(a)
+    tsa.check_device_status(ws)
+    torch.cuda.synchronize()
+    for li, (L, m) in enumerate(zip(layers, w.route)):
+        if m == tsa.FULL:
+            _check_attn_units(L, None, Os[li], None, 0, units, w.scale)
+        elif m == tsa.SELECT:
+            counts = _check_select_units(L, idx[li], Os[li], kreq, w.k, units, w.scale, block=w.block)
+            print(f"hybrid layer {li} (select): {counts}")
+        else:
+            _check_attn_units(L, idx[w.reuse_from[li]], Os[li], kreq, w.k, units, w.scale, block=w.block)

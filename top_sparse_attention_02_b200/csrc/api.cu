@@ -492,12 +492,18 @@ tsa_status tsa_decode_step(const tsa_step_args* a, void* stream) {
             cudaStream_t st = static_cast<cudaStream_t>(stream);
             cudaError_t e;
             if (a->block == 1) {
+                // the attention also counts the scores' first radix digit, so the
+                // top-k that follows starts from that histogram (and zeroes it)
                 e = tsa::launch_attn(a->Q, a->K, a->V, a->seq_lens, nullptr, nullptr, 0, 1, d, a->scale, L.splits,
-                                     partials, counters, a->O, flag_of(a->ws), st, early_in ? 2 : 0, scores);
+                                     partials, counters, a->O, flag_of(a->ws), st, early_in ? 2 : 0, scores, false,
+                                     nullptr, hist);
                 if (e != cudaSuccess) return cuda_fail(e, "tsa_decode_step (full attention)");
-                e = tsa::launch_topk(scores, a->seq_lens, a->k_per_seq, a->k_max, d, 1, a->idx_out, nullptr,
+                e = tsa::launch_topk(scores, a->seq_lens, a->k_per_seq, a->k_max, d, 1, a->idx_out, hist,
                                      flag_of(a->ws), st);
-                if (e != cudaSuccess) return cuda_fail(e, "tsa_decode_step (top-k)");
+                if (e != cudaSuccess) {
+                    cudaMemsetAsync(hist, 0, (size_t)d.units() * tsa::kHistBins * sizeof(uint32_t), st);
+                    return cuda_fail(e, "tsa_decode_step (top-k)");
+                }
                 return TSA_OK;
             }
             e = tsa::launch_score(a->Q, a->Kmean, a->seq_lens, d, a->block, a->scale, scores, hist, flag_of(a->ws), st);

@@ -194,7 +194,8 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
             const int32_t* __restrict__ idx, const int32_t* __restrict__ kreq, int k_max,
             int block, int Hkv, int Ncap, float scale_log2, int S, float* __restrict__ part,
             unsigned* __restrict__ counters, float* __restrict__ O, unsigned* __restrict__ flag, int early,
-            float* __restrict__ sout, float scale, float* __restrict__ lse, int work) {
+            float* __restrict__ sout, float scale, float* __restrict__ lse, int work,
+            uint32_t* __restrict__ hout) {
     using Cfg = AttnCfg<G>;
     extern __shared__ __align__(128) unsigned char smem_raw[];
     // 1024-byte aligned work area (the swizzled layout needs it)
@@ -340,6 +341,12 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
             mbar_arrive(&s_bar[st]);
         }
     };
+    // full attention handing on its top-k: a histogram of the emitted scores'
+    // top 11 key bits (the top-k's first radix digit), past the work area
+    uint32_t* const s_hist = (CONTIG && sout && hout)
+        ? reinterpret_cast<uint32_t*>(smem + work + (CLUSTER ? Cfg::kRecvBytes : 0)) : nullptr;
+    if (s_hist)
+        for (int i = tid; i < kHistBins; i += kAttnThreads) s_hist[i] = 0u;
     if (tid == 0) {
         s_fail = 0;
 #pragma unroll
@@ -521,8 +528,16 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
                     eb = fmaxf(eb, __shfl_xor_sync(0xffffffffu, eb, o2));
                 }
                 if (t4 == 0) {  // scale > 0: scale x max = max of the scaled logits
-                    if (va) su_out[first + r0 + g] = ea * scale;
-                    if (vb) su_out[first + r0 + g + 8] = eb * scale;
+                    if (va) {
+                        const float v = ea * scale;
+                        su_out[first + r0 + g] = v;
+                        if (s_hist) atomicAdd(&s_hist[order_key(v) >> 21], 1u);
+                    }
+                    if (vb) {
+                        const float v = eb * scale;
+                        su_out[first + r0 + g + 8] = v;
+                        if (s_hist) atomicAdd(&s_hist[order_key(v) >> 21], 1u);
+                    }
                 }
             }
         }
@@ -684,6 +699,11 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
         }
     }
     __syncthreads();
+    if (s_hist) {  // this CTA's counts into the unit's histogram (read once this grid is done)
+        uint32_t* hu = hout + (size_t)unit * kHistBins;
+        for (int i = tid; i < kHistBins; i += kAttnThreads)
+            if (const uint32_t c = s_hist[i]) atomicAdd(&hu[i], c);
+    }
     const int nslots = G * 32;  // (head, quad of dims) output slots: thread tid owns slot tid
     const bool has_slot = tid < nslots;
     const int h_me = tid >> 5, qd_me = tid & 31;
@@ -978,7 +998,8 @@ struct AttnArgs {
     float* sout;
     float scale;
     float* lse;
-    int slots;  // the cp.async gather: warp-tile slots its CTAs use
+    int slots;       // the cp.async gather: warp-tile slots its CTAs use
+    uint32_t* hout;  // with sout: the units' top-digit histograms of the emitted scores
 };
 
 template <int G, int STAGES, bool CLUSTER, bool CONTIG, bool ASYNC = false>
@@ -987,7 +1008,8 @@ static cudaError_t attn_launch_g(dim3 grid, cudaStream_t st, const AttnArgs& a) 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = dim3(kAttnThreads);
-    cfg.dynamicSmemBytes = 1024 + work + (CLUSTER ? AttnCfg<G>::kRecvBytes : 0);
+    cfg.dynamicSmemBytes = 1024 + work + (CLUSTER ? AttnCfg<G>::kRecvBytes : 0) +
+                           (a.sout && a.hout ? kHistBins * 4 : 0);
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -999,14 +1021,15 @@ static cudaError_t attn_launch_g(dim3 grid, cudaStream_t st, const AttnArgs& a) 
     cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, attn_kernel<G, STAGES, CLUSTER, CONTIG, ASYNC>, a.kmap, a.vmap, a.q, a.k, a.v, a.lens,
                               a.idx, a.kreq, a.k_max, a.block, a.Hkv, a.Ncap, a.sl2, a.splits, a.partials, a.counters,
-                              a.O, a.flag, a.early, a.sout, a.scale, a.lse, work);
+                              a.O, a.flag, a.early, a.sout, a.scale, a.lse, work, a.hout);
 }
 
 template <int G, int STAGES, bool CLUSTER, bool CONTIG, bool ASYNC = false>
 static cudaError_t attn_configure_one() {
     const void* f = (const void*)attn_kernel<G, STAGES, CLUSTER, CONTIG, ASYNC>;
+    // contiguous tiles may carry the emitted scores' histogram (8 KB more)
     cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         AttnCfg<G>::smem_bytes(STAGES, CLUSTER));
+                                         AttnCfg<G>::smem_bytes(STAGES, CLUSTER) + (CONTIG ? kHistBins * 4 : 0));
     if (e == cudaSuccess && CLUSTER) e = cudaFuncSetAttribute(f, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     return e;
 }
@@ -1070,7 +1093,7 @@ cudaError_t launch_attn(const void* Q, const void* K, const void* V, const int32
                         const int32_t* idx, const int32_t* kreq, int k_max, int block,
                         const Dims& d, float scale, int splits, float* partials,
                         unsigned* counters, float* O, unsigned* flag, cudaStream_t st, int early,
-                        float* scores_out, bool host_kv, float* lse_out) {
+                        float* scores_out, bool host_kv, float* lse_out, uint32_t* hist_out) {
     if (d.units() == 0) return cudaSuccess;
     // scores come with full attention on the tensor-map path only
     if (scores_out && (idx != nullptr || host_kv)) return cudaErrorInvalidValue;
@@ -1146,6 +1169,7 @@ cudaError_t launch_attn(const void* Q, const void* K, const void* V, const int32
     a.scale = scale;
     a.lse = lse_out;
     a.slots = slots;
+    a.hout = scores_out ? hist_out : nullptr;
     dim3 grid(splits, d.units());
     switch (d.G) {
         case 1: e = attn_dispatch<1>(var, cluster, grid, st, a); break;

@@ -101,7 +101,8 @@ cudaError_t launch_attn(const void* Q, const void* K, const void* V, const int32
                         int early = 0,  // 1: lens and k's not written by the previous kernel; 2: nor idx, K, V
                         float* scores_out = nullptr,  // full attention: each row's group-max scaled score
                         bool host_kv = false,         // K, V in mapped page-locked host memory: gather only
-                        float* lse_out = nullptr);    // [units*G]: base-2 log-sum-exp of each head's scaled logits
+                        float* lse_out = nullptr,     // [units*G]: base-2 log-sum-exp of each head's scaled logits
+                        uint32_t* hist_out = nullptr);  // with scores_out: adds the scores' top-digit histograms
 
 cudaError_t launch_copy(const void* src, void* dst, size_t bytes, cudaStream_t st);
 cudaError_t launch_gather(const void* base, size_t base_bytes, const int32_t* rows, int nrows, unsigned* flag,
