@@ -344,6 +344,8 @@ def run_ours(args, rank, world, dev):
     if args.probes:
         res["probes"] = {"handoff": handoff_probe(tsa, w, plan, layers, kreq_t, stream),
                          "overlap": overlap_probe(tsa, w, plan, lens, dev, stream)}
+        if w.block == 1:
+            res["probes"]["sequence_sharded"] = shard_probe(tsa, w, plan, layers, kreq_t, stream)
     return res
 
 
@@ -511,7 +513,7 @@ def offload_probe(tsa, w, plan, layers, Kmean, ws, kreq_t, idx, O, stream, reps=
                     "128-token blocks across the host link; cold L2, median of %d single launches" % reps}
 
 
-def handoff_probe(tsa, w, plan, layers, kreq_t, stream, reps=10):
+def handoff_probe(tsa, w, plan, layers, kreq_t, stream, reps=10, only=None):
     """Layer 0's tensors as a full layer (dense attention), as a full layer that
     hands on its top-k (HyLRA's sensitive layer), and as a SELECT step: each in a
     CUDA graph of `reps` decode steps, warm and after an L2 flush (cold)."""
@@ -532,6 +534,11 @@ def handoff_probe(tsa, w, plan, layers, kreq_t, stream, reps=10):
              "full_handing_on_topk": tsa.step_args(L.Q, L.K, L.V, L.seq_lens, O, ws, mode=tsa.FULL,
                                                    idx_out=ix, **common),
              "select": tsa.step_args(L.Q, L.K, L.V, L.seq_lens, O, ws, mode=tsa.SELECT, idx_out=ix, **common)}
+    if reps == 0:  # --profile: the chosen step twice, untimed
+        for _ in range(2):
+            tsa.decode_step(steps[only], stream)
+        tsa.check_device_status(ws, stream)
+        return {}
     flush = L2Flush(dev)
     f_us = graph_us(flush, stream, reps)
     out = {}
@@ -540,6 +547,76 @@ def handoff_probe(tsa, w, plan, layers, kreq_t, stream, reps=10):
                      "cold_us": graph_us(lambda a=a: (flush(), tsa.decode_step(a, stream)), stream, reps) - f_us}
     tsa.check_device_status(ws, stream)
     out["kv_bytes"] = (L.K.numel() + L.V.numel()) * 2
+    return out
+
+
+def shard_probe(tsa, w, plan, layers, kreq_t, stream, R=2, reps=10):
+    """Layer 0 as a sequence-sharded SELECT step with R shards emulated on one GPU
+    (each shard's calls on its own slice of the cache, one after another; the two
+    all-gathers replaced by writing straight into the stacked buffers, which is
+    what they deliver).  Each call timed alone in a CUDA graph of `reps`
+    launches, warm and after an L2 flush; the whole emulated step is their sum."""
+    L = layers[0]
+    dev = L.Q.device
+    B, Hkv, N = w.B, w.Hkv, w.Ncap
+    bounds = [N * r // R for r in range(R + 1)]
+    k = plan.k_max
+    shards = []
+    for r in range(R):
+        lo, hi = bounds[r], bounds[r + 1]
+        K_r, V_r = L.K[:, :, lo:hi].contiguous(), L.V[:, :, lo:hi].contiguous()
+        lens_r = (L.seq_lens - lo).clamp(0, hi - lo).to(torch.int32)
+        ws = torch.empty(tsa.shard_workspace_size(tsa.shape_of(L.Q, K_r), k, R), dtype=torch.uint8, device=dev)
+        tsa.workspace_init(ws)
+        shards.append((lo, K_r, V_r, lens_r, ws))
+    cs = torch.empty(R, B, Hkv, k, dtype=torch.float32, device=dev)
+    cr = torch.empty(R, B, Hkv, k, dtype=torch.int32, device=dev)
+    idx = torch.empty(B, Hkv, k, dtype=torch.int32, device=dev)
+    O_parts = torch.empty(R, B, w.Hq, 128, dtype=torch.float32, device=dev)
+    lse = torch.empty(R, B, w.Hq, dtype=torch.float32, device=dev)
+    O = torch.empty(B, w.Hq, 128, dtype=torch.float32, device=dev)
+    shape = tsa.shape_of(L.Q, L.K)
+    lo0, K0, V0, l0, ws0 = shards[0]
+    calls = {
+        "shard_select (one shard)": lambda: tsa.shard_select(L.Q, K0, l0, kreq_t, k, w.scale, lo0, cs[0], cr[0],
+                                                             ws0, stream),
+        "shard_merge": lambda: tsa.shard_merge(cs, cr, shape, kreq_t, k, idx, ws0, stream),
+        "shard_attend (one shard)": lambda: tsa.shard_attend(L.Q, K0, V0, l0, idx, kreq_t, k, lo0, w.scale,
+                                                             O_parts[0], lse[0], ws0, stream),
+        "shard_combine": lambda: tsa.shard_combine(O_parts, lse, shape, O, stream),
+    }
+    for r, (lo, K_r, V_r, lens_r, ws) in enumerate(shards):  # fill every shard's candidates and parts once
+        with torch.cuda.stream(stream):
+            tsa.shard_select(L.Q, K_r, lens_r, kreq_t, k, w.scale, lo, cs[r], cr[r], ws, stream)
+    with torch.cuda.stream(stream):
+        tsa.shard_merge(cs, cr, shape, kreq_t, k, idx, ws0, stream)
+    for r, (lo, K_r, V_r, lens_r, ws) in enumerate(shards):
+        with torch.cuda.stream(stream):
+            tsa.shard_attend(L.Q, K_r, V_r, lens_r, idx, kreq_t, k, lo, w.scale, O_parts[r], lse[r], ws, stream)
+    if reps == 0:  # --profile: every shard's calls once more, untimed
+        for r, (lo, K_r, V_r, lens_r, ws) in enumerate(shards):
+            tsa.shard_select(L.Q, K_r, lens_r, kreq_t, k, w.scale, lo, cs[r], cr[r], ws, stream)
+        tsa.shard_merge(cs, cr, shape, kreq_t, k, idx, ws0, stream)
+        for r, (lo, K_r, V_r, lens_r, ws) in enumerate(shards):
+            tsa.shard_attend(L.Q, K_r, V_r, lens_r, idx, kreq_t, k, lo, w.scale, O_parts[r], lse[r], ws, stream)
+        tsa.shard_combine(O_parts, lse, shape, O, stream)
+        stream.synchronize()
+        return {}
+    flush = L2Flush(dev)
+    f_us = graph_us(flush, stream, reps)
+    out = {}
+    for name, fn in calls.items():
+        out[name] = {"warm_us": graph_us(fn, stream, reps),
+                     "cold_us": graph_us(lambda fn=fn: (flush(), fn()), stream, reps) - f_us}
+    for _, _, _, _, ws in shards:
+        tsa.check_device_status(ws, stream)
+    per_shard = out["shard_select (one shard)"]["cold_us"] + out["shard_attend (one shard)"]["cold_us"]
+    out["shards"] = R
+    out["exchanged_bytes"] = {"candidates": R * B * Hkv * k * 8, "parts": R * B * w.Hq * 129 * 4}
+    out["step_cold_us_one_gpu_emulation"] = (per_shard * R + out["shard_merge"]["cold_us"] +
+                                             out["shard_combine"]["cold_us"])
+    out["note"] = ("one GPU runs every shard in turn; on R GPUs the shards' select and attend calls run at once "
+                   "and two all-gathers of the exchanged bytes are added")
     return out
 
 
@@ -557,6 +634,9 @@ def overlap_probe(tsa, w, plan, lens, dev, stream, n_layers=32, keep=0.7, reps=1
     M = torch.empty(n_layers, n_layers, dtype=torch.float64, device=dev)
     ws = torch.zeros(256, dtype=torch.uint8, device=dev)
     tsa.index_overlap(idx, counts, M, ws, stream)
+    if reps == 0:  # --profile: one launch, untimed
+        stream.synchronize()
+        return {}
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         e0.record(stream)
@@ -852,6 +932,36 @@ def launch_ranks(n, argv):
     return subprocess.call(cmd)
 
 
+def profile_case(args, dev):
+    """--profile NAME: one call path of the library, run twice eagerly and not
+    timed, so that a profiler capture (-k <kernel> -s 1 -c 1) lands on a known
+    launch: "handoff" (a full layer handing on its top-k: the dense attention
+    writing scores and their histogram, then the top-k), "overlap" (the layer
+    overlap matrix), "shard" (the four sequence-sharded calls, two shards)."""
+    from top_sparse_attention_02_b200 import binding as tsa
+
+    w = workload_of(args)
+    lens = workload_lens(w)
+    plan = Plan(w, lens)
+    stream = torch.cuda.Stream(device=dev)
+    kreq_t = torch.tensor(plan.kreq, dtype=torch.int32, device=dev)
+    if args.profile == "overlap":
+        for _ in range(2):
+            overlap_probe(tsa, w, plan, lens, dev, stream, reps=0)
+    else:
+        from top_sparse_attention_02_b200 import inputs
+
+        L0 = inputs.decode_layer(w.B, w.Hq, w.Hkv, w.Ncap, lens, plant_frac=w.plant_frac, seed=w.seed, device=dev)
+        if args.profile == "handoff":
+            handoff_probe(tsa, w, plan, [L0], kreq_t, stream, reps=0, only="full_handing_on_topk")
+        elif args.profile == "shard":
+            shard_probe(tsa, w, plan, [L0], kreq_t, stream, reps=0)
+        else:
+            raise SystemExit(f"--profile: unknown case {args.profile!r}")
+    torch.cuda.synchronize()
+    print(json.dumps({"profile": args.profile, "workload": w.name}), flush=True)
+
+
 def dry_run(args, rank, world):
     """The multi-rank plumbing alone, on the CPU (gloo, no CUDA): every rank takes
     a stand-in time, the max goes over the ranks, rank 0 prints the line."""
@@ -893,6 +1003,8 @@ def main():
                     help="shrink the workload's context to this many tokens (profiler captures only)")
     ap.add_argument("--dry-run", action="store_true",
                     help="only the rank plumbing (start, barrier, max over ranks) on the CPU over gloo")
+    ap.add_argument("--profile", default="",
+                    help="run one call path twice, untimed, for a profiler capture: handoff | overlap | shard")
     args = ap.parse_args()
 
     if "WORLD_SIZE" not in os.environ and args.gpus > 1:
@@ -917,6 +1029,9 @@ def main():
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    if args.profile:
+        profile_case(args, dev)
+        return
     if world > 1:
         import datetime
 
