@@ -220,6 +220,8 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
         len = __ldcg(lens + b);
         if (kreq) kreq_b = __ldcg(kreq + b);
     }
+    // Q's lines into L2 while the previous kernel finishes (G x 256 bytes)
+    if (tid < 2 * G) prefetch_l2(Q + (size_t)unit * G * kD + tid * 64);
     if (early < 2) {
         griddep_wait();
         griddep_launch();
@@ -786,7 +788,10 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
             }
             if (live && j == 0) {
                 float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (den > 0.f) r = make_float4(num.x / den, num.y / den, num.z / den, num.w / den);
+                if (den > 0.f) {
+                    const float inv = __frcp_rn(den);  // one rounding more than a division: ~1e-7 relative
+                    r = make_float4(num.x * inv, num.y * inv, num.z * inv, num.w * inv);
+                }
                 *reinterpret_cast<float4*>(O + ((size_t)unit * G + h) * kD + 4 * qd) = r;
                 if (lse && qd == 0) lse[(size_t)unit * G + h] = den > 0.f ? M + log2f(den) : -INFINITY;
             }

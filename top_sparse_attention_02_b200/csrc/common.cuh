@@ -83,6 +83,11 @@ __device__ __forceinline__ void halfwarp_reduce_scatter16(float (&v)[16], int c)
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
 __device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
 
+// A hint that brings the 128-byte line holding p into L2; no data returns, so
+// it may be issued before waiting on the kernel that writes p (L2 is where that
+// kernel's writes land: the read after the wait sees them).
+__device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];\n" ::"l"(p)); }
+
 __device__ __forceinline__ int clamp_len(int len, int Ncap, unsigned* flag) {
     if (len < 0 || len > Ncap) {
         atomicOr(flag, kFlagBounds);

@@ -185,6 +185,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16* _
     };
     int issued = 0;  // warp 0, lane 0: tiles requested so far
     if (early) {
+        if (tid >= 64 && tid < 64 + 2 * G) prefetch_l2(Q + (size_t)unit * G * kD + (tid - 64) * 64);  // Q into L2
         // the first stages' loads before waiting on the previous kernel
         __syncthreads();  // the barriers are initialised
         if (warp == 0 && lane == 0)
