@@ -367,17 +367,33 @@ def test_block_select_steps_share_one_workspace(cuda_dev):
         check_output(O.cpu().numpy(), ref, f"block step with seed {seed}")
 
 
-@pytest.mark.parametrize("case", ["plain", "tied_top", "k_near_len"])
+@pytest.mark.parametrize("case", ["plain", "tied_top", "k_near_len", "tie_cut", "tie_overflow"])
 def test_decode_step_topk_from_the_scorers_histogram(cuda_dev, case):
     """Inside a decode step the top-k of long units starts from the scorer's
     first-digit histogram (a cluster per unit, lists in registers and shared
     memory).  Its paths: the plain one; 7000 identical top keys (exact ties at T:
     the lists overflow and every later pass runs over all keys); k one short of
-    the length.  Two steps on one workspace check that the histogram is zeroed."""
+    the length; the k-th row's key copied to 20 other rows (exact ties at the
+    boundary, cut by the lowest rows across the cluster's CTAs); the same with
+    300 copies (more keys sharing the first two digits than a CTA sends: the
+    histogram fallback).  Two steps on one workspace check that the histogram
+    is zeroed."""
     B, Hq, Hkv, N = 2, 16, 4, 20000
     lens = [20000, 15000]
     L = layer(B, Hq, Hkv, N, lens, seed=71)
-    if case == "tied_top":
+    if case in ("tie_cut", "tie_overflow"):
+        kreq, k_max = [400, 300], 400
+        S0 = oracle.scores(L.Q, L.K, L.seq_lens, SCALE)
+        rng = np.random.default_rng(7)
+        ncopy = 20 if case == "tie_cut" else 300
+        for b in range(B):
+            n = lens[b]
+            for h in range(Hkv):
+                order = np.lexsort((np.arange(n), -S0[b, h, :n]))
+                r = int(order[kreq[b] - 1])  # the k-th row
+                dst = rng.choice(n, size=ncopy, replace=False)
+                L.K[b, h, dst] = L.K[b, h, r].clone()
+    elif case == "tied_top":
         S0 = oracle.scores(L.Q, L.K, L.seq_lens, SCALE)
         for b in range(B):
             for h in range(Hkv):
@@ -739,3 +755,45 @@ def test_sequence_sharded_select_on_one_gpu(cuda_dev, case):
         ref_r = oracle.attn(L.Q, L.K[:, :, lo:lo + K_r.shape[2]].contiguous(), L.V[:, :, lo:lo + K_r.shape[2]].contiguous(),
                             lens_r.cpu(), own, kreq, k_max, 1, SCALE)
         check_output(O_parts[r].cpu().numpy(), ref_r, f"{case} shard {r} part")
+
+
+def test_sequence_sharded_step_through_nccl(cuda_dev):
+    """shard.sharded_select_step on a real NCCL process group (one rank on this
+    GPU: every all-gather is a device NCCL collective, nothing waits on another
+    rank), against the one-GPU SELECT step and the oracle."""
+    import os
+    import socket
+
+    import torch.distributed as dist
+
+    from top_sparse_attention_02_b200 import shard
+
+    B, Hq, Hkv, N, lens, kreq = 2, 32, 8, 9000, [9000, 5000], [300, 200]
+    k_max = max(kreq)
+    L = layer(B, Hq, Hkv, N, lens, seed=141, tail_fill=float("nan"))
+    Q, K, V, ln = G.to_dev(L, cuda_dev)
+    kr = torch.tensor(kreq, dtype=torch.int32, device=cuda_dev)
+    _, idx_one = G.step(Q, K, V, ln, mode=tsa.SELECT, scale=SCALE, k_max=k_max, kreq=kreq)
+    with socket.socket() as so:
+        so.bind(("127.0.0.1", 0))
+        port = so.getsockname()[1]
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+
+    dist.init_process_group("nccl", rank=0, world_size=1, timeout=datetime.timedelta(seconds=60),
+                            device_id=cuda_dev)
+    try:
+        ws = torch.empty(tsa.shard_workspace_size(tsa.shape_of(Q, K), k_max, 1), dtype=torch.uint8,
+                         device=cuda_dev)
+        tsa.workspace_init(ws)
+        O = torch.full((B, Hq, 128), float("nan"), dtype=torch.float32, device=cuda_dev)
+        idx = torch.full((B, Hkv, k_max), -7, dtype=torch.int32, device=cuda_dev)
+        stream = torch.cuda.Stream(device=cuda_dev)
+        shard.sharded_select_step(Q, K, V, ln, kr, k_max, SCALE, 0, O, idx, ws, stream=stream)
+        stream.synchronize()
+        tsa.check_device_status(ws)
+    finally:
+        dist.destroy_process_group()
+    assert torch.equal(idx, idx_one)
+    ref = oracle.attn(L.Q, L.K, L.V, L.seq_lens, idx.cpu().numpy(), kreq, k_max, 1, SCALE)
+    check_output(O.cpu().numpy(), ref, "sharded step over NCCL")
