@@ -374,10 +374,11 @@ def test_decode_step_topk_from_the_scorers_histogram(cuda_dev, case):
     memory).  Its paths: the plain one; 7000 identical top keys (exact ties at T:
     the lists overflow and every later pass runs over all keys); k one short of
     the length; the k-th row's key copied to 20 other rows (exact ties at the
-    boundary, cut by the lowest rows across the cluster's CTAs); the same with
-    300 copies (more keys sharing the first two digits than a CTA sends: the
-    histogram fallback).  Two steps on one workspace check that the histogram
-    is zeroed."""
+    boundary, cut by the lowest rows across the cluster's CTAs: rank 0 ranks the
+    few keys sharing the first two digits directly); the same with 300 copies
+    (more than 64 keys share the first two digits: the last digit by a
+    histogram pass).  Two steps on one workspace check that the histogram is
+    zeroed."""
     B, Hq, Hkv, N = 2, 16, 4, 20000
     lens = [20000, 15000]
     L = layer(B, Hq, Hkv, N, lens, seed=71)
