@@ -140,11 +140,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity, unsign
     if (flag) atomicOr(flag, kFlagTimeout);
     return false;
 }
-// 1-D bulk copy (TMA engine) global -> this CTA's shared memory, completing on `bar`
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned bytes, uint64_t* bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
-                 ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
-}
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
 __device__ __forceinline__ void ldsm_x4(unsigned addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];\n"
@@ -180,11 +175,11 @@ __device__ __forceinline__ int roff(int row, int chunk) { return row * kRowStrid
 
 // CONTIG: every tile is 128 consecutive cache rows (a full-attention range, or
 // one 128-token block in block mode) and arrives by 2-D TMA tensor loads in the
-// 128-byte-swizzled layout (4 loads per tile); otherwise each row is its own
-// 256-byte bulk copy into rows padded to 272 bytes.
+// 128-byte-swizzled layout (4 loads per tile) into a ring of STAGES tiles;
+// otherwise (a gather) rows are padded to 272 bytes.
 // ASYNC (gather only): rows are copied straight into shared memory (cp.async)
-// into a per-warp ring of STAGES tiles; with STAGES == 1 (every CTA's range is
-// one tile) two CTAs fit an SM.  Otherwise (K and V in mapped host memory) each
+// into per-warp slots, a ring of STAGES tiles; launched two CTAs an SM when the
+// slots a CTA uses allow it.  Otherwise (K and V in mapped host memory) each
 // warp loads its rows into registers one tile ahead and stores them.
 template <int G, int STAGES, bool CLUSTER, bool CONTIG, bool ASYNC>
 __global__ void __launch_bounds__(kAttnThreads, ASYNC ? 2 : 1)
