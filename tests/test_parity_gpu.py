@@ -519,6 +519,22 @@ def test_index_overlap_random_layers(cuda_dev, keep):
         assert (M[np.tril_indices(6)] == 1.0).all()
 
 
+@pytest.mark.parametrize("k_max", [33, 256])
+def test_index_overlap_short_lists_a_warp_a_unit(cuda_dev, k_max):
+    """Lists of at most 256 entries take the warp-a-unit kernel: 150 units (three
+    rounds of 64, the last partial), ragged lengths, empty and full units; counts
+    exact and M against the oracle."""
+    rng = np.random.default_rng(k_max)
+    units = 150
+    n = rng.integers(1, 2000, units).tolist()
+    n[7] = 0
+    k = [int(min(x, rng.integers(1, k_max + 1))) for x in n]
+    k[9] = k_max
+    n[9] = max(n[9], k_max)
+    idx = inputs.layer_index_lists(5, n, k, k_max, 0.6, seed=21).to(cuda_dev)
+    _check_overlap(idx)
+
+
 def test_index_overlap_long_lists_and_degenerate_sizes(cuda_dev):
     """Lists longer than the shared-memory stage (13000 rows of 40000), one layer,
     no units, and k_max = 0."""

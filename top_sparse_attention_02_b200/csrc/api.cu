@@ -288,14 +288,21 @@ tsa_status tsa_shard_merge(const float* cand_scores, const int32_t* cand_rows, i
     int32_t* pk_rows = reinterpret_cast<int32_t*>(w + S.pk_rows);
     int32_t* n_cand = reinterpret_cast<int32_t*>(w + S.n_cand);
     int32_t* pos = reinterpret_cast<int32_t*>(w + S.pos);
+    // the packing counts the candidates' first radix digit into the
+    // histograms (zero here: every call that used them zeroed them), and the
+    // top-k over the candidates starts from it
+    uint32_t* hist = reinterpret_cast<uint32_t*>(w + S.front.hist);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e = tsa::launch_merge_pack(cand_scores, cand_rows, n_shards, d.units(), d.Hkv, k_max, pk_scores,
-                                           pk_rows, n_cand, flag_of(ws), st);
+                                           pk_rows, n_cand, hist, flag_of(ws), st);
     if (e != cudaSuccess) return cuda_fail(e, "tsa_shard_merge (pack)");
     tsa::Dims dc = d;
     dc.Ncap = (int)width;  // the candidates are the rows of this top-k
-    e = tsa::launch_topk(pk_scores, n_cand, k_per_seq, k_max, dc, 1, pos, nullptr, flag_of(ws), st);
-    if (e != cudaSuccess) return cuda_fail(e, "tsa_shard_merge (top-k)");
+    e = tsa::launch_topk(pk_scores, n_cand, k_per_seq, k_max, dc, 1, pos, hist, flag_of(ws), st);
+    if (e != cudaSuccess) {
+        cudaMemsetAsync(hist, 0, (size_t)d.units() * tsa::kHistBins * sizeof(uint32_t), st);
+        return cuda_fail(e, "tsa_shard_merge (top-k)");
+    }
     e = tsa::launch_merge_map(pos, pk_rows, d.units(), (int)width, k_max, idx, st);
     if (e != cudaSuccess) return cuda_fail(e, "tsa_shard_merge (rows)");
     return TSA_OK;

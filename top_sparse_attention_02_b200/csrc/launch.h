@@ -42,9 +42,11 @@ cudaError_t launch_index_overlap(const int32_t* idx, int L, int units, int k_max
 constexpr int kMaxShards = 64;
 cudaError_t launch_shard_pack(const float* scores, int rows_cap, int units, int k_max, int row0, int32_t* cand_rows,
                               float* cand_scores, unsigned* flag, cudaStream_t st);
+// also adds the packed scores' first radix digit into hist [units][kHistBins]
+// (zero on entry; the top-k over the packed candidates reads and zeroes it)
 cudaError_t launch_merge_pack(const float* cand_scores, const int32_t* cand_rows, int R, int units, int Hkv,
-                              int k_max, float* pk_scores, int32_t* pk_rows, int32_t* n_cand, unsigned* flag,
-                              cudaStream_t st);
+                              int k_max, float* pk_scores, int32_t* pk_rows, int32_t* n_cand, uint32_t* hist,
+                              unsigned* flag, cudaStream_t st);
 cudaError_t launch_merge_map(const int32_t* pos, const int32_t* pk_rows, int units, int width, int k_max,
                              int32_t* idx, cudaStream_t st);
 cudaError_t launch_localize(const int32_t* idx, int units, int k_max, int row0, int rows_cap, int32_t* local,

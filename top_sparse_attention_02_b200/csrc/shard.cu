@@ -79,13 +79,15 @@ __global__ void __launch_bounds__(kShThreads) shard_pack_kernel(const float* __r
 
 // the R shards' candidates of a unit (each list: valid rows, then -1) packed
 // one after another, then padded with (-inf, -1); CTA x writes packed
-// positions [x*256, x*256 + 256)
+// positions [x*256, x*256 + 256), and counts their scores' first radix digit
+// into the unit's histogram for the top-k over them
 __global__ void __launch_bounds__(kShThreads) merge_pack_kernel(const float* __restrict__ cand_scores,
                                                                const int32_t* __restrict__ cand_rows, int R,
                                                                int units, int Hkv, int k_max,
                                                                float* __restrict__ pk_scores,
                                                                int32_t* __restrict__ pk_rows,
-                                                               int32_t* __restrict__ n_cand, unsigned* flag) {
+                                                               int32_t* __restrict__ n_cand, uint32_t* __restrict__ hist,
+                                                               unsigned* flag) {
     __shared__ int s_off[kMaxShards + 1];
     __shared__ int s_red[33];
     const int u = blockIdx.y, tid = threadIdx.x;
@@ -131,8 +133,10 @@ __global__ void __launch_bounds__(kShThreads) merge_pack_kernel(const float* __r
     int r = 0;
     while (s_off[r + 1] <= p) ++r;  // the shard of packed position p
     const size_t src = ((size_t)r * units + u) * k_max + (p - s_off[r]);
-    ps[p] = cand_scores[src];
+    const float sc = cand_scores[src];
+    ps[p] = sc;
     pr[p] = cand_rows[src];
+    atomicAdd(&hist[(size_t)u * kHistBins + (order_key(sc) >> 21)], 1u);
 }
 
 __global__ void __launch_bounds__(kShThreads) merge_map_kernel(const int32_t* __restrict__ pos,
@@ -200,12 +204,12 @@ cudaError_t launch_shard_pack(const float* scores, int rows_cap, int units, int 
 }
 
 cudaError_t launch_merge_pack(const float* cand_scores, const int32_t* cand_rows, int R, int units, int Hkv,
-                              int k_max, float* pk_scores, int32_t* pk_rows, int32_t* n_cand, unsigned* flag,
-                              cudaStream_t st) {
+                              int k_max, float* pk_scores, int32_t* pk_rows, int32_t* n_cand, uint32_t* hist,
+                              unsigned* flag, cudaStream_t st) {
     if (units == 0) return cudaSuccess;
     if (k_max == 0) return cudaSuccess;
     merge_pack_kernel<<<dim3(ceil_div(R * k_max, kShThreads), units), kShThreads, 0, st>>>(
-        cand_scores, cand_rows, R, units, Hkv, k_max, pk_scores, pk_rows, n_cand, flag);
+        cand_scores, cand_rows, R, units, Hkv, k_max, pk_scores, pk_rows, n_cand, hist, flag);
     note_launch();
     return cudaGetLastError();
 }
