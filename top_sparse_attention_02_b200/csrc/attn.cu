@@ -33,22 +33,35 @@
 //   S^T = K Q^T    (8 k-steps of 16 dims: 8 MMAs; K fragments by ldmatrix,
 //                  Q^T fragments held in registers for the whole kernel),
 //   online softmax per head on the S^T fragments (fp32, log2 units),
-//   O^T += V^T P^T (8 m-tiles of 16 dims: 16 MMAs with P split as bf16 hi +
-//                  bf16 lo so that the weights keep ~16 bits; V^T fragments by
+//   O^T += V^T P^T (8 m-tiles of 16 dims, P split as bf16 hi + bf16 lo so
+//                  that the weights keep ~16 bits; V^T fragments by
 //                  ldmatrix.trans, P^T fragments from the S^T accumulator by
-//                  movmatrix.trans).
+//                  movmatrix.trans).  With g <= 4 the n-tile's columns
+//                  G .. 2G-1 repeat the heads (Q^T column c is head c mod G),
+//                  and carry lo while columns 0 .. G-1 carry hi: one MMA an
+//                  m-tile (8), the two column sets summed once at the end.
+//                  With g = 8 there is no spare column: two MMAs an m-tile.
+// A warp-tile is a chain of dependent steps (on sm_100a: ~20 cycles an
+// mma.sync, ~30 a shuffle, an exp2 or a shared load), so when a CTA's whole
+// range is in its cp.async ring, each warp takes all its 16-row groups in one
+// pass: their S^T products are independent MMA chains, one pair of row
+// reductions serves them all, and the PV products accumulate in turn.
 // With the heads as M instead (padded to 16), each 16 rows took twice the
 // MMAs and twice the accumulator registers.  tcgen05's smallest M is 64, so
 // a GQA group would leave most of every tcgen05 MMA idle.  The 8 warps are merged at the end into
 // the CTA's partial (M, L, acc[128]) per head.  When a unit has at most 8
 // splits and every unit's cluster can be resident at once, the splits of a unit
-// form one thread-block cluster: each CTA pushes the slices of its partial to
-// the CTAs that own those output slices (posted distributed-shared-memory
-// stores), one cluster barrier, and each CTA combines its slice locally (no
-// scratch).  Otherwise (more splits, or more clusters than fit: a B200 holds
-// only 15 clusters of 8 CTAs of ~226 KB) each CTA writes its partial to the
-// workspace and the last CTA of the unit to arrive (an atomic counter in the
-// workspace, reset by that CTA) combines the partials into O.
+// form one thread-block cluster: output slot q (4 dims of one head) belongs
+// to CTA q / ceil(32g / S); each CTA sends every owner its slots of the
+// partial and its (M, L) per head with st.async, which counts the bytes on the
+// owner's mbarrier, so an owner waits for exactly the bytes it needs (no
+// cluster-wide barrier, ~0.5 us less than posted stores and one), then
+// combines its slots (no scratch).  Otherwise (more splits, or more clusters
+// than fit: a B200 holds only 15 clusters of 8 CTAs of ~226 KB) each CTA
+// writes its partial to the workspace and the last CTA of the unit to arrive
+// (an atomic counter in the workspace, reset by that CTA) combines the
+// partials into O.  (Each warp sending its own partial to the owners, with
+// no merge inside the CTA, moved 8x the bytes between SMs: slower.)
 //
 // Programmatic dependent launch: the kernel may start while the kernel before
 // it on the stream is still running.  It waits for it (griddepcontrol.wait)
@@ -59,15 +72,13 @@
 // just before does not write them), so that a reuse layer's gather overlaps the
 // end of the layer before it.  Q, the workspace and O are touched only after
 // the wait.
-#include <cooperative_groups.h>
 #include <cstring>
+#include <type_traits>
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
 #include "launch.h"
-
-namespace cg = cooperative_groups;
 
 namespace tsa {
 
@@ -92,6 +103,7 @@ constexpr long kWaitSpins = 1L << 22;  // bounded mbarrier wait (then flag, drai
 #else
 constexpr long kWaitSpins = TSA_WAIT_SPINS;  // a debug build's short limit
 #endif
+constexpr long kRecvSpins = 1L << 22;  // bounded wait for the cluster peers' partials
 #ifdef TSA_DEBUG_KNOBS
 // Debug build only (never in the product library): the contiguous tile (of CTA
 // (0, 0)) whose loads are left out, so that the wait on it runs out; -1: none.
@@ -100,14 +112,23 @@ __device__ int g_debug_attn_skip_tile = -1;
 
 template <int G>
 struct AttnCfg {
-    // cluster combine: S sources x ceil(G*32/S) float4 output slots per owner
-    static constexpr int kRecvBytes = (G * 32 + kClusterMax) * 16;
+    // receive area of a cluster of S CTAs: from each source CTA, its partial's
+    // float4 slots that this CTA owns (ceil(32G / S) at most: 4 dims of one
+    // head a slot), then its (M, L) per head
+    __host__ __device__ static constexpr int recv_bytes(int S) {
+        return S <= 1 ? 0 : S * ((G * 32 + S - 1) / S) * 16 + S * G * 8;
+    }
+    static constexpr int recv_max() {
+        int m = 0;
+        for (int S = 2; S <= kClusterMax; ++S) m = recv_bytes(S) > m ? recv_bytes(S) : m;
+        return m;
+    }
     static constexpr int kAccBytes = kAttnWarps * G * kAccStride * 4;
     static constexpr int work_bytes(int stages) {
         return stages * kStageBytes > kAccBytes ? stages * kStageBytes : kAccBytes;
     }
     static constexpr int smem_bytes(int stages, bool cluster) {
-        return 1024 /* alignment slack */ + work_bytes(stages) + (cluster ? kRecvBytes : 0);
+        return 1024 /* alignment slack */ + work_bytes(stages) + (cluster ? recv_max() : 0);
     }
     // the cp.async gather with `slots` warp-tile slots in use
     static constexpr int slot_work_bytes(int slots) {
@@ -129,9 +150,9 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, unsigned by
 // Wait for the phase with the given parity; gives up after kWaitSpins polls,
 // raising the timeout flag, and returns false (the CTA then stops its tile loop;
 // see the contiguous-tile loop).  flag == nullptr: no flag (a drain wait).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity, unsigned* flag) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity, unsigned* flag, long spins = kWaitSpins) {
     const unsigned a = smem_u32(bar);
-    for (long i = 0; i < kWaitSpins; ++i) {
+    for (long i = 0; i < spins; ++i) {
         unsigned done;
         asm volatile("{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
                      : "=r"(done) : "r"(a), "r"(parity) : "memory");
@@ -141,6 +162,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity, unsign
     return false;
 }
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
+__device__ __forceinline__ void st_async_f2(unsigned dst, float x, float y, unsigned bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];\n"
+                 ::"r"(dst), "f"(x), "f"(y), "r"(bar) : "memory");
+}
+// the address of the same shared-memory location in cluster CTA `rank`
+__device__ __forceinline__ unsigned cluster_addr(unsigned local, unsigned rank) {
+    unsigned r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(local), "r"(rank));
+    return r;
+}
+// 16 bytes into another cluster CTA's shared memory, counted on that CTA's
+// mbarrier (complete_tx): its wait ends once every byte it expects has landed
+__device__ __forceinline__ void st_async_f4(unsigned dst, float x, float y, float z, float w, unsigned bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];\n"
+                 ::"r"(dst), "f"(x), "f"(y), "f"(z), "f"(w), "r"(bar) : "memory");
+}
 __device__ __forceinline__ void ldsm_x4(unsigned addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];\n"
                  : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
@@ -173,6 +210,182 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 // byte offset of 16-byte chunk `chunk` of row `row` in a tile of padded rows
 __device__ __forceinline__ int roff(int row, int chunk) { return row * kRowStride + (chunk << 4); }
 
+// The two contractions of flash decoding on one warp's rows, R groups of 16
+// (group q: K at kt[q], V at vt[q], each seen as rows r0 .. r0 + 15 of a tile;
+// bit x of vm[q]: row r0 + x of the group is in the set), with one online-
+// softmax step over all of them.  The groups' S^T products are independent
+// MMA chains and share one pair of row reductions, and the PV products of all
+// groups accumulate in turn, so R groups cost far less than R calls of one.
+// su_out (CONTIG, R = 1: full attention that also emits its top-k): the scores
+// of the group's rows -- scale x the max over the group's heads of q.k, the
+// criterion a SELECT layer scores by -- written as S is formed (row first +
+// r0 + x), with their top-digit histogram in s_hist.
+template <int G, int R, bool CONTIG>
+__device__ __forceinline__ void warp_rows(const unsigned (&kt)[R], const unsigned (&vt)[R], const uint32_t (&vm)[R],
+                                          const uint32_t (&qa)[8][2], float (&o)[8][4], float (&m_run)[2],
+                                          float (&l_run)[2], float scale_log2, int lane, int r0, float* su_out,
+                                          int first, float scale, uint32_t* s_hist) {
+    const int g = lane >> 2, t4 = lane & 3;
+    // byte offset of 16-byte chunk c of tile row r (padded rows, or the
+    // 128-byte swizzle of the TMA tensor loads: two 64-dim halves)
+    auto off = [&](int r, int c) -> unsigned {
+        if constexpr (CONTIG)
+            return (unsigned)((c >> 3) * 64 * kTileRows * 2 + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+        else
+            return (unsigned)roff(r, c);
+    };
+    // ---- S^T = K Q^T over each group's 16 rows (M = rows, N = heads)
+    // c[q][0], [1]: row g, heads 2t4, 2t4 + 1; [2], [3]: row g + 8
+    float c[R][4];
+    {
+        float sc[R][2][4];  // even / odd k-steps: two chains a group
+#pragma unroll
+        for (int q = 0; q < R; ++q)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sc[q][0][e] = sc[q][1][e] = 0.f;
+        const int m = lane >> 3, i = lane & 7;  // ldmatrix: matrix m, row i
+        const int row = r0 + (m & 1) * 8 + i;    // rows +8 (m&1), dims +8 (m>>1)
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+#pragma unroll
+            for (int q = 0; q < R; ++q) {
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4(kt[q] + off(row, 2 * ks + (m >> 1)), a0, a1, a2, a3);
+                mma_bf16(sc[q][ks & 1], a0, a1, a2, a3, qa[ks][0], qa[ks][1]);
+            }
+#pragma unroll
+        for (int q = 0; q < R; ++q)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) c[q][e] = sc[q][0][e] + sc[q][1][e];
+    }
+    const int h0 = 2 * t4, h1 = 2 * t4 + 1;  // this lane's two heads (columns)
+    if constexpr (CONTIG && R == 1) {
+        const bool va = (vm[0] >> g) & 1u, vb = (vm[0] >> (g + 8)) & 1u;
+        if (su_out) {  // uniform: each row's max over the heads < G, across the 4 lanes of the row
+            float ea = fmaxf(h0 < G ? c[0][0] : -INFINITY, h1 < G ? c[0][1] : -INFINITY);
+            float eb = fmaxf(h0 < G ? c[0][2] : -INFINITY, h1 < G ? c[0][3] : -INFINITY);
+#pragma unroll
+            for (int o2 = 1; o2 < 4; o2 <<= 1) {
+                ea = fmaxf(ea, __shfl_xor_sync(0xffffffffu, ea, o2));
+                eb = fmaxf(eb, __shfl_xor_sync(0xffffffffu, eb, o2));
+            }
+            if (t4 == 0) {  // scale > 0: scale x max = max of the scaled logits
+                if (va) {
+                    const float v = ea * scale;
+                    su_out[first + r0 + g] = v;
+                    if (s_hist) atomicAdd(&s_hist[order_key(v) >> 21], 1u);
+                }
+                if (vb) {
+                    const float v = eb * scale;
+                    su_out[first + r0 + g + 8] = v;
+                    if (s_hist) atomicAdd(&s_hist[order_key(v) >> 21], 1u);
+                }
+            }
+        }
+    }
+    // ---- online softmax per head (columns of S^T): rows not in the set are -inf
+    float z[R][4];
+    float mt[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+    for (int q = 0; q < R; ++q) {
+        const bool va = (vm[q] >> g) & 1u, vb = (vm[q] >> (g + 8)) & 1u;  // rows g, g + 8 in the set
+        z[q][0] = va ? c[q][0] * scale_log2 : -INFINITY;
+        z[q][1] = va ? c[q][1] * scale_log2 : -INFINITY;
+        z[q][2] = vb ? c[q][2] * scale_log2 : -INFINITY;
+        z[q][3] = vb ? c[q][3] * scale_log2 : -INFINITY;
+        mt[0] = fmaxf(mt[0], fmaxf(z[q][0], z[q][2]));
+        mt[1] = fmaxf(mt[1], fmaxf(z[q][1], z[q][3]));
+    }
+#pragma unroll
+    for (int o2 = 4; o2 < 32; o2 <<= 1) {  // over the 8 lanes of a t4 (the rows)
+        mt[0] = fmaxf(mt[0], __shfl_xor_sync(0xffffffffu, mt[0], o2));
+        mt[1] = fmaxf(mt[1], __shfl_xor_sync(0xffffffffu, mt[1], o2));
+    }
+    float alpha[2], p[R][4];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const float mnew = fmaxf(m_run[j], mt[j]);
+        // a head with no finite logit yet keeps m = -inf, alpha = 0 and p = 0
+        alpha[j] = m_run[j] == -INFINITY ? 0.f : exp2f(m_run[j] - mnew);
+        m_run[j] = mnew;
+    }
+    float ps[2] = {0.f, 0.f};
+#pragma unroll
+    for (int q = 0; q < R; ++q) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) p[q][e] = z[q][e] == -INFINITY ? 0.f : exp2f(z[q][e] - m_run[e & 1]);
+        ps[0] += p[q][0] + p[q][2];
+        ps[1] += p[q][1] + p[q][3];
+    }
+#pragma unroll
+    for (int o2 = 4; o2 < 32; o2 <<= 1) {
+        ps[0] += __shfl_xor_sync(0xffffffffu, ps[0], o2);
+        ps[1] += __shfl_xor_sync(0xffffffffu, ps[1], o2);
+    }
+    l_run[0] = l_run[0] * alpha[0] + ps[0];
+    l_run[1] = l_run[1] * alpha[1] + ps[1];
+#pragma unroll
+    for (int n = 0; n < 8; ++n) {
+        o[n][0] *= alpha[0];
+        o[n][1] *= alpha[1];
+        o[n][2] *= alpha[0];
+        o[n][3] *= alpha[1];
+    }
+    // P^T as the B operand (k = group rows, n = heads), split hi + lo: the
+    // accumulator holds row g / heads 2t4.. of each 8x8 block, the operand
+    // rows 2t4.. / head g, so each block is transposed in registers
+    const int m = lane >> 3, i = lane & 7;  // ldmatrix.trans: matrix m, row i
+    const int row = r0 + (m >> 1) * 8 + i;   // rows +8 (m>>1), dims +8 (m&1)
+    if constexpr (G <= 4) {
+        // column c of this lane (2t4 + j) carries part c / G of its head's
+        // weight: 0 the bf16 value, 1 the bf16 remainder, 2+ nothing
+        auto piece = [&](float v, int part) -> float {
+            const float hi = __bfloat162float(__float2bfloat16_rn(v));
+            return part == 0 ? hi : (part == 1 ? v - hi : 0.f);
+        };
+        const int part0 = h0 / G, part1 = h1 / G;
+        uint32_t b0[R], b1[R];
+#pragma unroll
+        for (int q = 0; q < R; ++q) {
+            b0[q] = movmatrix_t(pack_bf16(piece(p[q][0], part0), piece(p[q][1], part1)));
+            b1[q] = movmatrix_t(pack_bf16(piece(p[q][2], part0), piece(p[q][3], part1)));
+        }
+        // ---- O^T += V^T P^T over 8 m-tiles of 16 dims, one MMA a group
+#pragma unroll
+        for (int mt2 = 0; mt2 < 8; ++mt2)
+#pragma unroll
+            for (int q = 0; q < R; ++q) {
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4_t(vt[q] + off(row, 2 * mt2 + (m & 1)), a0, a1, a2, a3);
+                mma_bf16(o[mt2], a0, a1, a2, a3, b0[q], b1[q]);
+            }
+    } else {
+        uint32_t bh0[R], bh1[R], bl0[R], bl1[R];
+#pragma unroll
+        for (int q = 0; q < R; ++q) {
+            const uint32_t pa = pack_bf16(p[q][0], p[q][1]), pb = pack_bf16(p[q][2], p[q][3]);
+            const __nv_bfloat162 ha = *reinterpret_cast<const __nv_bfloat162*>(&pa);
+            const __nv_bfloat162 hb = *reinterpret_cast<const __nv_bfloat162*>(&pb);
+            const uint32_t la = pack_bf16(p[q][0] - __low2float(ha), p[q][1] - __high2float(ha));
+            const uint32_t lb = pack_bf16(p[q][2] - __low2float(hb), p[q][3] - __high2float(hb));
+            bh0[q] = movmatrix_t(pa);
+            bh1[q] = movmatrix_t(pb);
+            bl0[q] = movmatrix_t(la);
+            bl1[q] = movmatrix_t(lb);
+        }
+        // ---- O^T += V^T P^T over 8 m-tiles of 16 dims, hi then lo a group
+#pragma unroll
+        for (int mt2 = 0; mt2 < 8; ++mt2)
+#pragma unroll
+            for (int q = 0; q < R; ++q) {
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4_t(vt[q] + off(row, 2 * mt2 + (m & 1)), a0, a1, a2, a3);
+                mma_bf16(o[mt2], a0, a1, a2, a3, bh0[q], bh1[q]);
+                mma_bf16(o[mt2], a0, a1, a2, a3, bl0[q], bl1[q]);
+            }
+    }
+}
+
 // CONTIG: every tile is 128 consecutive cache rows (a full-attention range, or
 // one 128-token block in block mode) and arrives by 2-D TMA tensor loads in the
 // 128-byte-swizzled layout (4 loads per tile) into a ring of STAGES tiles;
@@ -191,16 +404,17 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
             unsigned* __restrict__ counters, float* __restrict__ O, unsigned* __restrict__ flag, int early,
             float* __restrict__ sout, float scale, float* __restrict__ lse, int work,
             uint32_t* __restrict__ hout) {
+    static_assert(G == 1 || G == 2 || G == 4 || G == 8, "the group's heads fill a power-of-two part of one n-tile");
     using Cfg = AttnCfg<G>;
     extern __shared__ __align__(128) unsigned char smem_raw[];
     // 1024-byte aligned work area (the swizzled layout needs it)
     unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     __shared__ float s_wm[kAttnWarps][G], s_wl[kAttnWarps][G];
-    __shared__ float s_Mr[kClusterMax][G], s_Lr[kClusterMax][G];  // cluster path: received (M, L)
     __shared__ int s_last;
     __shared__ int s_fail;  // CONTIG: a bounded wait gave up; the CTA stops its tile loop
     __shared__ __align__(8) uint64_t s_bar[STAGES];
     __shared__ int s_first[STAGES];  // CONTIG: first cache row of the tile in each stage, or -1
+    __shared__ __align__(8) uint64_t s_rbar;  // cluster combine: the peers' slices have landed
 
     const int s = blockIdx.x, unit = blockIdx.y;
     const int b = unit / Hkv;
@@ -341,16 +555,28 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
     // full attention handing on its top-k: a histogram of the emitted scores'
     // top 11 key bits (the top-k's first radix digit), past the work area
     uint32_t* const s_hist = (CONTIG && sout && hout)
-        ? reinterpret_cast<uint32_t*>(smem + work + (CLUSTER ? Cfg::kRecvBytes : 0)) : nullptr;
+        ? reinterpret_cast<uint32_t*>(smem + work + (CLUSTER ? Cfg::recv_bytes(S) : 0)) : nullptr;
+    const bool ccomb = CLUSTER && S > 1;  // the splits combine in this cluster (uniform)
     if (s_hist)
         for (int i = tid; i < kHistBins; i += kAttnThreads) s_hist[i] = 0u;
     if (tid == 0) {
         s_fail = 0;
 #pragma unroll
         for (int i = 0; i < STAGES; ++i) mbar_init(&s_bar[i], CONTIG ? 1 : kTileRows);
+        if (ccomb) {
+            // every CTA of the cluster sends this CTA the slots of its partial
+            // that this CTA owns, and its (M, L) per head
+            const int per = ceil_div(G * 32, S);
+            const int own = max(0, min(per, G * 32 - s * per));
+            mbar_init(&s_rbar, 1);
+            mbar_arrive_expect_tx(&s_rbar, (unsigned)(S * (own * 16 + G * 8)));
+        }
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
     __syncthreads();
+    // every CTA of the cluster has started and armed its receive barrier once
+    // this phase completes (waited for just before the first remote store)
+    if (ccomb) asm volatile("barrier.cluster.arrive.relaxed;\n" ::: "memory");
     // CONTIG: the first STAGES tiles' block indices in one round, then their loads
     int next_first = -1;  // CONTIG, thread 0: first row of the tile that refills the stage next
     int issued = 0;       // CONTIG, thread 0: tiles whose loads have been issued
@@ -462,14 +688,16 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
     }
 
     // B fragments of Q^T (bf16, unscaled: the scale is applied to S in fp32):
-    // column g = query head g of the group (zero for g >= G), rows = dims.
+    // column g = query head g mod G of the group, rows = dims.  (G <= 4: the
+    // columns past G repeat the heads, so every lane's softmax state is that
+    // of real heads and the P^T columns past G can carry P's low parts.)
     uint32_t qa[8][2];
     {
-        const uint32_t* qrow = reinterpret_cast<const uint32_t*>(Q + ((size_t)unit * G + (g < G ? g : 0)) * kD);
+        const uint32_t* qrow = reinterpret_cast<const uint32_t*>(Q + ((size_t)unit * G + (g & (G - 1))) * kD);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-            qa[ks][0] = g < G ? qrow[ks * 8 + t4] : 0u;       // dims 16ks + 2t4, +1
-            qa[ks][1] = g < G ? qrow[ks * 8 + 4 + t4] : 0u;   // dims 16ks + 8 + 2t4, +1
+            qa[ks][0] = qrow[ks * 8 + t4];       // dims 16ks + 2t4, +1
+            qa[ks][1] = qrow[ks * 8 + 4 + t4];   // dims 16ks + 8 + 2t4, +1
         }
     }
     // O^T fragments: o[mt][0], [1] = dim 16mt + g, heads 2t4, 2t4 + 1; [2], [3] = dim 16mt + g + 8
@@ -482,119 +710,13 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
     float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
 
     const unsigned sbase = smem_u32(smem);
-    // The two contractions of flash decoding on this warp's 16 rows of a tile
-    // (K at kt, V at vt); bit i of vm: row r0 + i is in the set.
-    // sout (full attention that also emits its top-k, contiguous tiles only): the
-    // scores of the tile's rows -- scale x the max over the group's heads of q.k,
-    // the criterion a SELECT layer scores by -- written as S is formed
+    // this warp's 16 rows of one tile (K at kt, V at vt; bit i of vm: row r0 + i
+    // is in the set); sout: the emitted scores (full attention handing on its top-k)
     float* const su_out = (CONTIG && sout) ? sout + (size_t)unit * Ncap : nullptr;
     auto warp_tile = [&](unsigned kt, unsigned vt, uint32_t vm, int first) {
-        // byte offset of 16-byte chunk c of tile row r (padded rows, or the
-        // 128-byte swizzle of the TMA tensor loads: two 64-dim halves)
-        auto off = [&](int r, int c) -> unsigned {
-            if constexpr (CONTIG)
-                return (unsigned)((c >> 3) * 64 * kTileRows * 2 + r * 128 + (((c & 7) ^ (r & 7)) << 4));
-            else
-                return (unsigned)roff(r, c);
-        };
-        // ---- S^T = K Q^T over this warp's 16 rows (M = rows, N = heads)
-        float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};  // even / odd k-steps: two chains
-        {
-            const int m = lane >> 3, i = lane & 7;  // ldmatrix: matrix m, row i
-            const int row = r0 + (m & 1) * 8 + i;    // rows +8 (m&1), dims +8 (m>>1)
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                uint32_t a0, a1, a2, a3;
-                ldsm_x4(kt + off(row, 2 * ks + (m >> 1)), a0, a1, a2, a3);
-                mma_bf16(sc[ks & 1], a0, a1, a2, a3, qa[ks][0], qa[ks][1]);
-            }
-        }
-        // c[0], c[1]: row g, heads 2t4, 2t4 + 1; c[2], c[3]: row g + 8
-        float c[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) c[e] = sc[0][e] + sc[1][e];
-        const int h0 = 2 * t4, h1 = 2 * t4 + 1;  // this lane's two heads
-        const bool va = (vm >> g) & 1u, vb = (vm >> (g + 8)) & 1u;  // rows g, g + 8 in the set
-        if constexpr (CONTIG) {
-            if (su_out) {  // uniform: each row's max over the heads < G, across the 4 lanes of the row
-                float ea = fmaxf(h0 < G ? c[0] : -INFINITY, h1 < G ? c[1] : -INFINITY);
-                float eb = fmaxf(h0 < G ? c[2] : -INFINITY, h1 < G ? c[3] : -INFINITY);
-#pragma unroll
-                for (int o2 = 1; o2 < 4; o2 <<= 1) {
-                    ea = fmaxf(ea, __shfl_xor_sync(0xffffffffu, ea, o2));
-                    eb = fmaxf(eb, __shfl_xor_sync(0xffffffffu, eb, o2));
-                }
-                if (t4 == 0) {  // scale > 0: scale x max = max of the scaled logits
-                    if (va) {
-                        const float v = ea * scale;
-                        su_out[first + r0 + g] = v;
-                        if (s_hist) atomicAdd(&s_hist[order_key(v) >> 21], 1u);
-                    }
-                    if (vb) {
-                        const float v = eb * scale;
-                        su_out[first + r0 + g + 8] = v;
-                        if (s_hist) atomicAdd(&s_hist[order_key(v) >> 21], 1u);
-                    }
-                }
-            }
-        }
-        // ---- online softmax per head (columns of S^T): rows not in the set are -inf
-        float z[4];
-        z[0] = va ? c[0] * scale_log2 : -INFINITY;
-        z[1] = va ? c[1] * scale_log2 : -INFINITY;
-        z[2] = vb ? c[2] * scale_log2 : -INFINITY;
-        z[3] = vb ? c[3] * scale_log2 : -INFINITY;
-        float mt[2] = {fmaxf(z[0], z[2]), fmaxf(z[1], z[3])};
-#pragma unroll
-        for (int o2 = 4; o2 < 32; o2 <<= 1) {  // over the 8 lanes of a t4 (the rows)
-            mt[0] = fmaxf(mt[0], __shfl_xor_sync(0xffffffffu, mt[0], o2));
-            mt[1] = fmaxf(mt[1], __shfl_xor_sync(0xffffffffu, mt[1], o2));
-        }
-        float alpha[2], p[4];
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            const float mnew = fmaxf(m_run[j], mt[j]);
-            // a head with no finite logit yet keeps m = -inf, alpha = 0 and p = 0
-            alpha[j] = m_run[j] == -INFINITY ? 0.f : exp2f(m_run[j] - mnew);
-            m_run[j] = mnew;
-        }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) p[e] = z[e] == -INFINITY ? 0.f : exp2f(z[e] - m_run[e & 1]);
-        float ps[2] = {p[0] + p[2], p[1] + p[3]};
-#pragma unroll
-        for (int o2 = 4; o2 < 32; o2 <<= 1) {
-            ps[0] += __shfl_xor_sync(0xffffffffu, ps[0], o2);
-            ps[1] += __shfl_xor_sync(0xffffffffu, ps[1], o2);
-        }
-        l_run[0] = l_run[0] * alpha[0] + ps[0];
-        l_run[1] = l_run[1] * alpha[1] + ps[1];
-#pragma unroll
-        for (int n = 0; n < 8; ++n) {
-            o[n][0] *= alpha[0];
-            o[n][1] *= alpha[1];
-            o[n][2] *= alpha[0];
-            o[n][3] *= alpha[1];
-        }
-        // P^T as the B operand (k = tile rows, n = heads), split hi + lo: the
-        // accumulator holds row g / heads 2t4.. of each 8x8 block, the operand
-        // rows 2t4.. / head g, so each block is transposed in registers
-        const uint32_t pa = pack_bf16(p[0], p[1]), pb = pack_bf16(p[2], p[3]);
-        const __nv_bfloat162 ha = *reinterpret_cast<const __nv_bfloat162*>(&pa);
-        const __nv_bfloat162 hb = *reinterpret_cast<const __nv_bfloat162*>(&pb);
-        const uint32_t la = pack_bf16(p[0] - __low2float(ha), p[1] - __high2float(ha));
-        const uint32_t lb = pack_bf16(p[2] - __low2float(hb), p[3] - __high2float(hb));
-        const uint32_t bh0 = movmatrix_t(pa), bh1 = movmatrix_t(pb);
-        const uint32_t bl0 = movmatrix_t(la), bl1 = movmatrix_t(lb);
-        // ---- O^T += V^T P^T over 8 m-tiles of 16 dims
-        const int m = lane >> 3, i = lane & 7;  // ldmatrix.trans: matrix m, row i
-        const int row = r0 + (m >> 1) * 8 + i;   // rows +8 (m>>1), dims +8 (m&1)
-#pragma unroll
-        for (int mt2 = 0; mt2 < 8; ++mt2) {
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4_t(vt + off(row, 2 * mt2 + (m & 1)), a0, a1, a2, a3);
-            mma_bf16(o[mt2], a0, a1, a2, a3, bh0, bh1);
-            mma_bf16(o[mt2], a0, a1, a2, a3, bl0, bl1);
-        }
+        const unsigned kk[1] = {kt}, vv[1] = {vt};
+        const uint32_t mm[1] = {vm};
+        warp_rows<G, 1, CONTIG>(kk, vv, mm, qa, o, m_run, l_run, scale_log2, lane, r0, su_out, first, scale, s_hist);
     };
 
     if constexpr (CONTIG) {
@@ -643,20 +765,53 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
         if (t < ntiles && tid == 0)
             for (int j = t; j < issued; ++j) mbar_wait(&s_bar[j % STAGES], (unsigned)(j / STAGES) & 1u, nullptr);
     } else if constexpr (ASYNC) {
-        for (int t = 0; t < ntiles; ++t) {
-            // this lane's copies of tile t have landed (at most STAGES - 1 newer
-            // groups still pending), then the warp's
-            asm volatile("cp.async.wait_group %0;\n" ::"n"(STAGES - 1) : "memory");
+        if (ntiles <= STAGES) {
+            // the whole range is in the ring: once it has landed, every row
+            // group of this warp in one pass (groups past the last non-empty
+            // one skipped; masks are warp-uniform)
+            asm volatile("cp.async.wait_all;\n" ::: "memory");
             __syncwarp();
-            const int st = t % STAGES;
-            // the slot's rows seen as rows r0 .. r0 + 15 of a tile (the math's row offsets)
-            const unsigned ks = sbase + (unsigned)((st * kAttnWarps + warp) * kSlotBytes) - (unsigned)(r0 * kRowStride);
-            if (vmr[0]) warp_tile(ks, ks + 16 * kRowStride, vmr[0], 0);
-            __syncwarp();  // the math has read these rows before the stage is refilled
+            int nw = 0;
 #pragma unroll
-            for (int i = 0; i + 1 < STAGES; ++i) vmr[i] = vmr[i + 1];
-            vmr[STAGES - 1] = t + STAGES < ntiles ? issue_async(t + STAGES, st, my_row(t + STAGES)) : 0u;
-            asm volatile("cp.async.commit_group;\n" ::: "memory");
+            for (int q = 0; q < STAGES; ++q)
+                if (vmr[q]) nw = q + 1;
+            auto groups = [&](auto rc) {
+                constexpr int R = decltype(rc)::value;
+                unsigned kk[R], vv[R];
+                uint32_t mm[R];
+#pragma unroll
+                for (int q = 0; q < R; ++q) {
+                    kk[q] = sbase + (unsigned)((q * kAttnWarps + warp) * kSlotBytes) - (unsigned)(r0 * kRowStride);
+                    vv[q] = kk[q] + 16 * kRowStride;
+                    mm[q] = vmr[q];
+                }
+                warp_rows<G, R, false>(kk, vv, mm, qa, o, m_run, l_run, scale_log2, lane, r0, nullptr, 0, scale,
+                                       nullptr);
+            };
+            if constexpr (STAGES >= 3) {
+                if (nw == 3) groups(std::integral_constant<int, 3>{});
+            }
+            if constexpr (STAGES >= 2) {
+                if (nw == 2) groups(std::integral_constant<int, 2>{});
+            }
+            if (nw == 1) groups(std::integral_constant<int, 1>{});
+            static_assert(STAGES <= 3, "the one-pass branch covers rings of up to 3 tiles");
+        } else {  // a longer range streams through the ring, a tile at a time
+            for (int t = 0; t < ntiles; ++t) {
+                // this lane's copies of tile t have landed (at most STAGES - 1 newer
+                // groups still pending), then the warp's
+                asm volatile("cp.async.wait_group %0;\n" ::"n"(STAGES - 1) : "memory");
+                __syncwarp();
+                const int st = t % STAGES;
+                // the slot's rows seen as rows r0 .. r0 + 15 of a tile (the math's row offsets)
+                const unsigned ks = sbase + (unsigned)((st * kAttnWarps + warp) * kSlotBytes) - (unsigned)(r0 * kRowStride);
+                if (vmr[0]) warp_tile(ks, ks + 16 * kRowStride, vmr[0], 0);
+                __syncwarp();  // the math has read these rows before the stage is refilled
+#pragma unroll
+                for (int i = 0; i + 1 < STAGES; ++i) vmr[i] = vmr[i + 1];
+                vmr[STAGES - 1] = t + STAGES < ntiles ? issue_async(t + STAGES, st, my_row(t + STAGES)) : 0u;
+                asm volatile("cp.async.commit_group;\n" ::: "memory");
+            }
         }
         asm volatile("cp.async.wait_all;\n" ::: "memory");  // nothing in flight over the merge below
     } else {
@@ -673,6 +828,19 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
             if (t + 1 < ntiles) fetch(t + 1, my_row(t + 1));  // the next tile's loads fly during this tile's math
             if (vm) warp_tile(sbase, sbase + kTileRows * kRowStride, vm, 0);
             __syncwarp();  // the math has read these rows before the next store
+        }
+    }
+    // G <= 4: head h's output is the sum of columns h (hi) and h + G (lo)
+    if constexpr (G == 4 || G == 2) {
+#pragma unroll
+        for (int n = 0; n < 8; ++n)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o[n][e] += __shfl_xor_sync(0xffffffffu, o[n][e], G / 2);
+    } else if constexpr (G == 1) {
+#pragma unroll
+        for (int n = 0; n < 8; ++n) {
+            o[n][0] += o[n][1];
+            o[n][2] += o[n][3];
         }
     }
     __syncthreads();
@@ -738,60 +906,64 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
             }
             return;
         }
-        // the S splits of this unit are the S CTAs of this cluster (rank = split)
-        cg::cluster_group cluster = cg::this_cluster();
-        const int per = ceil_div(nslots, S);  // output slots owned by each CTA
-        float4* recv = reinterpret_cast<float4*>(smem + work);  // [src][per], past the work area
+        // the S splits of this unit are the S CTAs of this cluster (rank =
+        // split).  Output slot q (4 dims of one head) is owned by CTA q / per;
+        // each CTA sends every owner its slots of its merged partial and its
+        // (M, L) per head with st.async, counted on the owner's barrier, so an
+        // owner waits only for the bytes it needs (no cluster-wide barrier).
+        const int per = ceil_div(nslots, S);
+        float4* recv = reinterpret_cast<float4*>(smem + work);      // [src][per]
+        float2* rml = reinterpret_cast<float2*>(recv + S * per);    // [src][G]: (M, L)
+        const unsigned rbar = smem_u32(&s_rbar);
+        asm volatile("barrier.cluster.wait;\n" ::: "memory");  // every peer has armed its barrier
         if (has_slot) {
             const int owner = tid / per, lslot = tid - owner * per;
-            *cluster.map_shared_rank(recv + s * per + lslot, owner) = A;
+            st_async_f4(cluster_addr(smem_u32(recv + s * per + lslot), owner), A.x, A.y, A.z, A.w,
+                        cluster_addr(rbar, owner));
+            if (qd_me < S)  // head h_me's (M, L) to CTA qd_me
+                st_async_f2(cluster_addr(smem_u32(rml + s * G + h_me), qd_me), M_me, L_me,
+                            cluster_addr(rbar, qd_me));
         }
-        if (has_slot && qd_me < S) {  // head h_me's (M, L) to rank qd_me
-            *cluster.map_shared_rank(&s_Mr[s][h_me], qd_me) = M_me;
-            *cluster.map_shared_rank(&s_Lr[s][h_me], qd_me) = L_me;
+        // this CTA's slices: one bounded wait, the same outcome for the whole CTA
+        const bool ok = mbar_wait(&s_rbar, 0u, nullptr, kRecvSpins);
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) atomicOr(flag, kFlagTimeout);
+            return;  // the output is unspecified, and the flag says so
         }
-        cluster.sync();  // every slice has arrived at its owner
-        // this CTA's `per` output slots, each from the S sources: one thread a
-        // (slot, source) pair, the S2 (S rounded up to a power of two) threads
-        // of a slot adjacent in a warp and reduced by shuffles
-        const int S2 = S <= 2 ? 2 : S <= 4 ? 4 : 8;
-        const int lg2 = S2 == 2 ? 1 : S2 == 4 ? 2 : 3;
-        const int total = (per * S2 + 31) & ~31;  // whole warps: every lane of a warp takes part
-        for (int q = tid; q < total; q += kAttnThreads) {
-            const int ls = q >> lg2, j = q & (S2 - 1);
-            const int slot = s * per + ls;
-            const bool live = ls < per && slot < nslots;
-            const bool src = live && j < S;
-            const int h = live ? slot >> 5 : 0, qd = slot & 31;
-            const float mj = src ? s_Mr[j][h] : -INFINITY;
-            float M = mj;
-            for (int o2 = 1; o2 < S2; o2 <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o2));
-            const float w = mj == -INFINITY ? 0.f : exp2f(mj - M);
+        // one thread an owned slot, over the S sources
+        const int own = min(per, nslots - s * per);
+        if (tid < own) {
+            const int slot = s * per + tid;
+            const int h = slot >> 5, qd = slot & 31;
+            float mj[kClusterMax], M = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < kClusterMax; ++j) {
+                mj[j] = j < S ? rml[j * G + h].x : -INFINITY;
+                M = fmaxf(M, mj[j]);
+            }
             float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
             float den = 0.f;
-            if (src) {
-                const float4 oj = recv[j * per + ls];
-                den = w * s_Lr[j][h];
-                num = make_float4(w * oj.x, w * oj.y, w * oj.z, w * oj.w);
-            }
-            for (int o2 = 1; o2 < S2; o2 <<= 1) {
-                den += __shfl_xor_sync(0xffffffffu, den, o2);
-                num.x += __shfl_xor_sync(0xffffffffu, num.x, o2);
-                num.y += __shfl_xor_sync(0xffffffffu, num.y, o2);
-                num.z += __shfl_xor_sync(0xffffffffu, num.z, o2);
-                num.w += __shfl_xor_sync(0xffffffffu, num.w, o2);
-            }
-            if (live && j == 0) {
-                float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (den > 0.f) {
-                    const float inv = __frcp_rn(den);  // one rounding more than a division: ~1e-7 relative
-                    r = make_float4(num.x * inv, num.y * inv, num.z * inv, num.w * inv);
+#pragma unroll
+            for (int j = 0; j < kClusterMax; ++j) {
+                if (j < S && mj[j] != -INFINITY) {
+                    const float w = exp2f(mj[j] - M);
+                    const float4 oj = recv[j * per + tid];
+                    den += w * rml[j * G + h].y;
+                    num.x += w * oj.x;
+                    num.y += w * oj.y;
+                    num.z += w * oj.z;
+                    num.w += w * oj.w;
                 }
-                *reinterpret_cast<float4*>(O + ((size_t)unit * G + h) * kD + 4 * qd) = r;
-                if (lse && qd == 0) lse[(size_t)unit * G + h] = den > 0.f ? M + log2f(den) : -INFINITY;
             }
+            float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (den > 0.f) {
+                const float inv = __frcp_rn(den);  // one rounding more than a division: ~1e-7 relative
+                r = make_float4(num.x * inv, num.y * inv, num.z * inv, num.w * inv);
+            }
+            *reinterpret_cast<float4*>(O + ((size_t)unit * G + h) * kD + 4 * qd) = r;
+            if (lse && qd == 0) lse[(size_t)unit * G + h] = den > 0.f ? M + log2f(den) : -INFINITY;
         }
-        return;  // no remote access after the barrier: CTAs may leave in any order
+        return;  // nothing of this CTA is read remotely: CTAs may leave in any order
     } else {
         if (has_slot) {
             float* pu = part + (((size_t)unit * S + s) * G + h_me) * kPartStride;
@@ -915,7 +1087,7 @@ enum AttnVariant { kContig1 = 0, kContigRing = 1, kGatherReg = 2, kGatherAsync1 
 // co-resident clusters by (device, log2 G, variant, S, warp-tile slots of the
 // cp.async gather or 0); 0 = not queried yet
 constexpr int kCacheDevs = 16;
-static int g_max_clusters[kCacheDevs][4][kVariants][kClusterMax + 1][3 * kAttnWarps + 1];
+static int g_max_clusters[kCacheDevs][4][kVariants][kClusterMax + 1][3 * kAttnWarps + 1][2];
 
 // the work area (staging, merge buffer) of an instance: the cp.async gather by
 // the slots its CTAs use, every other instance its whole ring
@@ -924,12 +1096,28 @@ static int work_bytes_of(int slots) {
     return (ASYNC && !CONTIG) ? AttnCfg<G>::slot_work_bytes(slots) : AttnCfg<G>::work_bytes(STAGES);
 }
 
+// dynamic shared memory of a launch: the work area, the cluster's receive
+// area, and the emitted scores' histogram
+template <int G, int STAGES, bool CLUSTER, bool CONTIG, bool ASYNC>
+static int smem_of(int S, int slots, bool hist) {
+    return 1024 + work_bytes_of<G, STAGES, CONTIG, ASYNC>(slots) + (CLUSTER ? AttnCfg<G>::recv_bytes(S) : 0) +
+           (hist ? kHistBins * 4 : 0);
+}
+
 template <int G, int STAGES, bool CONTIG, bool ASYNC>
-static int max_active_clusters(int S, int slots) {
+static int max_active_clusters(int S, int slots, bool hist) {
+    const void* f = (const void*)attn_kernel<G, STAGES, true, CONTIG, ASYNC>;
+    const int smem = smem_of<G, STAGES, true, CONTIG, ASYNC>(S, slots, hist);
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, f) != cudaSuccess) {
+        cudaGetLastError();
+        return -1;
+    }
+    if (smem > fa.maxDynamicSharedSizeBytes) return -1;  // past what the kernel was configured for: no cluster
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)S, 1);
     cfg.blockDim = dim3(kAttnThreads);
-    cfg.dynamicSmemBytes = 1024 + work_bytes_of<G, STAGES, CONTIG, ASYNC>(slots) + AttnCfg<G>::kRecvBytes;
+    cfg.dynamicSmemBytes = smem;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)S;
@@ -946,17 +1134,19 @@ static int max_active_clusters(int S, int slots) {
 }
 
 template <int G>
-static int max_clusters_g(int var, int S, int slots) {
+static int max_clusters_g(int var, int S, int slots, bool hist) {
     switch (var) {
-        case kContig1: return max_active_clusters<G, 1, true, false>(S, 0);
-        case kContigRing: return max_active_clusters<G, kRing, true, false>(S, 0);
-        case kGatherReg: return max_active_clusters<G, 1, false, false>(S, 0);
-        case kGatherAsync1: return max_active_clusters<G, 1, false, true>(S, slots);
-        default: return max_active_clusters<G, kRing, false, true>(S, slots);
+        case kContig1: return max_active_clusters<G, 1, true, false>(S, 0, hist);
+        case kContigRing: return max_active_clusters<G, kRing, true, false>(S, 0, hist);
+        case kGatherReg: return max_active_clusters<G, 1, false, false>(S, 0, hist);
+        case kGatherAsync1: return max_active_clusters<G, 1, false, true>(S, slots, hist);
+        default: return max_active_clusters<G, kRing, false, true>(S, slots, hist);
     }
 }
 
-static bool attn_cluster_fits(int G, int var, int S, int units, int slots) {
+// whether the S splits of every unit can combine in a cluster: every cluster
+// resident at once, with the shared memory the launch needs
+static bool attn_cluster_fits(int G, int var, int S, int units, int slots, bool hist) {
     if (S > kClusterMax) return false;
     if (S == 1) return true;  // a cluster of one: no co-scheduling constraint
     int dev = 0;
@@ -964,17 +1154,17 @@ static bool attn_cluster_fits(int G, int var, int S, int units, int slots) {
     if (var != kGatherAsync1 && var != kGatherAsyncRing) slots = 0;
     auto query = [&]() {
         switch (G) {
-            case 1: return max_clusters_g<1>(var, S, slots);
-            case 2: return max_clusters_g<2>(var, S, slots);
-            case 4: return max_clusters_g<4>(var, S, slots);
-            case 8: return max_clusters_g<8>(var, S, slots);
+            case 1: return max_clusters_g<1>(var, S, slots, hist);
+            case 2: return max_clusters_g<2>(var, S, slots, hist);
+            case 4: return max_clusters_g<4>(var, S, slots, hist);
+            case 8: return max_clusters_g<8>(var, S, slots, hist);
             default: return -1;
         }
     };
     int n;
     if (dev < kCacheDevs) {
         const int lg = G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : 3;
-        int& c = g_max_clusters[dev][lg][var][S][slots];
+        int& c = g_max_clusters[dev][lg][var][S][slots][hist ? 1 : 0];
         if (c == 0) c = query();
         n = c;
     } else {
@@ -1008,8 +1198,7 @@ static cudaError_t attn_launch_g(dim3 grid, cudaStream_t st, const AttnArgs& a) 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = dim3(kAttnThreads);
-    cfg.dynamicSmemBytes = 1024 + work + (CLUSTER ? AttnCfg<G>::kRecvBytes : 0) +
-                           (a.sout && a.hout ? kHistBins * 4 : 0);
+    cfg.dynamicSmemBytes = smem_of<G, STAGES, CLUSTER, CONTIG, ASYNC>(a.splits, a.slots, a.sout && a.hout);
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1027,9 +1216,18 @@ static cudaError_t attn_launch_g(dim3 grid, cudaStream_t st, const AttnArgs& a) 
 template <int G, int STAGES, bool CLUSTER, bool CONTIG, bool ASYNC = false>
 static cudaError_t attn_configure_one() {
     const void* f = (const void*)attn_kernel<G, STAGES, CLUSTER, CONTIG, ASYNC>;
-    // contiguous tiles may carry the emitted scores' histogram (8 KB more)
-    cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         AttnCfg<G>::smem_bytes(STAGES, CLUSTER) + (CONTIG ? kHistBins * 4 : 0));
+    // contiguous tiles may carry the emitted scores' histogram (8 KB more);
+    // at most what the device allows next to the kernel's static shared
+    // memory (a cluster launch that would need more combines in the workspace)
+    int dev = 0, optin = 0;
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, f);
+    if (e != cudaSuccess) return e;
+    const int want = AttnCfg<G>::smem_bytes(STAGES, CLUSTER) + (CONTIG ? kHistBins * 4 : 0);
+    const int cap = optin - (int)fa.sharedSizeBytes;
+    e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, want < cap ? want : cap);
     if (e == cudaSuccess && CLUSTER) e = cudaFuncSetAttribute(f, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     return e;
 }
@@ -1138,9 +1336,29 @@ cudaError_t launch_attn(const void* Q, const void* K, const void* V, const int32
         const int cap = var == kGatherAsync1 ? kAttnWarps : kRing * kAttnWarps;
         return (int)(wt < cap ? (wt < 1 ? 1 : wt) : cap);
     };
+    // Early inputs (the caller's promise): this launch's gathers are meant to
+    // run while the launch before it on the stream finishes, so its clusters
+    // must find room beside that launch's.  When 2 x units clusters of
+    // `splits` CTAs cannot be resident at once (a B200 holds 15 clusters of 8
+    // one-CTA-an-SM gathers, 22 of 6), the largest split count down to 3/4 of
+    // it whose clusters can: fewer, longer splits that all start early beat
+    // more splits of which one cluster waits for the previous launch to leave.
+    // (The workspace is sized for `splits`, an upper bound.)
+    if (early >= 2 && !contig && !host_kv && splits > 2 && splits <= kClusterMax) {
+        auto fits_twice = [&](int S) {
+            const int v = variant_of(S);
+            return attn_cluster_fits(d.G, v, S, 2 * d.units(), slots_of(S, v), false);
+        };
+        if (!fits_twice(splits))
+            for (int S = splits - 1; 4 * S >= 3 * splits; --S)
+                if (fits_twice(S)) {
+                    splits = S;
+                    break;
+                }
+    }
     const int var = variant_of(splits);
     const int slots = slots_of(splits, var);
-    const bool cluster = attn_cluster_fits(d.G, var, splits, d.units(), slots);
+    const bool cluster = attn_cluster_fits(d.G, var, splits, d.units(), slots, scores_out && hist_out);
     AttnArgs a;
     memset(&a.kmap, 0, sizeof a.kmap);
     memset(&a.vmap, 0, sizeof a.vmap);
