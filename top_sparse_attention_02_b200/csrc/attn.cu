@@ -36,11 +36,14 @@
 //   O^T += V^T P^T (8 m-tiles of 16 dims, P split as bf16 hi + bf16 lo so
 //                  that the weights keep ~16 bits; V^T fragments by
 //                  ldmatrix.trans, P^T fragments from the S^T accumulator by
-//                  movmatrix.trans).  With g <= 4 the n-tile's columns
-//                  G .. 2G-1 repeat the heads (Q^T column c is head c mod G),
-//                  and carry lo while columns 0 .. G-1 carry hi: one MMA an
-//                  m-tile (8), the two column sets summed once at the end.
-//                  With g = 8 there is no spare column: two MMAs an m-tile.
+//                  movmatrix.trans).  In the gather with g <= 4 the n-tile's
+//                  columns G .. 2G-1 repeat the heads (Q^T column c is head
+//                  c mod G) and carry lo while columns 0 .. G-1 carry hi: one
+//                  MMA an m-tile (8), the two column sets summed once at the
+//                  end.  With g = 8 there is no spare column, and contiguous
+//                  tiles (HBM-bound) keep zero columns: two MMAs an m-tile
+//                  (the spare-column form made the 128K full layer 1.5 us
+//                  slower).
 // A warp-tile is a chain of dependent steps (on sm_100a: ~20 cycles an
 // mma.sync, ~30 a shuffle, an exp2 or a shared load), so when a CTA's whole
 // range is in its cp.async ring, each warp takes all its 16-row groups in one
@@ -220,7 +223,7 @@ __device__ __forceinline__ int roff(int row, int chunk) { return row * kRowStrid
 // of the group's rows -- scale x the max over the group's heads of q.k, the
 // criterion a SELECT layer scores by -- written as S is formed (row first +
 // r0 + x), with their top-digit histogram in s_hist.
-template <int G, int R, bool CONTIG>
+template <int G, int R, bool CONTIG, bool SPARE>
 __device__ __forceinline__ void warp_rows(const unsigned (&kt)[R], const unsigned (&vt)[R], const uint32_t (&vm)[R],
                                           const uint32_t (&qa)[8][2], float (&o)[8][4], float (&m_run)[2],
                                           float (&l_run)[2], float scale_log2, int lane, int r0, float* su_out,
@@ -336,7 +339,7 @@ __device__ __forceinline__ void warp_rows(const unsigned (&kt)[R], const unsigne
     // rows 2t4.. / head g, so each block is transposed in registers
     const int m = lane >> 3, i = lane & 7;  // ldmatrix.trans: matrix m, row i
     const int row = r0 + (m >> 1) * 8 + i;   // rows +8 (m>>1), dims +8 (m&1)
-    if constexpr (G <= 4) {
+    if constexpr (SPARE) {
         // column c of this lane (2t4 + j) carries part c / G of its head's
         // weight: 0 the bf16 value, 1 the bf16 remainder, 2+ nothing
         auto piece = [&](float v, int part) -> float {
@@ -406,6 +409,11 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
             uint32_t* __restrict__ hout) {
     static_assert(G == 1 || G == 2 || G == 4 || G == 8, "the group's heads fill a power-of-two part of one n-tile");
     using Cfg = AttnCfg<G>;
+    // the gather (latency-bound: its MMAs are on the chain) puts P's low part
+    // in the n-tile's spare columns; contiguous tiles (HBM-bound, the math
+    // hidden under the stream) keep zero columns and a second MMA, which
+    // measured faster there (128K full layer 86.1 against 88.0 us cold)
+    constexpr bool SPARE = G <= 4 && !CONTIG;
     extern __shared__ __align__(128) unsigned char smem_raw[];
     // 1024-byte aligned work area (the swizzled layout needs it)
     unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -693,11 +701,12 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
     // of real heads and the P^T columns past G can carry P's low parts.)
     uint32_t qa[8][2];
     {
+        const bool live = SPARE || g < G;  // without spare columns, columns past G are zero
         const uint32_t* qrow = reinterpret_cast<const uint32_t*>(Q + ((size_t)unit * G + (g & (G - 1))) * kD);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-            qa[ks][0] = qrow[ks * 8 + t4];       // dims 16ks + 2t4, +1
-            qa[ks][1] = qrow[ks * 8 + 4 + t4];   // dims 16ks + 8 + 2t4, +1
+            qa[ks][0] = live ? qrow[ks * 8 + t4] : 0u;       // dims 16ks + 2t4, +1
+            qa[ks][1] = live ? qrow[ks * 8 + 4 + t4] : 0u;   // dims 16ks + 8 + 2t4, +1
         }
     }
     // O^T fragments: o[mt][0], [1] = dim 16mt + g, heads 2t4, 2t4 + 1; [2], [3] = dim 16mt + g + 8
@@ -716,7 +725,8 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
     auto warp_tile = [&](unsigned kt, unsigned vt, uint32_t vm, int first) {
         const unsigned kk[1] = {kt}, vv[1] = {vt};
         const uint32_t mm[1] = {vm};
-        warp_rows<G, 1, CONTIG>(kk, vv, mm, qa, o, m_run, l_run, scale_log2, lane, r0, su_out, first, scale, s_hist);
+        warp_rows<G, 1, CONTIG, SPARE>(kk, vv, mm, qa, o, m_run, l_run, scale_log2, lane, r0, su_out, first, scale,
+                                       s_hist);
     };
 
     if constexpr (CONTIG) {
@@ -785,8 +795,8 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
                     vv[q] = kk[q] + 16 * kRowStride;
                     mm[q] = vmr[q];
                 }
-                warp_rows<G, R, false>(kk, vv, mm, qa, o, m_run, l_run, scale_log2, lane, r0, nullptr, 0, scale,
-                                       nullptr);
+                warp_rows<G, R, false, SPARE>(kk, vv, mm, qa, o, m_run, l_run, scale_log2, lane, r0, nullptr, 0,
+                                              scale, nullptr);
             };
             if constexpr (STAGES >= 3) {
                 if (nw == 3) groups(std::integral_constant<int, 3>{});
@@ -830,13 +840,13 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
             __syncwarp();  // the math has read these rows before the next store
         }
     }
-    // G <= 4: head h's output is the sum of columns h (hi) and h + G (lo)
-    if constexpr (G == 4 || G == 2) {
+    // spare columns: head h's output is the sum of columns h (hi) and h + G (lo)
+    if constexpr (SPARE && (G == 4 || G == 2)) {
 #pragma unroll
         for (int n = 0; n < 8; ++n)
 #pragma unroll
             for (int e = 0; e < 4; ++e) o[n][e] += __shfl_xor_sync(0xffffffffu, o[n][e], G / 2);
-    } else if constexpr (G == 1) {
+    } else if constexpr (SPARE && G == 1) {
 #pragma unroll
         for (int n = 0; n < 8; ++n) {
             o[n][0] += o[n][1];
