@@ -143,6 +143,25 @@ def test_attn_stage_random_sets(cuda_dev, Hq, Hkv):
     check_output(O.cpu().numpy(), ref, "random sets")
 
 
+@pytest.mark.parametrize("g", [1, 2, 4, 8])
+@pytest.mark.parametrize("k", [300, 600, 850])
+def test_attn_cluster_combine_uneven_owners(cuda_dev, g, k):
+    """4 units (2 sequences x 2 kv-heads) with k = 300, 600, 850 take ceil(k / 128)
+    = 3, 5, 7 splits, one cluster a unit: the 32g output slots split unevenly
+    among the owner CTAs (the last owns fewer).  The second sequence's 3 rows
+    leave most of its CTAs without rows (they still send their empty partials)."""
+    rng = np.random.default_rng(k * 10 + g)
+    Hkv = 2
+    lens = [2000, 5]
+    L = layer(2, g * Hkv, Hkv, 2000, lens, seed=k + g, tail_fill=float("nan"))
+    Q, K, V, ln = G.to_dev(L, cuda_dev)
+    kb = [k, 3]
+    idx = _rand_idx(rng, 2, Hkv, lens, k, kb)
+    O, _ = G.run_attn(Q, K, V, ln, torch.from_numpy(idx).to(cuda_dev), kb, k, 1, SCALE)
+    ref = oracle.attn(L.Q, L.K, L.V, L.seq_lens, idx, kb, k, 1, SCALE)
+    check_output(O.cpu().numpy(), ref, f"g={g}, k={k}")
+
+
 def test_attn_stage_sliding_window_and_padding(cuda_dev):
     lens = [500, 64]
     L = layer(2, 8, 2, 512, lens, seed=9, tail_fill=float("nan"))
@@ -717,19 +736,33 @@ def test_hylra_calibrate_then_run_the_policy(cuda_dev):
 
 # ------------------------------------------------------------------ sequence sharding (one GPU, shards in turn)
 
-@pytest.mark.parametrize("case", ["two_uneven", "three_with_an_empty_shard", "four_k_eq_len"])
+@pytest.mark.parametrize("case", ["two_uneven", "three_with_an_empty_shard", "four_k_eq_len", "ties_across_shards",
+                                  "wide_fallback"])
 def test_sequence_sharded_select_on_one_gpu(cuda_dev, case):
     """The sharded SELECT step with its R shards run one after another on one
     GPU and the all-gathers replaced by stacking: the same indices as the one-GPU
-    SELECT step (exact top-k of the whole cache) and the same attention."""
+    SELECT step (exact top-k of the whole cache) and the same attention.  Up to
+    24576 candidates a unit the merge is one kernel; "wide_fallback" (4 x 7000)
+    takes the pack / top-k / map path."""
     if case == "two_uneven":
         B, Hq, Hkv, N, lens, kreq, bounds = 2, 32, 8, 7000, [7000, 3500], [200, 120], [0, 2900, 7000]
     elif case == "three_with_an_empty_shard":  # sequence 1 ends inside shard 0
         B, Hq, Hkv, N, lens, kreq, bounds = 2, 16, 4, 9000, [9000, 100], [300, 300], [0, 4000, 4100, 9000]
+    elif case == "ties_across_shards":  # 21 equal scores around the k-th, either side of the shard boundary
+        B, Hq, Hkv, N, lens, kreq, bounds = 1, 8, 2, 6000, [6000], [150], [0, 3000, 6000]
+    elif case == "wide_fallback":
+        B, Hq, Hkv, N, lens, kreq, bounds = 1, 8, 2, 28672, [28000], [7000], [0, 7168, 14336, 21504, 28672]
     else:  # k = len: every row, spread over four shards
         B, Hq, Hkv, N, lens, kreq, bounds = 1, 8, 2, 4096, [4000], [4000], [0, 1024, 2048, 3072, 4096]
     R, k_max = len(bounds) - 1, max(kreq)
     L = layer(B, Hq, Hkv, N, lens, seed=131, tail_fill=float("nan"))
+    if case == "ties_across_shards":
+        S0 = oracle.scores(L.Q, L.K, L.seq_lens, SCALE)
+        for h in range(Hkv):
+            src = int(np.argsort(-S0[0, h, :lens[0]], kind="stable")[kreq[0] - 6])  # rank k - 5
+            for dst in list(range(2990, 3000)) + list(range(3000, 3010)):
+                if dst != src:
+                    L.K[0, h, dst] = L.K[0, h, src].clone()
     Q, K, V, ln = G.to_dev(L, cuda_dev)
     kr = torch.tensor(kreq, dtype=torch.int32, device=cuda_dev)
     _, idx_one = G.step(Q, K, V, ln, mode=tsa.SELECT, scale=SCALE, k_max=k_max, kreq=kreq)

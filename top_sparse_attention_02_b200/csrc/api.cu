@@ -283,6 +283,13 @@ tsa_status tsa_shard_merge(const float* cand_scores, const int32_t* cand_rows, i
         return fail(TSA_ERR_UNSUPPORTED, "tsa_shard_merge: %lld candidates per unit exceed the top-k capacity", width);
     const ShardLayout S = shard_layout(d, k_max, n_shards);  // merge offsets do not depend on Ncap
     TSA_TRY(check_ws(ws, ws_bytes, S.merge_total));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (tsa::merge_topk_fits(n_shards, k_max)) {  // one kernel: the lists in one CTA's shared memory a unit
+        const cudaError_t e = tsa::launch_merge_topk(cand_scores, cand_rows, n_shards, d.units(), d.Hkv, k_max,
+                                                     k_per_seq, idx, flag_of(ws), st);
+        if (e != cudaSuccess) return cuda_fail(e, "tsa_shard_merge");
+        return TSA_OK;
+    }
     char* w = static_cast<char*>(ws);
     float* pk_scores = reinterpret_cast<float*>(w + S.pk_scores);
     int32_t* pk_rows = reinterpret_cast<int32_t*>(w + S.pk_rows);
@@ -292,7 +299,6 @@ tsa_status tsa_shard_merge(const float* cand_scores, const int32_t* cand_rows, i
     // histograms (zero here: every call that used them zeroed them), and the
     // top-k over the candidates starts from it
     uint32_t* hist = reinterpret_cast<uint32_t*>(w + S.front.hist);
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e = tsa::launch_merge_pack(cand_scores, cand_rows, n_shards, d.units(), d.Hkv, k_max, pk_scores,
                                            pk_rows, n_cand, hist, flag_of(ws), st);
     if (e != cudaSuccess) return cuda_fail(e, "tsa_shard_merge (pack)");

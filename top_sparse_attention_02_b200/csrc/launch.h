@@ -44,6 +44,13 @@ cudaError_t launch_shard_pack(const float* scores, int rows_cap, int units, int 
                               float* cand_scores, unsigned* flag, cudaStream_t st);
 // also adds the packed scores' first radix digit into hist [units][kHistBins]
 // (zero on entry; the top-k over the packed candidates reads and zeroes it)
+// the exact top-k of each unit's candidates from R shards in one kernel, rows
+// straight into idx (ascending, then -1); only when R * k_max <= kMergeCap
+// (they fit one CTA's shared memory as (key, row))
+constexpr int kMergeCap = 24576;
+bool merge_topk_fits(int R, int k_max);
+cudaError_t launch_merge_topk(const float* cand_scores, const int32_t* cand_rows, int R, int units, int Hkv,
+                              int k_max, const int32_t* kreq, int32_t* idx, unsigned* flag, cudaStream_t st);
 cudaError_t launch_merge_pack(const float* cand_scores, const int32_t* cand_rows, int R, int units, int Hkv,
                               int k_max, float* pk_scores, int32_t* pk_rows, int32_t* n_cand, uint32_t* hist,
                               unsigned* flag, cudaStream_t st);
