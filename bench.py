@@ -308,6 +308,17 @@ def run_ours(args, rank, world, dev):
 
     # per-stage device times: each stage alone, repeated in its own graph
     stages = stage_times(tsa, w, plan, layers, Kmean, ws, kreq_t, idx, O, stream)
+    # each layer's share of the step as captured: the step cut after layer i,
+    # timed the same way (a graph of back-to-back copies), minus the step cut
+    # after layer i - 1 (with early inputs a layer's launch overlaps the end of
+    # the one before, which the stages timed alone do not show)
+    prefix = [graph_us(lambda n=n: [tsa.decode_step(a, stream) for a in step_args[:n]], stream, 10)
+              for n in range(1, w.layers + 1)]
+    kinds = {tsa.SELECT: "select_step", tsa.REUSE: "attn", tsa.FULL: "full"}
+    stages["in_step"] = {f"L{li}_{kinds[w.route[li]]}": prefix[li] - (prefix[li - 1] if li else 0.0)
+                         for li in range(w.layers)}
+    stages["in_step_note"] = ("us a layer adds to the captured step (TSA_EARLY_INPUTS): the step cut after the "
+                              "layer minus the step cut before it, each timed as 10 back-to-back copies in a graph")
     copy_gbs = copy_probe(tsa, dev, stream)
     gather = gather_probe(tsa, w, plan, layers, idx, ws, stream)
 
