@@ -320,6 +320,7 @@ def run_ours(args, rank, world, dev):
     stages["in_step_note"] = ("us a layer adds to the captured step (TSA_EARLY_INPUTS): the step cut after the "
                               "layer minus the step cut before it, each timed as 10 back-to-back copies in a graph")
     copy_gbs = copy_probe(tsa, dev, stream)
+    read_gbs = read_probe(tsa, dev, ws, stream)
     gather = gather_probe(tsa, w, plan, layers, idx, ws, stream)
 
     peak, peak_kind = measured_peaks()
@@ -341,6 +342,8 @@ def run_ours(args, rank, world, dev):
                      "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, torch copy)",
                      "copy_probe_gbs_this_run": copy_gbs,
+                     "read_probe_gbs_this_run": read_gbs,
+                     "frac_of_read_probe": achieved / read_gbs,
                      "traffic": recorded_traffic("score_tc_kernel") if w is workloads.REUSE128K else None,
                      "algorithmic_bytes_per_launch": score_bytes},
         "attn_roofline": attn_roofline(w, plan, stages, gather),
@@ -673,6 +676,24 @@ def copy_probe(tsa, dev, stream, nbytes=2 << 30):
         torch.cuda.synchronize()
         best = max(best, 2 * a.numel() / (e0.elapsed_time(e1) * 1e-3) / 1e9)
     del a, b
+    return best
+
+
+def read_probe(tsa, dev, ws, stream, nbytes=2 << 30, reps=10):
+    """Read-only stream ceiling: tsa_hbm_read over 2 GiB (no stores), `reps`
+    launches back to back between two events, best of 3."""
+    a = torch.ones(nbytes, dtype=torch.uint8, device=dev)
+    tsa.hbm_read(a, a.numel(), ws, stream)
+    best = 0.0
+    for _ in range(3):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            tsa.hbm_read(a, a.numel(), ws, stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        best = max(best, reps * a.numel() / (e0.elapsed_time(e1) * 1e-3) / 1e9)
+    del a
     return best
 
 

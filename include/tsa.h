@@ -341,6 +341,13 @@ uint64_t tsa_launch_count(void);
  * and stores over a grid sized to the SM count.  bytes must be a multiple of 16. */
 tsa_status tsa_hbm_copy(const void* src, void* dst, size_t bytes, void* stream);
 
+/* HBM read probe: reads src[0:bytes] with the copy probe's 16-byte loads over a
+ * grid of 16 CTAs an SM, and stores nothing (a fold of the words lands in the workspace's flag block only
+ * for a value no buffer of repeated bytes gives).  Its bandwidth is the ceiling
+ * of a read-only stream, above the copy's.  src and bytes must be multiples of
+ * 16 bytes; ws >= 256 bytes (its first 8 bytes are the flag and that word). */
+tsa_status tsa_hbm_read(const void* src, size_t bytes, void* ws, size_t ws_bytes, void* stream);
+
 /* Random-row gather probe: fetch the 256-byte rows base[rows[i]*256 .. +256)
  * (rows[] on the device, nrows of them) into shared memory with bulk copies and
  * drop them.  Its bandwidth is the ceiling of a gather-bound stage (the

@@ -191,6 +191,15 @@ def test_hbm_copy_argument_errors(tsa):
     assert tsa.lib().tsa_hbm_copy(None, 0x2000, 16, None) == 1
 
 
+def test_hbm_read_argument_errors(tsa):
+    # rejected on the host, before any launch: size or pointer not 16-byte multiples, NULL, no workspace
+    assert tsa.lib().tsa_hbm_read(0x1000, 17, 0x100000, 256, None) == 1
+    assert tsa.lib().tsa_hbm_read(0x1008, 16, 0x100000, 256, None) == 1
+    assert tsa.lib().tsa_hbm_read(None, 16, 0x100000, 256, None) == 1
+    assert tsa.lib().tsa_hbm_read(0x1000, 16, None, 256, None) == 3
+    assert tsa.lib().tsa_hbm_read(0x1000, 16, 0x100000, 255, None) == 3
+
+
 def test_binding_raises_on_error(tsa):
     with pytest.raises(tsa.TsaError) as e:
         tsa.workspace_size(tsa.tsa_shape(1, 8, 2, 64, 96), 4, 1, tsa.SELECT)

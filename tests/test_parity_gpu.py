@@ -335,6 +335,19 @@ def test_attn_many_splits_workspace_combine(cuda_dev, dense):
     check_output(O.cpu().numpy(), ref, "many splits")
 
 
+def test_read_probe_runs_clean(cuda_dev):
+    """tsa_hbm_read streams a buffer and writes nothing: the workspace's flag and
+    fold words stay zero, and the buffer is unchanged."""
+    buf = torch.full((1 << 20,), 7, dtype=torch.uint8, device=cuda_dev)
+    ws = torch.zeros(256, dtype=torch.uint8, device=cuda_dev)
+    tsa.hbm_read(buf, buf.numel(), ws)
+    tsa.hbm_read(buf, 4096 + 16, ws)  # a size that leaves a ragged tail for the last loop
+    torch.cuda.synchronize()
+    assert int(ws[:8].sum()) == 0
+    assert bool((buf == 7).all())
+    tsa.check_device_status(ws)
+
+
 def test_gather_probe_runs_and_flags_bad_rows(cuda_dev):
     base = torch.zeros(1 << 20, dtype=torch.uint8, device=cuda_dev)  # 4096 rows of 256 B
     ws = torch.zeros(256, dtype=torch.uint8, device=cuda_dev)

@@ -68,6 +68,7 @@ _SIGS = {
     "tsa_last_error_string": (ctypes.c_char_p, []),
     "tsa_launch_count": (ctypes.c_uint64, []),
     "tsa_hbm_copy": (ctypes.c_int, [_vp, _vp, _sz, _vp]),
+    "tsa_hbm_read": (ctypes.c_int, [_vp, _sz, _vp, _sz, _vp]),
     "tsa_hbm_gather": (ctypes.c_int, [_vp, _sz, _vp, _i32, _vp, _sz, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -257,6 +258,10 @@ def launch_count() -> int:
 
 def hbm_copy(src, dst, nbytes: int, stream=None):
     _ok(_lib.tsa_hbm_copy(_ptr(src), _ptr(dst), nbytes, _stream(stream)))
+
+
+def hbm_read(src, nbytes: int, ws, stream=None):
+    _ok(_lib.tsa_hbm_read(_ptr(src), nbytes, *_wsargs(ws), _stream(stream)))
 
 
 def hbm_gather(base, rows, ws, stream=None):

@@ -611,6 +611,18 @@ tsa_status tsa_hbm_copy(const void* src, void* dst, size_t bytes, void* stream) 
     return TSA_OK;
 }
 
+tsa_status tsa_hbm_read(const void* src, size_t bytes, void* ws, size_t ws_bytes, void* stream) {
+    if (!src) return fail(TSA_ERR_INVALID_ARG, "tsa_hbm_read: NULL pointer");
+    if (!aligned16(src) || bytes % 16 != 0)
+        return fail(TSA_ERR_INVALID_ARG, "tsa_hbm_read: pointer and size must be multiples of 16 bytes");
+    TSA_TRY(check_ws(ws, ws_bytes, kFlagBytes));
+    // the fold's landing word: inside the flag block, past the flag itself
+    unsigned* sink = flag_of(ws) + 1;
+    cudaError_t e = tsa::launch_read(src, bytes, sink, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "tsa_hbm_read");
+    return TSA_OK;
+}
+
 tsa_status tsa_hbm_gather(const void* base, size_t base_bytes, const int32_t* rows, int32_t nrows, void* ws,
                           size_t ws_bytes, void* stream) {
     if (!base || (!rows && nrows > 0)) return fail(TSA_ERR_INVALID_ARG, "tsa_hbm_gather: NULL pointer");

@@ -2,6 +2,9 @@
 //  - copy: a plain 16-byte-vector device-to-device copy over a grid sized to the
 //    SM count; its bandwidth (read + write bytes / time) is the streaming peak
 //    the scan kernels are compared against in the same run.
+//  - read: the same loads with no stores; its bandwidth is the ceiling
+//    of a read-only stream (the scorer's scan of K reads and hardly writes),
+//    which a copy (half of its bytes written) understates;
 //  - gather: 256-byte rows at given row numbers, fetched by TMA bulk copies into
 //    shared memory and dropped; its bandwidth is the random-row ceiling the
 //    attention stage (which gathers the selected K/V rows) is compared against.
@@ -23,6 +26,23 @@ __global__ void __launch_bounds__(256) copy_kernel(const uint4* __restrict__ src
         dst[i + 3 * stride] = d;
     }
     for (; i < n16; i += stride) dst[i] = ld_stream(src + i);
+}
+
+// the loaded words are folded into one value, stored only when it equals a
+// value it cannot have for the probe's buffer of repeated bytes (so no load is
+// removed and nothing is written)
+__global__ void __launch_bounds__(256) read_kernel(const uint4* __restrict__ src, size_t n16,
+                                                   unsigned* __restrict__ sink) {
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    unsigned acc = 0u;
+    for (; i + 3 * stride < n16; i += 4 * stride) {
+        const uint4 a = ld_stream(src + i), b = ld_stream(src + i + stride);
+        const uint4 c = ld_stream(src + i + 2 * stride), d = ld_stream(src + i + 3 * stride);
+        acc += (a.x ^ a.w) + (b.x ^ b.w) + (c.x ^ c.w) + (d.x ^ d.w);
+    }
+    for (; i < n16; i += stride) acc += ld_stream(src + i).y;
+    if (acc == 0x9e3779b9u) *sink = acc;
 }
 
 constexpr int kGatherRowsPerCta = 256;  // a 64 KB shared-memory window per CTA
@@ -87,6 +107,19 @@ cudaError_t launch_gather(const void* base, size_t base_bytes, const int32_t* ro
     }
     gather_kernel<<<ceil_div(nrows, kGatherRowsPerCta), 128, kGatherRowsPerCta * 256, st>>>(
         static_cast<const unsigned char*>(base), base_bytes / 256, rows, nrows, flag);
+    note_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_read(const void* src, size_t bytes, unsigned* sink, cudaStream_t st) {
+    if (bytes == 0) return cudaSuccess;
+    int dev = 0, sms = 148;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    // 16 CTAs an SM (more requests in flight than the copy's 8; measured fastest)
+    read_kernel<<<sms * 16, 256, 0, st>>>(static_cast<const uint4*>(src), bytes / 16, sink);
     note_launch();
     return cudaGetLastError();
 }

@@ -114,6 +114,8 @@ cudaError_t launch_attn(const void* Q, const void* K, const void* V, const int32
                         uint32_t* hist_out = nullptr);  // with scores_out: adds the scores' top-digit histograms
 
 cudaError_t launch_copy(const void* src, void* dst, size_t bytes, cudaStream_t st);
+// reads src (16-byte loads, nothing stored unless a fold hits an impossible value: then *sink)
+cudaError_t launch_read(const void* src, size_t bytes, unsigned* sink, cudaStream_t st);
 cudaError_t launch_gather(const void* base, size_t base_bytes, const int32_t* rows, int nrows, unsigned* flag,
                           cudaStream_t st);
 
