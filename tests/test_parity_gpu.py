@@ -820,6 +820,66 @@ def test_sequence_sharded_select_on_one_gpu(cuda_dev, case):
         check_output(O_parts[r].cpu().numpy(), ref_r, f"{case} shard {r} part")
 
 
+@pytest.mark.parametrize("case", ["random", "all_equal", "heavy_ties", "k_edges", "one_shard", "past_cap"])
+def test_shard_merge_against_the_oracle(cuda_dev, case):
+    """tsa_shard_merge on candidate lists built here: the exact top-k of the
+    union of the shards' valid prefixes (ties to the lower row), against the
+    oracle's top-k over the union packed in row order.  Entries after a list's
+    first -1 hold junk that must be ignored.  "all_equal" takes the kernel's
+    no-pass branch (every key equal); "past_cap" (4 x 7000 candidates) the
+    pack / top-k / map path."""
+    rng = np.random.default_rng(len(case))
+    B, Hkv = 2, 2
+    R, k_max = {"one_shard": (1, 300), "past_cap": (4, 7000), "all_equal": (3, 200)}.get(case, (2, 300))
+    cnt = rng.integers(0, k_max + 1, size=(R, B))
+    cnt[0, 0] = k_max  # a full list (no -1 in it)
+    kreq = {"k_edges": [0, int(cnt[:, 1].sum())]}.get(case, [int(rng.integers(1, k_max + 1)), k_max + 50])
+    cs = np.full((R, B, Hkv, k_max), np.nan, dtype=np.float32)
+    cr = rng.integers(-50, 100000, size=(R, B, Hkv, k_max)).astype(np.int32)  # junk past the prefix
+    for r in range(R):
+        for b in range(B):
+            c = int(cnt[r, b])
+            for h in range(Hkv):
+                cr[r, b, h, :c] = np.sort(rng.choice(20000, size=c, replace=False)) + 20000 * r
+                if c < k_max:
+                    cr[r, b, h, c] = -1
+                if case == "all_equal":
+                    cs[r, b, h, :c] = 1.25
+                elif case == "heavy_ties":
+                    cs[r, b, h, :c] = rng.integers(-2, 3, size=c) * 0.5
+                else:
+                    cs[r, b, h, :c] = rng.standard_normal(c).astype(np.float32) + 2.0
+    # the oracle: top-k over the packed union, positions -> rows
+    n = cnt.sum(axis=0)
+    width = R * k_max
+    S_pack = np.zeros((B, Hkv, width))
+    rows_pack = np.full((B, Hkv, width), -1, dtype=np.int64)
+    for b in range(B):
+        for h in range(Hkv):
+            sc = np.concatenate([cs[r, b, h, :cnt[r, b]] for r in range(R)])
+            rw = np.concatenate([cr[r, b, h, :cnt[r, b]] for r in range(R)])
+            S_pack[b, h, :len(sc)] = sc.astype(np.float64)
+            rows_pack[b, h, :len(rw)] = rw
+    # k_b = min(k, n): above k_max the library takes k_max and raises the bounds flag
+    k_eff = [min(max(kreq[b], 0), int(n[b])) for b in range(B)]
+    flagged = any(k > k_max for k in k_eff)
+    pos = oracle.topk(S_pack, n.tolist(), [min(k, k_max) for k in k_eff], k_max)
+    want = np.where(pos >= 0, np.take_along_axis(rows_pack, np.maximum(pos, 0).astype(np.int64), axis=-1), -1)
+    shape = tsa.tsa_shape(B, Hkv * 4, Hkv, 20000 * R, 128)
+    ws = torch.zeros(tsa.shard_workspace_size(tsa.tsa_shape(B, Hkv * 4, Hkv, 20000, 128), k_max, R),
+                     dtype=torch.uint8, device=cuda_dev)
+    idx = torch.full((B, Hkv, k_max), -7, dtype=torch.int32, device=cuda_dev)
+    kr = torch.tensor(kreq, dtype=torch.int32, device=cuda_dev)
+    tsa.shard_merge(torch.from_numpy(cs).to(cuda_dev), torch.from_numpy(cr).to(cuda_dev), shape, kr, k_max, idx, ws)
+    got = idx.cpu().numpy()
+    np.testing.assert_array_equal(got, want.astype(np.int32))
+    if flagged:
+        with pytest.raises(tsa.TsaError):
+            tsa.check_device_status(ws)
+    else:
+        tsa.check_device_status(ws)
+
+
 def test_sequence_sharded_step_through_nccl(cuda_dev):
     """shard.sharded_select_step on a real NCCL process group (one rank on this
     GPU: every all-gather is a device NCCL collective, nothing waits on another
