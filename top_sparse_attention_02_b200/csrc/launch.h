@@ -12,7 +12,7 @@ constexpr unsigned kFlagBoundsBit = 1u;  // device flag: length / k / index out 
 constexpr unsigned kFlagTimeoutBit = 2u; // device flag: a bounded wait gave up
 
 struct Dims {
-    int B, Hq, Hkv, Ncap, G;  // G = Hq / Hkv
+    int B = 0, Hq = 0, Hkv = 0, Ncap = 0, G = 1;  // G = Hq / Hkv
     int units() const { return B * Hkv; }
 };
 
