@@ -439,6 +439,34 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
     }
     // Q's lines into L2 while the previous kernel finishes (G x 256 bytes)
     if (tid < 2 * G) prefetch_l2(Q + (size_t)unit * G * kD + tid * 64);
+    // The set-up below reads nothing the previous kernel writes, so it runs
+    // before the wait on it: out of the chain after the wait (barrier inits and
+    // their fence, a CTA barrier, the cluster arrive).
+    // Full attention handing on its top-k: a histogram of the emitted scores'
+    // top 11 key bits (the top-k's first radix digit), past the work area.
+    uint32_t* const s_hist = (CONTIG && sout && hout)
+        ? reinterpret_cast<uint32_t*>(smem + work + (CLUSTER ? Cfg::recv_bytes(S) : 0)) : nullptr;
+    const bool ccomb = CLUSTER && S > 1;  // the splits combine in this cluster (uniform)
+    if (s_hist)
+        for (int i = tid; i < kHistBins; i += kAttnThreads) s_hist[i] = 0u;
+    if (tid == 0) {
+        s_fail = 0;
+#pragma unroll
+        for (int i = 0; i < STAGES; ++i) mbar_init(&s_bar[i], CONTIG ? 1 : kTileRows);
+        if (ccomb) {
+            // every CTA of the cluster sends this CTA the slots of its partial
+            // that this CTA owns, and its (M, L) per head
+            const int per = ceil_div(G * 32, S);
+            const int own = max(0, min(per, G * 32 - s * per));
+            mbar_init(&s_rbar, 1);
+            mbar_arrive_expect_tx(&s_rbar, (unsigned)(S * (own * 16 + G * 8)));
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    __syncthreads();
+    // every CTA of the cluster has started and armed its receive barrier once
+    // this phase completes (waited for just before the first remote store)
+    if (ccomb) asm volatile("barrier.cluster.arrive.relaxed;\n" ::: "memory");
     if (early < 2) {
         griddep_wait();
         griddep_launch();
@@ -560,31 +588,6 @@ attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CU
             mbar_arrive(&s_bar[st]);
         }
     };
-    // full attention handing on its top-k: a histogram of the emitted scores'
-    // top 11 key bits (the top-k's first radix digit), past the work area
-    uint32_t* const s_hist = (CONTIG && sout && hout)
-        ? reinterpret_cast<uint32_t*>(smem + work + (CLUSTER ? Cfg::recv_bytes(S) : 0)) : nullptr;
-    const bool ccomb = CLUSTER && S > 1;  // the splits combine in this cluster (uniform)
-    if (s_hist)
-        for (int i = tid; i < kHistBins; i += kAttnThreads) s_hist[i] = 0u;
-    if (tid == 0) {
-        s_fail = 0;
-#pragma unroll
-        for (int i = 0; i < STAGES; ++i) mbar_init(&s_bar[i], CONTIG ? 1 : kTileRows);
-        if (ccomb) {
-            // every CTA of the cluster sends this CTA the slots of its partial
-            // that this CTA owns, and its (M, L) per head
-            const int per = ceil_div(G * 32, S);
-            const int own = max(0, min(per, G * 32 - s * per));
-            mbar_init(&s_rbar, 1);
-            mbar_arrive_expect_tx(&s_rbar, (unsigned)(S * (own * 16 + G * 8)));
-        }
-        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-    }
-    __syncthreads();
-    // every CTA of the cluster has started and armed its receive barrier once
-    // this phase completes (waited for just before the first remote store)
-    if (ccomb) asm volatile("barrier.cluster.arrive.relaxed;\n" ::: "memory");
     // CONTIG: the first STAGES tiles' block indices in one round, then their loads
     int next_first = -1;  // CONTIG, thread 0: first row of the tile that refills the stage next
     int issued = 0;       // CONTIG, thread 0: tiles whose loads have been issued
